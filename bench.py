@@ -1,0 +1,385 @@
+"""Benchmark: GPTQ single-layer quantization on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...      (N > 1)
+
+Workload (one "step" = the whole hot path over one layer): the Llama-7B
+attention projection W [4096, 4096] bf16, calibration X [262144, 4096] bf16
+in 16 batches of 16384 rows, 4-bit, groupsize 128, B = 128, percdamp 0.01:
+  widen W (bf16 -> fp32 working copy), zero H,
+  16 x gptq_hessian_accumulate, gptq_prepare_hinv, gptq_quantize_layer.
+Inputs are resident in HBM when the timed region starts; L2 is flushed
+(256 MiB write) before every step, outside the per-step events.
+
+Metric: quantized weights per second (whole job) and ms per layer.  Extra
+keys: per-stage ms, the roofline of the dominant kernel (the tcgen05 X^T X),
+the oracle's CPU time on a bounded sample, an end-to-end number through the
+public API with host buffers, the library's kernel launches, SM clocks.
+
+With N > 1 (torchrun, NCCL) every rank quantizes its own replica of the
+layer (the path has no exchange step): weak scaling, value = all ranks'
+weights / max-over-ranks time.
+
+`--impl reference` times the fp64 CPU oracle (the reference arm here) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GPTQ layer quantization weights/s & ms/layer (4096², n=262k); stage %roofline"
+WORKLOAD = ("attn4096: W [4096,4096] bf16 ~N(0,0.02^2), X [262144,4096] bf16 AR(1) rho=0.9 "
+            "in 16 batches of 16384, 4-bit, groupsize 128, B=128, percdamp 0.01")
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- the oracle (CPU) sample
+def cpu_sample(problem, x0, rows=64):
+    """Time the fp64 oracle on a bounded sample of the workload: one of the
+    16 calibration batches (x16), the full factorization, and the sweep on
+    `rows` of the 4096 rows (x 4096/rows).  Returns (seconds per layer
+    estimate, description, cores)."""
+    import oracle
+    from post_weight_quantization_05_b200 import synth
+    cores = len(os.sched_getaffinity(0))
+    xf = synth.x_as_f32(problem, x0)
+    t0 = time.perf_counter()
+    H = oracle.hessian([xf])
+    t_h = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    Hd, _ = oracle.damp(H, problem.percdamp)
+    U = oracle.hinv_upper_factor(Hd)
+    t_u = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.gptq_quantize(problem.W[:rows], U, problem.bits, problem.blocksize, problem.groupsize)
+    t_s = time.perf_counter() - t0
+    est = t_h * problem.n_batches + t_u + t_s * (problem.d_out / rows)
+    desc = (f"oracle fp64 on 1/{problem.n_batches} of the calibration rows (H, x{problem.n_batches}), "
+            f"full damp+factor chain, sweep on {rows}/{problem.d_out} rows (x{problem.d_out // rows}); "
+            f"measured {t_h:.1f}+{t_u:.1f}+{t_s:.1f} s")
+    return est, desc, cores
+
+
+def run_reference(args):
+    """--impl reference: the oracle on the host cores, same metric/config."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from post_weight_quantization_05_b200 import synth
+    p = synth.attn4096()
+    x0 = p.x_batch(0)
+    for _ in range(args.warmup):
+        pass   # the oracle has no warm-up state; the sample below is timed as is
+    ests = []
+    desc = cores = None
+    for _ in range(max(1, args.steps)):
+        est, desc, cores = cpu_sample(p, x0)
+        ests.append(est)
+    sec = statistics.mean(ests)
+    value = p.d_out * p.d_in / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": value, "unit": "weights/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from post_weight_quantization_05_b200 import api, build_lib, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    build_lib.build() if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    api.abi_version()
+
+    # ---- inputs (seeded, host), then resident in HBM
+    p = synth.attn4096()
+    t0 = time.time()
+    xs_host = synth.x_batches_threaded(p, min(16, os.cpu_count() or 8))
+    w_bits = synth.f32_to_bf16_bits(p.W)
+    gen_s = time.time() - t0
+    X_dev = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in xs_host]
+    W_dev = torch.from_numpy(w_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    lq = api.LayerQuantizer(p.d_out, p.d_in, p.bits, p.groupsize, p.blocksize, p.percdamp, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    n_ev = p.n_batches + 3
+    def step(evs):
+        evs[0].record(stream)
+        lq.begin(W_dev)
+        for b in range(p.n_batches):
+            evs[1 + b].record(stream)
+            lq.add_batch(X_dev[b])
+        evs[1 + p.n_batches].record(stream)
+        api.prepare_hinv(lq.H, lq.U, lq.ws_hinv, p.percdamp, lq.info)
+        evs[2 + p.n_batches].record(stream)
+        api.quantize_layer(lq.W, lq.U, p.bits, p.blocksize, p.groupsize, lq.codes, lq.scales, lq.zeros, lq.ws_q)
+
+    def new_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        evs = new_events()
+        step(evs)
+        evs[n_ev].record(stream)
+    api.get_status(stream)
+
+    clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = api.launch_count()
+    all_evs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        evs = new_events()
+        step(evs)
+        evs[n_ev].record(stream)
+        all_evs.append(evs)
+    torch.cuda.synchronize(dev)
+    launches = api.launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    api.get_status(stream)
+
+    step_ms = [e[0].elapsed_time(e[n_ev]) for e in all_evs]
+    h_ms = [e[1].elapsed_time(e[1 + p.n_batches]) for e in all_evs]
+    h_launch_ms = [e[1 + b].elapsed_time(e[2 + b]) for e in all_evs for b in range(p.n_batches)]
+    prep_ms = [e[1 + p.n_batches].elapsed_time(e[2 + p.n_batches]) for e in all_evs]
+    quant_ms = [e[2 + p.n_batches].elapsed_time(e[n_ev]) for e in all_evs]
+    begin_ms = [e[0].elapsed_time(e[1]) for e in all_evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    weights = p.d_out * p.d_in * world * args.steps
+    value = weights / (total_ms / 1e3)
+
+    # roofline of the dominant kernel: the X^T X launch (one per batch)
+    burst, sustained, hbm, src = peaks()
+    n_b = p.batch_rows
+    flops_per_launch = n_b * p.d_in * (p.d_in + 1)       # upper triangle incl. diagonal, 2 flops per MAC
+    h_launch_avg = statistics.mean(h_launch_ms)
+    achieved = flops_per_launch / (h_launch_avg / 1e3) / 1e12
+    roof = {"kernel": "hessian syrk_kernel (tcgen05)", "bound": "tensor", "achieved": achieved,
+            "peak": sustained, "unit": "TFLOP/s", "frac": achieved / sustained,
+            "peak_kind": f"bf16 dense sustained ({src})", "traffic": None,
+            "algorithmic_per_launch": f"{flops_per_launch:.4e} flop ({n_b}x{p.d_in}x{p.d_in + 1})",
+            "avg_launch_ms": h_launch_avg}
+
+    stages = {"widen_W+zero_H": statistics.mean(begin_ms), "hessian_16_batches": statistics.mean(h_ms),
+              "prepare_hinv": statistics.mean(prep_ms), "quantize_layer": statistics.mean(quant_ms)}
+
+    # ---- end to end through the public API with host buffers (rank 0 .. all ranks)
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(p, xs_host, w_bits, lq, dev, args, world, dist if world > 1 else None)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        est, desc, cores = cpu_sample(p, xs_host[0])
+        cpu = {"value": p.d_out * p.d_in / est, "unit": "weights/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp32", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "d_out": p.d_out, "d_in": p.d_in, "n": p.n,
+                           "batches": p.n_batches, "bits": p.bits, "groupsize": p.groupsize,
+                           "blocksize": p.blocksize, "parallelism": f"replicas x{world}",
+                           "l2": "flushed before every step (256 MiB write, outside the step events)"},
+                "ms_per_layer": ms_per_step, "stages_ms": stages, "roofline": roof, "cpu_baseline": cpu,
+                "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+                "input_generation_s": gen_s}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def end_to_end(p, xs_host, w_bits, lq, dev, args, world, dist):
+    """Same metric through the public API, inputs in pinned host memory:
+    every step copies W and the 16 X batches host -> device (copy stream,
+    double-buffered, overlapped with the Hessian kernels) and reads the
+    packed codes, scales and zeros back."""
+    import torch
+
+    from post_weight_quantization_05_b200 import api
+    pin_x = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_host]
+    pin_w = torch.from_numpy(w_bits.view(np.int16)).pin_memory()
+    out_codes = torch.empty(lq.codes.shape, dtype=lq.codes.dtype).pin_memory()
+    out_s = torch.empty(lq.scales.shape, dtype=lq.scales.dtype).pin_memory()
+    out_z = torch.empty(lq.zeros.shape, dtype=lq.zeros.dtype).pin_memory()
+    slots = [torch.empty(xs_host[0].shape, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    w_dev = torch.empty(w_bits.shape, dtype=torch.bfloat16, device=dev)
+    comp = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(device=dev)
+    h2d = pin_w.numel() * 2 + sum(x.numel() * 2 for x in pin_x)
+    d2h = out_codes.numel() * 4 + out_s.numel() * 2 + out_z.numel() * 2
+
+    def one_step():
+        freed = [torch.cuda.Event() for _ in range(2)]
+        for e in freed:
+            e.record(comp)
+        with torch.cuda.stream(copy):
+            w_dev.copy_(pin_w.view(torch.bfloat16), non_blocking=True)
+            wready = torch.cuda.Event()
+            wready.record(copy)
+        comp.wait_event(wready)
+        lq.begin(w_dev)
+        for b, px in enumerate(pin_x):
+            s = b % 2
+            copy.wait_event(freed[s])
+            with torch.cuda.stream(copy):
+                slots[s].copy_(px.view(torch.bfloat16), non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(copy)
+            comp.wait_event(ready)
+            lq.add_batch(slots[s])
+            freed[s] = torch.cuda.Event()
+            freed[s].record(comp)
+        lq.finish()
+        out_codes.copy_(lq.codes, non_blocking=True)
+        out_s.copy_(lq.scales, non_blocking=True)
+        out_z.copy_(lq.zeros, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        one_step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    steps = max(1, min(args.steps, 3))
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(comp)
+    copy.wait_event(start)          # host->device copies count from `start` too
+    for _ in range(steps):
+        one_step()
+    end.record(comp)
+    torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(end)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    api.get_status(comp)
+    return {"value": p.d_out * p.d_in * world * steps / (ms / 1e3), "unit": "weights/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps, "steps": steps}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,189 @@
+/*
+ * gptq.h -- C ABI of libgptq.so, a B200 (sm_100a) implementation of GPTQ
+ * single-layer post-training weight quantization.
+ *
+ * The method (itwiki "GPTQ" article, sections "문제 설정", "OBQ에서 GPTQ로",
+ * "알고리즘" and "실무 변형"; blog "GPTQ를 밑바닥부터 구현하며 배운 것들",
+ * section 3): given a linear layer's weights W [d_out, d_in] and its
+ * calibration inputs X [n, d_in], find W^ on a low-bit grid that keeps
+ * ||W X^T - W^ X^T||^2 small.  Four stream-ordered stages:
+ *
+ *   gptq_hessian_accumulate   H += 2 X^T X            (per calibration batch)
+ *   gptq_prepare_hinv         U = upper Cholesky factor of (H + lambda I)^-1
+ *   gptq_quantize_layer       blocked column sweep + lazy trailing updates
+ *                             + packing of the codes
+ *   gptq_rtn_layer            round-to-nearest on the same grid (baseline)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer named *_dev / W / X / H / U / codes / scales / zeros / Q / ws
+ *    is DEVICE memory owned by the caller.  The library never allocates or
+ *    frees device memory.  Host-side validation happens before any CUDA call:
+ *    an invalid argument returns an error code and launches nothing.
+ *  - Matrices are dense, row-major, with no padding (row stride = columns).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work; they return before it runs.
+ *  - Errors found on the device (a non-positive pivot, non-finite values, a
+ *    wait that ran out of time) are recorded in a per-device status word;
+ *    gptq_get_status() synchronizes the stream, returns it and clears it.
+ *    No kernel traps, asserts or waits without a bound.
+ *  - Sizes: d_in must be a multiple of 128 and at most 32768; d_out >= 1;
+ *    pointers to float / uint32 data must be 16-byte aligned.
+ *  - Calls on different streams may run concurrently if they touch
+ *    different buffers and workspaces; the status word is shared.
+ */
+#ifndef GPTQ_H
+#define GPTQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GPTQ_OK = 0,
+    GPTQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or workspace  */
+    GPTQ_ERR_UNSUPPORTED = 2,   /* valid for the method, not for this build   */
+    GPTQ_ERR_NOT_PD = 3,        /* damped H not positive definite             */
+    GPTQ_ERR_NONFINITE = 4,     /* NaN/Inf met in H, U, W or the grid         */
+    GPTQ_ERR_GRID = 5,          /* grid not representable in fp16             */
+    GPTQ_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up         */
+    GPTQ_ERR_CUDA = 7           /* a CUDA runtime call failed                 */
+} gptq_status;
+
+typedef enum { GPTQ_F32 = 0, GPTQ_BF16 = 1 } gptq_dtype;
+
+/* Version of this ABI (bumped on any incompatible change). */
+int gptq_abi_version(void);
+
+/* Number of kernels this library has enqueued in this process so far (all
+ * devices and streams).  A diagnostic: the difference across a region of
+ * code is how many of this library's kernels that region launched. */
+uint64_t gptq_launch_count(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gptq_status_string(int status);
+
+/* ------------------------------------------------------------------------
+ * Stage 1 -- Hessian accumulation.
+ * Source: blog "GPTQ를 밑바닥부터 구현하며 배운 것들", section 3 (H = 2 X^T X
+ * from the inputs captured at each linear layer); itwiki "GPTQ",
+ * "최소 구현" (H = 2 X^T X, X laid out [n, d_in]) and its closing paragraph
+ * (H accumulated per layer over the calibration data).
+ *
+ * H[a][b] += 2 * sum_r X[r][a] * X[r][b]   for all 0 <= a <= b < d_in.
+ *
+ *   X      device, [n, d_in] row-major, bf16 (xdt = GPTQ_BF16) or fp32
+ *          (xdt = GPTQ_F32), 16-byte aligned.  n may be 0 (no-op).
+ *   H      device, [d_in, d_in] fp32, 16-byte aligned.  Caller zeroes it
+ *          before the first batch (gptq_fill_f32) and calls this once per
+ *          batch.  The upper triangle (b >= a) is the result; entries below
+ *          the diagonal may be written with their (symmetric) values inside
+ *          tiles that straddle the diagonal and are otherwise left untouched.
+ *   ws     device workspace of at least gptq_hessian_workspace_size(xdt, n,
+ *          d_in) bytes (0 for bf16: ws may be NULL).  fp32 inputs are split
+ *          into three bf16 terms there.
+ * Products run on the tensor cores: bf16 x bf16 with fp32 accumulation
+ * (exact products); fp32 X is split x = h + m + l into bf16 terms and the six
+ * leading cross products are accumulated (about fp32 accuracy).
+ * ---------------------------------------------------------------------- */
+size_t gptq_hessian_workspace_size(int dtype, int64_t n, int64_t d_in);
+int gptq_hessian_accumulate(const void* X, int dtype, int64_t n, int64_t d_in,
+                            float* H, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 2 -- dampening and the upper Cholesky factor of the inverse.
+ * Source: itwiki "GPTQ", "GPTQ의 세 가지 변경" row 3 (add 1% of the mean
+ * diagonal; only the Cholesky form of H^-1 is needed, computed once up
+ * front); "알고리즘" (H^-1 <- Cholesky(H^-1)^T); "최소 구현" (chol ->
+ * cholesky_inverse -> chol(upper)).
+ *
+ * lambda = percdamp * mean(diag H);  U upper triangular with
+ * U^T U = (H + lambda I)^-1.  Computed as U = P L'^-1 P with P the index
+ * reversal and L' = chol(P (H + lambda I) P) -- the same U as the pages'
+ * chain by uniqueness of the Cholesky factor -- in fp32.
+ *
+ *   H        device [d_in, d_in] fp32; only the upper triangle is read; not
+ *            modified.
+ *   U        device [d_in, d_in] fp32 output; the strict lower triangle is
+ *            set to 0.  On failure U is filled with NaN.
+ *   info_dev device int32 (may be NULL): 0 on success, else k+1 where k is
+ *            the step (0-based, in the order the factorization visits the
+ *            columns of H: last column first) whose pivot was not positive
+ *            and finite.  The status word gets GPTQ_ERR_NOT_PD (or
+ *            GPTQ_ERR_NONFINITE for a NaN/Inf pivot).
+ *   ws       >= gptq_prepare_hinv_workspace_size(d_in) bytes.
+ * ---------------------------------------------------------------------- */
+size_t gptq_prepare_hinv_workspace_size(int64_t d_in);
+int gptq_prepare_hinv(const float* H, int64_t d_in, float percdamp, float* U,
+                      int* info_dev, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Stages 3-5 -- the blocked column sweep with lazy trailing updates and the
+ * packed output.
+ * Source: itwiki "GPTQ", "알고리즘" (Algorithm 1), "GPTQ의 세 가지 변경" rows
+ * 1-2 (one column order for all rows; updates inside a block of B columns,
+ * then one matrix product for the rest), "최소 구현" (per-row asymmetric
+ * min/max grid), "실무 변형" (group quantization, grid from the latest
+ * updated weights); blog, section 5 (store integer codes, not fp32).
+ *
+ * For each block i = 0, B, 2B, ... and each column j of the block:
+ *   c = clamp(rint(w_j / s) + z, 0, maxq);  q = s (c - z);
+ *   E[:, j-i] = (w_j - q) / U[j][j];  W[:, j:i+B] -= E[:, j-i] U[j, j:i+B];
+ * then W[:, i+B:] -= E U[i:i+B, i+B:].
+ * Grid: s32 = max(wmax - wmin, 1e-8) / maxq (fp32), s = fp16(s32) (2^-14 if
+ * that rounds to 0), z = fp16(rint(-wmin / s)); per row from the original W
+ * (groupsize = -1), or per group of `groupsize` columns from the current W
+ * when the sweep reaches the group's first column.
+ *
+ *   W        device [d_out, d_in] fp32 working copy, OVERWRITTEN (holds the
+ *            partially updated weights afterwards; not a result).
+ *   U        device [d_in, d_in] fp32 from gptq_prepare_hinv (upper read).
+ *   bits     2, 3, 4 or 8 (maxq = 2^bits - 1).
+ *   blocksize must be 128.
+ *   groupsize -1 (one grid per row) or a multiple of 128 dividing d_in.
+ *   codes    device uint32 [d_out, d_in * bits / 32]: per row a little-endian
+ *            bit stream, code k in stream bits [k*bits, (k+1)*bits).
+ *   scales, zeros  device fp16 bit patterns (uint16) [d_out, n_groups],
+ *            n_groups = 1 or d_in / groupsize.
+ *   Q        device [d_out, d_in] fp32 dequantized weights, or NULL.
+ *   ws       >= gptq_quantize_workspace_size(d_out, d_in, blocksize) bytes.
+ * ---------------------------------------------------------------------- */
+size_t gptq_quantize_workspace_size(int64_t d_out, int64_t d_in, int blocksize);
+int gptq_quantize_layer(float* W, int64_t d_out, int64_t d_in, const float* U,
+                        int bits, int blocksize, int groupsize,
+                        uint32_t* codes, uint16_t* scales, uint16_t* zeros,
+                        float* Q, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Baseline -- round to nearest on the same grid, no compensation.
+ * Source: itwiki "GPTQ", "문제 설정" (RTN moves each weight to its nearest
+ * grid point without looking at the inputs).  Group grids come from the
+ * original W.  Arguments as for gptq_quantize_layer; W is not modified.
+ * ---------------------------------------------------------------------- */
+int gptq_rtn_layer(const float* W, int64_t d_out, int64_t d_in, int bits, int groupsize,
+                   uint32_t* codes, uint16_t* scales, uint16_t* zeros, float* Q,
+                   void* stream);
+
+/* ------------------------------------------------------------------------
+ * Helpers on the same stream (not steps of the method).
+ * ---------------------------------------------------------------------- */
+/* dst[i] = (float) src[i] for bf16 bit patterns src (a bf16 layer's fp32
+ * working copy). src 16-byte aligned is not required; dst is. */
+int gptq_widen_bf16(const uint16_t* src, float* dst, int64_t count, void* stream);
+/* p[i] = value for i < count (zeroing H before the first batch). */
+int gptq_fill_f32(float* p, int64_t count, float value, void* stream);
+
+/* Synchronizes `stream`, returns the first device-side error recorded since
+ * the last call (GPTQ_OK if none) and clears it.  *detail_out (may be NULL)
+ * receives a code-specific detail (a row or pivot index).  Returns
+ * GPTQ_ERR_CUDA if the synchronization itself failed. */
+int gptq_get_status(void* stream, int* detail_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_H */

@@ -1,0 +1,48 @@
+// Host-side launchers shared between the translation units of libgptq.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace gptq {
+
+struct DevStatus;
+
+// Host-side count of kernels enqueued by this library (gptq_launch_count).
+void count_launch();
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// hessian.cu
+int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, void* ws, cudaStream_t stream,
+                   DevStatus* st, PFN_encodeTiled encode);
+
+// gemm.cu: C[M,N] = alpha * A[M,K] * op(B)[K,N] + beta * C, fp32, row-major.
+// trans_b = false: B(k, n) = B[k * ldb + n];  true: B(k, n) = B[n * ldb + k].
+// lower_only: skip 128x128 output tiles whose rows all lie above the diagonal
+// (tile entirely in the strict upper triangle: n0 > m0 + 127).
+// C_out may differ from C_in (beta applies to C_in); they may also alias.
+int launch_sgemm(int M, int N, int K, float alpha, const float* A, int lda, const float* B, int ldb, bool trans_b,
+                 float beta, const float* C_in, float* C_out, int ldc, bool lower_only, cudaStream_t stream);
+
+// factor.cu
+size_t factor_workspace_bytes(int64_t d);
+int launch_prepare_hinv(const float* H, int64_t d, float percdamp, float* U, int* info, void* ws,
+                        cudaStream_t stream, DevStatus* st);
+
+// sweep.cu
+size_t sweep_workspace_bytes(int64_t d_out, int64_t d_in);
+int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int bits, int groupsize,
+                    uint32_t* codes, uint16_t* scales, uint16_t* zeros, float* Q, void* ws, cudaStream_t stream,
+                    DevStatus* st);
+int launch_rtn(const float* W, int64_t d_out, int64_t d_in, int bits, int groupsize, uint32_t* codes,
+               uint16_t* scales, uint16_t* zeros, float* Q, cudaStream_t stream, DevStatus* st);
+int launch_widen_bf16(const uint16_t* src, float* dst, int64_t count, cudaStream_t stream);
+int launch_fill(float* p, int64_t count, float value, cudaStream_t stream);
+
+}  // namespace gptq

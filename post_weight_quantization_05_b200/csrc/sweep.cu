@@ -1,0 +1,365 @@
+// Stages 3-5: the blocked column sweep, the lazy trailing update and the
+// packed codes; plus the round-to-nearest baseline.
+//
+// Source: itwiki "GPTQ", "알고리즘" (Algorithm 1), "GPTQ의 세 가지 변경"
+// rows 1-2 (shared column order; updates inside a block of B = 128 columns,
+// one matrix product for the columns after it), "최소 구현" (per-row
+// asymmetric min/max grid, q = clamp(round(w/s) + z, 0, maxq)), "실무 변형"
+// (groups share a grid set from the latest updated weights); "문제 설정" (RTN).
+//
+// Sweep kernel design: rows are independent given U (the same U serves every
+// row), so one thread owns one row of the 128-column block: the block's 128
+// weights live in registers, the 128 x 128 diagonal block of U in shared
+// memory (every thread of a warp reads the same U element: broadcast).  The
+// block is walked in four 32-column sub-blocks: inside a sub-block the column
+// loop is unrolled (static register indices); the sub-block's E values are
+// then applied to the later sub-blocks in a rolled loop that reads E back from
+// shared memory -- the same additions in the same order as the plain rank-1
+// sweep, with a quarter of the code.  After column j is quantized its
+// register slot holds E[:, j], and the block's E is written once for the
+// trailing SGEMM.  The codes are packed in registers
+// (compile-time bit positions) and stored as 16-byte vectors.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gptq {
+namespace sweep {
+
+constexpr int B = 128;
+constexpr int ROWS = 32;  // rows (threads) per CTA
+constexpr size_t SMEM = (size_t(B) * B + size_t(ROWS) * 33) * sizeof(float);
+
+// Per-row grid over columns [c0, c0 + len) of the ORIGINAL W: one warp per
+// (row, group).  Writes fp16 scale/zero bit patterns.
+__global__ void grid_kernel(const float* __restrict__ W, int d_out, int d_in, int group, int n_groups, float maxq,
+                            uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, DevStatus* st) {
+    const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int r = warp_global / n_groups, g = warp_global % n_groups;
+    if (r >= d_out) return;
+    const float* row = W + size_t(r) * d_in + size_t(g) * group;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int c = lane * 4; c < group; c += 128) {
+        const float4 v = *reinterpret_cast<const float4*>(row + c);
+        mn = fminf(fminf(mn, v.x), fminf(v.y, fminf(v.z, v.w)));
+        mx = fmaxf(fmaxf(mx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+        float s, z;
+        __half s16, z16;
+        if (!grid_params(mn, mx, maxq, s, z, s16, z16)) record_error(st, GPTQ_ERR_NONFINITE, r);
+        scales[size_t(r) * n_groups + g] = __half_as_ushort(s16);
+        zeros[size_t(r) * n_groups + g] = __half_as_ushort(z16);
+    }
+}
+
+// Bit-stream packer with compile-time positions: code k of the block goes to
+// stream bits [k*BITS, (k+1)*BITS).
+template <int BITS>
+struct Packer {
+    static constexpr int WORDS = B * BITS / 32;
+    uint32_t w[WORDS];
+    __device__ __forceinline__ Packer() {
+#pragma unroll
+        for (int i = 0; i < WORDS; ++i) w[i] = 0u;
+    }
+    template <int K>
+    __device__ __forceinline__ void put(uint32_t c) {
+        constexpr int pos = K * BITS, word = pos / 32, off = pos % 32;
+        w[word] |= c << off;
+        if constexpr (off + BITS > 32) w[word + 1] |= c >> (32 - off);
+    }
+    __device__ __forceinline__ void store(uint32_t* dst) const {
+#pragma unroll
+        for (int i = 0; i < WORDS; i += 4)
+            *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+    }
+};
+
+// Column J of the block: quantize, record code and E, and apply the rank-1
+// correction to the remaining columns of J's 32-column sub-block.
+template <int BITS, int J>
+__device__ __forceinline__ void quant_column(float (&w)[B], const float* __restrict__ Us, float* __restrict__ Erow,
+                                             float s, float z, float maxq, Packer<BITS>& pk, float* Qrow,
+                                             bool& finite) {
+    constexpr int SUB_END = (J / 32 + 1) * 32;
+    const float wj = w[J];
+    const float c = quant_code(wj, s, z, maxq);
+    const float q = s * (c - z);
+    const float e = __fdiv_rn(wj - q, Us[J * B + J]);
+    finite &= isfinite(e);
+    if (Qrow) Qrow[J] = q;
+    pk.template put<J>(static_cast<uint32_t>(c));
+    const float* urow = Us + J * B;
+#pragma unroll
+    for (int k = J + 1; k < SUB_END; ++k) w[k] = fmaf(-e, urow[k], w[k]);
+    w[J] = e;
+    Erow[J % 32] = e;
+}
+
+template <int BITS, int SB, int J>
+struct SubCols {
+    __device__ __forceinline__ static void run(float (&w)[B], const float* Us, float* Erow, float s, float z,
+                                               float maxq, Packer<BITS>& pk, float* Qrow, bool& finite) {
+        quant_column<BITS, SB * 32 + J>(w, Us, Erow, s, z, maxq, pk, Qrow, finite);
+        if constexpr (J + 1 < 32) SubCols<BITS, SB, J + 1>::run(w, Us, Erow, s, z, maxq, pk, Qrow, finite);
+    }
+};
+
+// Updates of sub-block SB's 32 columns to the later sub-block SBK, in column
+// order j = 0..31 (the same order in which the plain rank-1 sweep applies
+// them), with E read back from shared memory so that j can be a loop index.
+template <int SB, int SBK>
+__device__ __forceinline__ void cross_update(float (&w)[B], const float* __restrict__ Us,
+                                             const float* __restrict__ Erow) {
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) {
+        const float e = Erow[j];
+        const float* urow = Us + (SB * 32 + j) * B + SBK * 32;
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+            const float4 u = *reinterpret_cast<const float4*>(urow + k);
+            w[SBK * 32 + k + 0] = fmaf(-e, u.x, w[SBK * 32 + k + 0]);
+            w[SBK * 32 + k + 1] = fmaf(-e, u.y, w[SBK * 32 + k + 1]);
+            w[SBK * 32 + k + 2] = fmaf(-e, u.z, w[SBK * 32 + k + 2]);
+            w[SBK * 32 + k + 3] = fmaf(-e, u.w, w[SBK * 32 + k + 3]);
+        }
+    }
+}
+
+template <int BITS, int SB>
+__device__ __forceinline__ void sub_block(float (&w)[B], const float* Us, float* Erow, float s, float z, float maxq,
+                                          Packer<BITS>& pk, float* Qrow, bool& finite) {
+    // Erow is private to this thread: no synchronization needed around it.
+    SubCols<BITS, SB, 0>::run(w, Us, Erow, s, z, maxq, pk, Qrow, finite);
+    if constexpr (SB < 1) cross_update<SB, 1>(w, Us, Erow);
+    if constexpr (SB < 2) cross_update<SB, 2>(w, Us, Erow);
+    if constexpr (SB < 3) cross_update<SB, 3>(w, Us, Erow);
+    if constexpr (SB + 1 < B / 32) sub_block<BITS, SB + 1>(w, Us, Erow, s, z, maxq, pk, Qrow, finite);
+}
+
+struct SweepArgs {
+    float* W;
+    const float* U;
+    int d_out, d_in, groupsize, n_groups;
+    float maxq;
+    uint32_t* codes;
+    uint16_t* scales;
+    uint16_t* zeros;
+    float* Q;
+    float* E;  // [d_out, B]
+    DevStatus* st;
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(ROWS) sweep_block_kernel(const SweepArgs a, int i0) {
+    extern __shared__ float Us[];  // U[i0:i0+B, i0:i0+B], row-major, then E of one sub-block per thread
+    float* Erow = Us + B * B + threadIdx.x * 33;   // stride 33: conflict-free per-thread rows
+    const float* ub = a.U + size_t(i0) * a.d_in + i0;
+    for (int idx = threadIdx.x * 4; idx < B * B; idx += ROWS * 4) {
+        const int r = idx / B, c = idx % B;
+        *reinterpret_cast<float4*>(Us + idx) = *reinterpret_cast<const float4*>(ub + size_t(r) * a.d_in + c);
+    }
+    __syncthreads();
+    const int r = blockIdx.x * ROWS + threadIdx.x;
+    if (r >= a.d_out) return;
+
+    float w[B];
+    float* wrow = a.W + size_t(r) * a.d_in + i0;
+#pragma unroll
+    for (int k = 0; k < B; k += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(wrow + k);
+        w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
+    }
+
+    float s, z;
+    bool finite = true;
+    if (a.groupsize < 0) {
+        s = __half2float(__ushort_as_half(a.scales[r]));
+        z = __half2float(__ushort_as_half(a.zeros[r]));
+    } else {
+        const int g = i0 / a.groupsize;
+        const size_t gi = size_t(r) * a.n_groups + g;
+        if (i0 % a.groupsize == 0) {
+            // grid from the current weights of the group (this block's columns
+            // from registers, later columns from W, already lazily updated)
+            float mn = w[0], mx = w[0];
+#pragma unroll
+            for (int k = 1; k < B; ++k) { mn = fminf(mn, w[k]); mx = fmaxf(mx, w[k]); }
+            for (int c = B; c < a.groupsize; c += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(wrow + c);
+                mn = fminf(fminf(mn, v.x), fminf(v.y, fminf(v.z, v.w)));
+                mx = fmaxf(fmaxf(mx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
+            }
+            __half s16, z16;
+            finite &= grid_params(mn, mx, a.maxq, s, z, s16, z16);
+            a.scales[gi] = __half_as_ushort(s16);
+            a.zeros[gi] = __half_as_ushort(z16);
+        } else {
+            s = __half2float(__ushort_as_half(a.scales[gi]));
+            z = __half2float(__ushort_as_half(a.zeros[gi]));
+        }
+    }
+
+    Packer<BITS> pk;
+    float* Qrow = a.Q ? a.Q + size_t(r) * a.d_in + i0 : nullptr;
+    sub_block<BITS, 0>(w, Us, Erow, s, z, a.maxq, pk, Qrow, finite);
+    if (!finite) record_error(a.st, GPTQ_ERR_NONFINITE, r);
+
+    pk.store(a.codes + size_t(r) * (size_t(a.d_in) * BITS / 32) + size_t(i0) * BITS / 32);
+    float* erow = a.E + size_t(r) * B;
+#pragma unroll
+    for (int k = 0; k < B; k += 4) *reinterpret_cast<float4*>(erow + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+}
+
+// RTN: one thread per 32 consecutive codes of a row (one packing unit for
+// every supported width); grid from the original W (grid_kernel).
+template <int BITS>
+__global__ void rtn_kernel(const float* __restrict__ W, int d_out, int d_in, int group, int n_groups, float maxq,
+                           const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
+                           uint32_t* __restrict__ codes, float* __restrict__ Q) {
+    const int units = d_in / 32;
+    const size_t t = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t >= size_t(d_out) * units) return;
+    const int r = int(t / units), u = int(t % units);
+    const int c0 = u * 32;
+    const size_t gi = size_t(r) * n_groups + c0 / group;
+    const float s = __half2float(__ushort_as_half(scales[gi]));
+    const float z = __half2float(__ushort_as_half(zeros[gi]));
+    const float* src = W + size_t(r) * d_in + c0;
+    uint32_t words[BITS] = {};
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src + k);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t c = static_cast<uint32_t>(quant_code(vv[i], s, z, maxq));
+            const int pos = (k + i) * BITS, word = pos / 32, off = pos % 32;
+            words[word] |= c << off;
+            if (off + BITS > 32) words[word + 1] |= c >> (32 - off);
+            if (Q) Q[size_t(r) * d_in + c0 + k + i] = s * (float(c) - z);
+        }
+    }
+    uint32_t* dst = codes + size_t(r) * (size_t(d_in) * BITS / 32) + size_t(u) * BITS;
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) dst[i] = words[i];
+}
+
+__global__ void widen_bf16_kernel(const uint16_t* __restrict__ src, float* __restrict__ dst, size_t n) {
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x)
+        dst[i] = __uint_as_float(uint32_t(src[i]) << 16);
+}
+
+__global__ void fill_kernel(float* __restrict__ p, size_t n, float v) {
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x)
+        p[i] = v;
+}
+
+template <int BITS>
+int run_sweep(const SweepArgs& a, cudaStream_t stream) {
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(sweep_block_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM)) !=
+            cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    const int blocks = (a.d_out + ROWS - 1) / ROWS;
+    for (int i0 = 0; i0 < a.d_in; i0 += B) {
+        sweep_block_kernel<BITS><<<blocks, ROWS, SMEM, stream>>>(a, i0); count_launch();
+        const int tail = a.d_in - i0 - B;
+        if (tail > 0) {
+            // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]
+            float* c = a.W + i0 + B;
+            const int rc = launch_sgemm(a.d_out, tail, B, -1.0f, a.E, B, a.U + size_t(i0) * a.d_in + i0 + B, a.d_in,
+                                        false, 1.0f, c, c, a.d_in, false, stream);
+            if (rc) return rc;
+        }
+    }
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+}  // namespace sweep
+
+size_t sweep_workspace_bytes(int64_t d_out, int64_t d_in) {
+    (void)d_in;
+    return size_t(d_out) * sweep::B * sizeof(float);
+}
+
+int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int bits, int groupsize,
+                    uint32_t* codes, uint16_t* scales, uint16_t* zeros, float* Q, void* ws, cudaStream_t stream,
+                    DevStatus* st) {
+    using namespace sweep;
+    SweepArgs a;
+    a.W = W;
+    a.U = U;
+    a.d_out = int(d_out);
+    a.d_in = int(d_in);
+    a.groupsize = groupsize;
+    a.n_groups = groupsize > 0 ? int(d_in / groupsize) : 1;
+    a.maxq = float((1 << bits) - 1);
+    a.codes = codes;
+    a.scales = scales;
+    a.zeros = zeros;
+    a.Q = Q;
+    a.E = static_cast<float*>(ws);
+    a.st = st;
+    if (groupsize < 0) {
+        const int warps = a.d_out;
+        grid_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(W, a.d_out, a.d_in, a.d_in, 1, a.maxq, scales,
+                                                                  zeros, st); count_launch();
+    }
+    switch (bits) {
+        case 2: return run_sweep<2>(a, stream);
+        case 3: return run_sweep<3>(a, stream);
+        case 4: return run_sweep<4>(a, stream);
+        case 8: return run_sweep<8>(a, stream);
+        default: return GPTQ_ERR_UNSUPPORTED;
+    }
+}
+
+int launch_rtn(const float* W, int64_t d_out, int64_t d_in, int bits, int groupsize, uint32_t* codes,
+               uint16_t* scales, uint16_t* zeros, float* Q, cudaStream_t stream, DevStatus* st) {
+    using namespace sweep;
+    const int group = groupsize > 0 ? groupsize : int(d_in);
+    const int n_groups = int(d_in / group);
+    const float maxq = float((1 << bits) - 1);
+    const int64_t warps = d_out * n_groups;
+    grid_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, stream>>>(W, int(d_out), int(d_in), group, n_groups,
+                                                                         maxq, scales, zeros, st); count_launch();
+    const int64_t units = d_out * (d_in / 32);
+    const unsigned blocks = unsigned((units + 255) / 256);
+    switch (bits) {
+        case 2: rtn_kernel<2><<<blocks, 256, 0, stream>>>(W, int(d_out), int(d_in), group, n_groups, maxq, scales, zeros, codes, Q); count_launch(); break;
+        case 3: rtn_kernel<3><<<blocks, 256, 0, stream>>>(W, int(d_out), int(d_in), group, n_groups, maxq, scales, zeros, codes, Q); count_launch(); break;
+        case 4: rtn_kernel<4><<<blocks, 256, 0, stream>>>(W, int(d_out), int(d_in), group, n_groups, maxq, scales, zeros, codes, Q); count_launch(); break;
+        case 8: rtn_kernel<8><<<blocks, 256, 0, stream>>>(W, int(d_out), int(d_in), group, n_groups, maxq, scales, zeros, codes, Q); count_launch(); break;
+        default: return GPTQ_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+int launch_widen_bf16(const uint16_t* src, float* dst, int64_t count, cudaStream_t stream) {
+    if (count <= 0) return GPTQ_OK;
+    const unsigned blocks = unsigned(std::min<int64_t>((count + 255) / 256, 148 * 32));
+    sweep::widen_bf16_kernel<<<blocks, 256, 0, stream>>>(src, dst, size_t(count)); count_launch();
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+int launch_fill(float* p, int64_t count, float value, cudaStream_t stream) {
+    if (count <= 0) return GPTQ_OK;
+    const unsigned blocks = unsigned(std::min<int64_t>((count + 255) / 256, 148 * 32));
+    sweep::fill_kernel<<<blocks, 256, 0, stream>>>(p, size_t(count), value); count_launch();
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+}  // namespace gptq

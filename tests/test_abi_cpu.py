@@ -1,0 +1,136 @@
+"""CPU-only checks of the C ABI: the library builds and loads without a GPU,
+exports every entry point include/gptq.h declares, and rejects invalid
+arguments on the host (before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_weight_quantization_05_b200 import _native, build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()          # no-op when up to date; nvcc cross-compiles here
+    return _native.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_stages():
+    names = declared_functions()
+    for n in ("gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer", "gptq_rtn_layer"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(_native.SIGNATURES) == set(names)
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.gptq_abi_version() == 1
+    for code, name in _native.STATUS.items():
+        assert lib.gptq_status_string(code).decode() == name
+
+
+def test_workspace_sizes(lib):
+    assert lib.gptq_hessian_workspace_size(_native.GPTQ_BF16, 1000, 512) == 0
+    assert lib.gptq_hessian_workspace_size(_native.GPTQ_F32, 1000, 512) == 3 * 1000 * 512 * 2
+    assert lib.gptq_prepare_hinv_workspace_size(512) >= 2 * 512 * 512 * 4
+    assert lib.gptq_prepare_hinv_workspace_size(100) == 0          # d_in % 128 != 0
+    assert lib.gptq_quantize_workspace_size(300, 512, 128) == 300 * 128 * 4
+    assert lib.gptq_quantize_workspace_size(300, 512, 64) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)   # 16-byte aligned, never dereferenced: validation fails first
+MIS = ctypes.c_void_p(0x10004)    # misaligned
+
+
+def test_hessian_rejects_bad_arguments(lib):
+    f = lib.gptq_hessian_accumulate
+    assert f(None, 1, 64, 512, FAKE, None, 0, None) == 1            # NULL X
+    assert f(FAKE, 1, 64, 512, None, None, 0, None) == 1            # NULL H
+    assert f(FAKE, 1, 64, 500, FAKE, None, 0, None) == 1            # d_in % 128
+    assert f(FAKE, 1, 64, 65536, FAKE, None, 0, None) == 1          # d_in too large
+    assert f(FAKE, 7, 64, 512, FAKE, None, 0, None) == 1            # dtype
+    assert f(MIS, 1, 64, 512, FAKE, None, 0, None) == 1             # alignment
+    assert f(FAKE, 0, 64, 512, FAKE, None, 0, None) == 1            # fp32 needs workspace
+    assert f(FAKE, 0, 64, 512, FAKE, FAKE, 100, None) == 1          # workspace too small
+    assert f(FAKE, 1, -1, 512, FAKE, None, 0, None) == 1            # negative n
+    assert f(None, 1, 0, 512, None, None, 0, None) == 0             # n == 0: no-op
+
+
+def test_prepare_hinv_rejects_bad_arguments(lib):
+    f = lib.gptq_prepare_hinv
+    ws = lib.gptq_prepare_hinv_workspace_size(512)
+    assert f(None, 512, 0.01, FAKE, None, FAKE, ws, None) == 1
+    assert f(FAKE, 512, 0.01, None, None, FAKE, ws, None) == 1
+    assert f(FAKE, 512, 0.01, FAKE, None, None, ws, None) == 1
+    assert f(FAKE, 512, 0.01, FAKE, None, FAKE, ws - 1, None) == 1
+    assert f(FAKE, 512, -0.1, FAKE, None, FAKE, ws, None) == 1
+    assert f(FAKE, 512, float("nan"), FAKE, None, FAKE, ws, None) == 1
+    assert f(FAKE, 384 + 1, 0.01, FAKE, None, FAKE, ws, None) == 1
+    assert f(FAKE, 512, 0.01, FAKE, ctypes.c_void_p(0x10002), FAKE, ws, None) == 1
+
+
+def test_quantize_rejects_bad_arguments(lib):
+    f = lib.gptq_quantize_layer
+    ws = lib.gptq_quantize_workspace_size(64, 512, 128)
+    ok = [FAKE, 64, 512, FAKE, 4, 128, -1, FAKE, FAKE, FAKE, None, FAKE, ws, None]
+
+    def call(**kw):
+        a = list(ok)
+        idx = {"W": 0, "d_out": 1, "d_in": 2, "U": 3, "bits": 4, "bs": 5, "g": 6, "codes": 7, "scales": 8,
+               "zeros": 9, "Q": 10, "ws": 11, "wsb": 12}
+        for k, v in kw.items():
+            a[idx[k]] = v
+        return f(*a)
+
+    assert call(W=None) == 1
+    assert call(U=None) == 1
+    assert call(codes=None) == 1
+    assert call(ws=None) == 1
+    assert call(wsb=ws - 4) == 1
+    assert call(d_out=0) == 1
+    assert call(d_in=320) == 1
+    assert call(bits=5) == 1
+    assert call(bits=1) == 1
+    assert call(g=64) == 1            # not a multiple of 128
+    assert call(g=384) == 1           # does not divide 512
+    assert call(bs=64) == 2           # valid for the method, unsupported here
+    assert call(W=MIS) == 1
+    assert call(Q=MIS) == 1
+    assert call(scales=ctypes.c_void_p(0x10001)) == 1
+
+
+def test_rtn_and_helpers_reject_bad_arguments(lib):
+    f = lib.gptq_rtn_layer
+    assert f(None, 64, 512, 4, -1, FAKE, FAKE, FAKE, None, None) == 1
+    assert f(FAKE, 64, 512, 6, -1, FAKE, FAKE, FAKE, None, None) == 1
+    assert f(FAKE, 64, 512, 4, 100, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.gptq_widen_bf16(None, FAKE, 10, None) == 1
+    assert lib.gptq_widen_bf16(FAKE, FAKE, -1, None) == 1
+    assert lib.gptq_widen_bf16(None, None, 0, None) == 0
+    assert lib.gptq_fill_f32(None, 10, 0.0, None) == 1
+    assert lib.gptq_fill_f32(ctypes.c_void_p(0x10001), 10, 0.0, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    with pytest.raises(RuntimeError):
+        _native._lib = None
+        try:
+            _native.load(str(tmp_path / "missing.so"))
+        finally:
+            _native._lib = None

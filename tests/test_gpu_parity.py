@@ -1,0 +1,280 @@
+"""GPU parity: every stage of the CUDA path (through the C ABI) against the
+fp64 oracle on the same seeded inputs.  Tolerances: tests/parity_util.py."""
+import numpy as np
+import pytest
+import scipy.linalg.blas as blas
+import torch
+
+import oracle
+from post_weight_quantization_05_b200 import api, build_lib, synth
+from parity_util import (CODE_MATCH, H_TOL, LOSS_TOL, U_TOL, check_codes, dequant_rows, fp16_values,
+                         oracle_pipeline, rel_fro, to_dev_x, unpack_gpu_codes, upper)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _ready():
+    build_lib.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    api.get_status(raise_on_error=False)
+    yield
+    code, _ = api.get_status(raise_on_error=False)
+    assert code == 0
+
+
+def _gpu_quantize(W, U, bits, groupsize, want_q=True):
+    d_out, d_in = W.shape
+    Wt = torch.from_numpy(np.ascontiguousarray(W, dtype=np.float32)).cuda()
+    Ut = torch.from_numpy(np.ascontiguousarray(U, dtype=np.float32)).cuda()
+    ng = api.n_groups(d_in, groupsize)
+    codes = torch.zeros((d_out, d_in * bits // 32), dtype=torch.int32, device="cuda")
+    scales = torch.zeros((d_out, ng), dtype=torch.float16, device="cuda")
+    zeros = torch.zeros((d_out, ng), dtype=torch.float16, device="cuda")
+    Q = torch.zeros((d_out, d_in), dtype=torch.float32, device="cuda") if want_q else None
+    ws = api.workspace(api.quantize_workspace_size(d_out, d_in), "cuda")
+    api.quantize_layer(Wt, Ut, bits, 128, groupsize, codes, scales, zeros, ws, Q)
+    api.get_status()
+    return codes, scales, zeros, Q
+
+
+# ---------------------------------------------------------------- RTN
+@pytest.mark.parametrize("bits,groupsize,d_out,d_in", [
+    (4, -1, 256, 512), (3, -1, 97, 384), (4, 128, 300, 640), (2, 256, 64, 512), (8, -1, 33, 256),
+    (3, 128, 1, 128)])
+def test_rtn_bit_exact(bits, groupsize, d_out, d_in):
+    rng = np.random.default_rng(100 + bits)
+    W = (rng.standard_normal((d_out, d_in)) * 0.02).astype(np.float32)
+    ref = oracle.rtn_quantize(W, bits, groupsize)
+    Wt = torch.from_numpy(W).cuda()
+    ng = api.n_groups(d_in, groupsize)
+    codes = torch.zeros((d_out, d_in * bits // 32), dtype=torch.int32, device="cuda")
+    scales = torch.zeros((d_out, ng), dtype=torch.float16, device="cuda")
+    zeros = torch.zeros((d_out, ng), dtype=torch.float16, device="cuda")
+    Q = torch.zeros((d_out, d_in), dtype=torch.float32, device="cuda")
+    api.rtn_layer(Wt, bits, groupsize, codes, scales, zeros, Q)
+    api.get_status()
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), oracle.pack_codes(ref["codes"], bits))
+    assert np.array_equal(fp16_values(scales), ref["scales"])
+    assert np.array_equal(fp16_values(zeros), ref["zeros"])
+    assert np.array_equal(Q.cpu().numpy().astype(np.float64), ref["Q"])
+
+
+def test_rtn_degenerate_rows():
+    """A zero row and a constant row (range below the 1e-8 floor)."""
+    W = np.zeros((4, 128), dtype=np.float32)
+    W[1] = 0.25
+    W[2] = -3.0
+    W[3, :64] = 1.0
+    ref = oracle.rtn_quantize(W, 4, -1)
+    Wt = torch.from_numpy(W).cuda()
+    codes = torch.zeros((4, 16), dtype=torch.int32, device="cuda")
+    scales = torch.zeros((4, 1), dtype=torch.float16, device="cuda")
+    zeros = torch.zeros((4, 1), dtype=torch.float16, device="cuda")
+    Q = torch.zeros((4, 128), dtype=torch.float32, device="cuda")
+    api.rtn_layer(Wt, 4, -1, codes, scales, zeros, Q)
+    api.get_status()
+    assert np.array_equal(fp16_values(scales), ref["scales"])
+    assert np.array_equal(fp16_values(zeros), ref["zeros"])
+    assert np.array_equal(Q.cpu().numpy().astype(np.float64), ref["Q"])
+
+
+# ---------------------------------------------------------------- H
+@pytest.mark.parametrize("n,d", [(1000, 384), (4096, 512), (333, 768), (64, 128), (20480, 1024)])
+def test_hessian_bf16(n, d):
+    p = synth.custom("h", 8, d, n, x_dtype="bf16", n_batches=2, layer=d + n)
+    H = torch.zeros((d, d), dtype=torch.float32, device="cuda")
+    batches = []
+    for b in range(p.n_batches):
+        xb = p.x_batch(b)
+        batches.append(synth.x_as_f32(p, xb))
+        api.hessian_accumulate(to_dev_x(p, xb), H)
+    api.get_status()
+    ref = oracle.hessian(batches)
+    assert rel_fro(upper(H.cpu().numpy()), upper(ref)) <= H_TOL
+
+
+def test_hessian_f32_split():
+    p = synth.smoke()
+    X = p.x_batch(0)
+    H = torch.zeros((512, 512), dtype=torch.float32, device="cuda")
+    ws = api.workspace(api.hessian_workspace_size(0, X.shape[0], 512), "cuda")
+    api.hessian_accumulate(to_dev_x(p, X), H, ws)
+    api.get_status()
+    ref = oracle.hessian([X])
+    assert rel_fro(upper(H.cpu().numpy()), upper(ref)) <= H_TOL
+
+
+def test_hessian_empty_batch_is_noop():
+    H = torch.full((256, 256), 3.0, dtype=torch.float32, device="cuda")
+    X = torch.zeros((0, 256), dtype=torch.bfloat16, device="cuda")
+    api.hessian_accumulate(X, H)
+    api.get_status()
+    assert torch.all(H == 3.0)
+
+
+# ---------------------------------------------------------------- U
+@pytest.mark.parametrize("d,rho", [(128, 0.9), (512, 0.9), (768, 0.8), (1024, 0.5)])
+def test_prepare_hinv(d, rho):
+    p = synth.custom("u", 8, d, 4 * d, rho=rho, x_dtype="bf16", layer=7 * d)
+    Xf = synth.x_as_f32(p, p.x_batch(0))
+    H = oracle.hessian([Xf])
+    Hd, lam = oracle.damp(H, 0.01)
+    Uref = oracle.hinv_upper_factor(Hd)
+    Ht = torch.from_numpy(np.triu(H).astype(np.float32)).cuda()   # only the upper triangle is read
+    Ut = torch.empty((d, d), dtype=torch.float32, device="cuda")
+    info = torch.full((1,), -5, dtype=torch.int32, device="cuda")
+    ws = api.workspace(api.prepare_hinv_workspace_size(d), "cuda")
+    api.prepare_hinv(Ht, Ut, ws, 0.01, info)
+    api.get_status()
+    assert int(info.item()) == 0
+    U = Ut.cpu().numpy()
+    assert np.all(np.tril(U, -1) == 0)
+    assert rel_fro(U, Uref) <= U_TOL
+
+
+def test_prepare_hinv_not_positive_definite():
+    d = 256
+    Ht = torch.zeros((d, d), dtype=torch.float32, device="cuda")    # X == 0 -> H = 0, lambda = 0
+    Ut = torch.empty((d, d), dtype=torch.float32, device="cuda")
+    info = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    ws = api.workspace(api.prepare_hinv_workspace_size(d), "cuda")
+    api.prepare_hinv(Ht, Ut, ws, 0.01, info)
+    code, detail = api.get_status(raise_on_error=False)
+    assert code == 3 and detail == 1
+    assert int(info.item()) == 1
+    assert torch.isnan(Ut).all()
+
+
+def test_prepare_hinv_nonfinite():
+    d = 128
+    H = np.eye(d, dtype=np.float32)
+    H[5, 5] = np.nan
+    Ut = torch.empty((d, d), dtype=torch.float32, device="cuda")
+    ws = api.workspace(api.prepare_hinv_workspace_size(d), "cuda")
+    api.prepare_hinv(torch.from_numpy(H).cuda(), Ut, ws, 0.01, None)
+    code, _ = api.get_status(raise_on_error=False)
+    assert code == 4
+
+
+# ---------------------------------------------------------------- sweep given the oracle's U
+@pytest.mark.parametrize("bits,groupsize,d_out,d_in", [
+    (4, -1, 512, 512), (3, -1, 200, 384), (4, 128, 300, 640), (4, 256, 128, 512), (2, -1, 64, 256),
+    (8, 128, 40, 256), (4, -1, 1, 128)])
+def test_sweep_given_oracle_u(bits, groupsize, d_out, d_in):
+    p = synth.custom("s", d_out, d_in, 3 * d_in, bits=bits, groupsize=groupsize, x_dtype="f32",
+                     layer=d_out * 7 + d_in + bits)
+    X = p.x_batch(0)
+    H = oracle.hessian([X])
+    Hd, _ = oracle.damp(H, 0.01)
+    U = oracle.hinv_upper_factor(Hd)
+    ref = oracle.gptq_quantize(p.W, U, bits, 128, groupsize)
+    codes, scales, zeros, Q = _gpu_quantize(p.W, U, bits, groupsize)
+    got = unpack_gpu_codes(codes, bits, d_in)
+    check_codes(got, ref["codes"], "sweep")
+    s, z = fp16_values(scales), fp16_values(zeros)
+    if groupsize < 0:
+        assert np.array_equal(s, ref["scales"]) and np.array_equal(z, ref["zeros"])
+    else:
+        g0 = 0   # the first group is set from the original weights on both sides
+        assert np.array_equal(s[:, g0], ref["scales"][:, g0]) and np.array_equal(z[:, g0], ref["zeros"][:, g0])
+        assert np.mean(s == ref["scales"]) >= 0.99
+        assert np.allclose(s, ref["scales"], rtol=2e-3)
+    Qg = Q.cpu().numpy().astype(np.float64)
+    assert np.array_equal(Qg, dequant_rows(got, s, z, groupsize))     # Q lies on the recorded grid
+    lg = oracle.layer_loss_hessian(p.W, Qg, H)
+    lo = oracle.layer_loss_hessian(p.W, ref["Q"], H)
+    assert abs(lg / lo - 1.0) <= LOSS_TOL
+
+
+# ---------------------------------------------------------------- end to end
+def _gpu_pipeline(p, batches_dev, want_q=True, ws_rows=0):
+    lq = api.LayerQuantizer(p.d_out, p.d_in, p.bits, p.groupsize, 128, p.percdamp, want_q=want_q,
+                            max_f32_rows=ws_rows)
+    lq.begin(torch.from_numpy(p.W).cuda())
+    for xb in batches_dev:
+        lq.add_batch(xb)
+    lq.finish()
+    api.get_status()
+    return lq
+
+
+def test_smoke_end_to_end():
+    """The 512-dim, 2048-sample correlated example: GPU vs oracle at every
+    stage, and GPTQ < RTN / 2 on the GPU result as the itwiki page states."""
+    p = synth.smoke()
+    X = p.x_batch(0)
+    lq = _gpu_pipeline(p, [to_dev_x(p, X)], ws_rows=X.shape[0])
+    H, U, ref = oracle_pipeline(p, [X])
+    assert rel_fro(upper(lq.H.cpu().numpy()), upper(H)) <= H_TOL
+    assert rel_fro(lq.U.cpu().numpy(), U) <= U_TOL
+    got = unpack_gpu_codes(lq.codes, 4, 512)
+    check_codes(got, ref["codes"], "smoke")
+    Qg = lq.Q.cpu().numpy().astype(np.float64)
+    lg = oracle.layer_loss_hessian(p.W, Qg, H)
+    lo = oracle.layer_loss_hessian(p.W, ref["Q"], H)
+    assert abs(lg / lo - 1.0) <= LOSS_TOL
+    rtn = oracle.rtn_quantize(p.W, 4)
+    assert lg < 0.5 * oracle.layer_loss_hessian(p.W, rtn["Q"], H)
+
+
+@pytest.mark.parametrize("d_out,d_in,n,bits,g", [(300, 640, 3000, 4, 128), (129, 384, 1500, 3, -1),
+                                                 (96, 1024, 5000, 4, 256)])
+def test_end_to_end_bf16(d_out, d_in, n, bits, g):
+    p = synth.custom("e2e", d_out, d_in, n, bits=bits, groupsize=g, x_dtype="bf16", n_batches=3,
+                     layer=d_out + d_in)
+    xs = [p.x_batch(b) for b in range(p.n_batches)]
+    lq = _gpu_pipeline(p, [to_dev_x(p, x) for x in xs])
+    H, U, ref = oracle_pipeline(p, [synth.x_as_f32(p, x) for x in xs])
+    assert rel_fro(upper(lq.H.cpu().numpy()), upper(H)) <= H_TOL
+    assert rel_fro(lq.U.cpu().numpy(), U) <= U_TOL
+    got = unpack_gpu_codes(lq.codes, bits, d_in)
+    check_codes(got, ref["codes"], "e2e")
+    Qg = lq.Q.cpu().numpy().astype(np.float64)
+    assert abs(oracle.layer_loss_hessian(p.W, Qg, H) / oracle.layer_loss_hessian(p.W, ref["Q"], H) - 1) <= LOSS_TOL
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+def test_gpt768_layer(layer):
+    """One layer of each shape of the 12-block d_model=768 GPT, full size
+    (20480 calibration rows in 10 batches)."""
+    p = synth.gpt768_layer(layer)
+    xs = [p.x_batch(b) for b in range(p.n_batches)]
+    lq = _gpu_pipeline(p, [to_dev_x(p, x) for x in xs])
+    H, U, ref = oracle_pipeline(p, [synth.x_as_f32(p, x) for x in xs])
+    assert rel_fro(upper(lq.H.cpu().numpy()), upper(H)) <= H_TOL
+    assert rel_fro(lq.U.cpu().numpy(), U) <= U_TOL
+    got = unpack_gpu_codes(lq.codes, 4, p.d_in)
+    check_codes(got, ref["codes"], p.name)
+    Qg = lq.Q.cpu().numpy().astype(np.float64)
+    assert abs(oracle.layer_loss_hessian(p.W, Qg, H) / oracle.layer_loss_hessian(p.W, ref["Q"], H) - 1) <= LOSS_TOL
+
+
+@pytest.mark.slow
+def test_attn4096_full_size_sampled_rows():
+    """The 4096 x 4096 layer with 262144 calibration rows (16 batches), in the
+    launch configuration the benchmark times.  The oracle computes H and U in
+    full (fp64) and the sweep on a sample of rows (rows are independent
+    given U)."""
+    p = synth.attn4096()
+    xs = synth.x_batches_threaded(p, 8)
+    lq = _gpu_pipeline(p, [to_dev_x(p, x) for x in xs], want_q=False)
+    Hu = np.zeros((4096, 4096), dtype=np.float64, order="F")
+    for x in xs:
+        xf = np.asfortranarray(synth.x_as_f32(p, x).astype(np.float64))
+        Hu = blas.dsyrk(2.0, xf, beta=1.0, c=Hu, trans=1, lower=0, overwrite_c=1)
+    H = np.triu(Hu) + np.triu(Hu, 1).T
+    assert rel_fro(upper(lq.H.cpu().numpy()), upper(H)) <= H_TOL
+    Hd, _ = oracle.damp(H, p.percdamp)
+    U = oracle.hinv_upper_factor(Hd)
+    assert rel_fro(lq.U.cpu().numpy(), U) <= U_TOL
+    rows = np.random.default_rng(0).choice(4096, size=48, replace=False)
+    ref = oracle.gptq_quantize(p.W[rows], U, p.bits, 128, p.groupsize)
+    got = unpack_gpu_codes(lq.codes, 4, 4096)[rows]
+    check_codes(got, ref["codes"], "attn4096")
+    s = fp16_values(lq.scales)[rows]
+    z = fp16_values(lq.zeros)[rows]
+    Qg = dequant_rows(got, s, z, p.groupsize)
+    lg = oracle.layer_loss_hessian(p.W[rows], Qg, H)
+    lo = oracle.layer_loss_hessian(p.W[rows], ref["Q"], H)
+    assert abs(lg / lo - 1.0) <= LOSS_TOL
