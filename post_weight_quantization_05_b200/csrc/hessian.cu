@@ -14,8 +14,13 @@
 //  - Per stage a TMA load brings 64 calibration rows of the a-columns
 //    (16 KB) and of the b-columns (32 KB); 4 stages in flight.  One thread
 //    issues TMA, one thread issues tcgen05.mma (M=128, N=256, K=16, fp32
-//    accumulator in 256 TMEM columns), and all four warps drain TMEM in the
-//    epilogue and add 2*acc into H.
+//    accumulator in TMEM).
+//  - Promotion: the tensor core's fp32 accumulation loses about half an ulp
+//    per accumulation step (measured: relative error ~4e-5 over a chain of
+//    16384 rows).  So the K loop is cut into chunks of 512 rows, each summed
+//    into one of two TMEM buffers (2 x 256 columns) while eight epilogue warps
+//    drain the other buffer and add it into fp32 registers (round to
+//    nearest); at the end they add 2 * sum into H.
 //  - fp32 inputs are split into three bf16 terms by `split3_kernel`; the
 //    contraction then runs over the six leading cross products
 //    (hh, hm, mh, mm, hl, lh), which the K loop walks one after another.
@@ -32,12 +37,14 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
 constexpr int STAGES = 4;
+constexpr int CHUNK = 8;          // k-steps (of BK rows) summed in TMEM before promotion
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int CHUNK_BYTES = 64 * BK * 2;  // one TMA box: 64 columns x 64 rows
-constexpr int TMEM_COLS = 256;
-constexpr int THREADS = 128;
+constexpr int TMEM_COLS = 2 * BN;         // two accumulator buffers
+constexpr int EPI_WARPS = 8;              // 4 TMEM lane quadrants x 2 column halves
+constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + size_t(STAGES) * STAGE_BYTES + 256 /*barriers*/;
 
 struct Params {
@@ -72,8 +79,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(STAGES) * STAGE_BYTES);
     uint64_t* empty = full + STAGES;
-    uint64_t* accum = empty + STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+    uint64_t* tfull = empty + STAGES;   // [2] MMA -> epilogue: chunk summed in buffer b
+    uint64_t* tempty = tfull + 2;       // [2] epilogue -> MMA: buffer b drained
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
 
     int ti, tj;
     tile_coords(blockIdx.x, p, ti, tj);
@@ -89,7 +97,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], EPI_WARPS);
+        }
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -103,84 +114,118 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int kper = (p.n + BK - 1) / BK;
     const int ksteps = kper * p.npairs;
-    bool ok = true;
+    const int nchunks = (ksteps + CHUNK - 1) / CHUNK;
 
-    if (warp == 0 && lane == 0) {
-        // ---------------- TMA producer
-        int last_round[STAGES];
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            bool ok = true;
+            int last_round[STAGES];
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
-        for (int ks = 0; ks < ksteps; ++ks) {
-            const int s = ks % STAGES;
-            const uint32_t round = ks / STAGES;
-            if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, st, 101)) { ok = false; break; }
-            const int pair = ks / kper;
-            const int r0 = (ks - pair * kper) * BK;
-            uint8_t* sa = smem + size_t(s) * STAGE_BYTES;
-            uint8_t* sb = sa + A_BYTES;
-            mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+            for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
+            for (int ks = 0; ks < ksteps; ++ks) {
+                const int s = ks % STAGES;
+                const uint32_t round = ks / STAGES;
+                if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, st, 101)) { ok = false; break; }
+                const int pair = ks / kper;
+                const int r0 = (ks - pair * kper) * BK;
+                uint8_t* sa = smem + size_t(s) * STAGE_BYTES;
+                uint8_t* sb = sa + A_BYTES;
+                mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
 #pragma unroll
-            for (int h = 0; h < BM / 64; ++h) tma_load_3d(sa + h * CHUNK_BYTES, &tmX, a0 + 64 * h, r0, p.pa[pair], &full[s]);
+                for (int h = 0; h < BM / 64; ++h)
+                    tma_load_3d(sa + h * CHUNK_BYTES, &tmX, a0 + 64 * h, r0, p.pa[pair], &full[s]);
 #pragma unroll
-            for (int h = 0; h < BN / 64; ++h) tma_load_3d(sb + h * CHUNK_BYTES, &tmX, b0 + 64 * h, r0, p.pb[pair], &full[s]);
-            last_round[s] = int(round);
-        }
-        if (!ok) {
-            // let the copies already in flight land before the CTA can exit
-#pragma unroll
-            for (int s = 0; s < STAGES; ++s)
-                if (last_round[s] >= 0) (void)mbar_wait(&full[s], uint32_t(last_round[s]) & 1u, st, 104);
-        }
-    } else if (warp == 1 && lane == 0) {
-        // ---------------- MMA issuer
-        constexpr uint32_t idesc = idesc_bf16_mn_mn(BM, BN);
-        for (int ks = 0; ks < ksteps; ++ks) {
-            const int s = ks % STAGES;
-            const uint32_t round = ks / STAGES;
-            if (!mbar_wait(&full[s], round & 1u, st, 102)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t sa = smem_u32(smem + size_t(s) * STAGE_BYTES);
-            const uint32_t sb = sa + A_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-                // 16 K rows = two 8-row groups of 128 bytes each
-                const uint64_t da = sdesc_sw128(sa + kk * 2048, CHUNK_BYTES, 1024);
-                const uint64_t db = sdesc_sw128(sb + kk * 2048, CHUNK_BYTES, 1024);
-                umma_f16(tmem_base, da, db, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                for (int h = 0; h < BN / 64; ++h)
+                    tma_load_3d(sb + h * CHUNK_BYTES, &tmX, b0 + 64 * h, r0, p.pb[pair], &full[s]);
+                last_round[s] = int(round);
             }
-            umma_commit(&empty[s]);  // frees the stage once these MMAs are done
+            if (!ok) {
+                // let the copies already in flight land before the CTA can exit
+#pragma unroll
+                for (int s = 0; s < STAGES; ++s)
+                    if (last_round[s] >= 0) (void)mbar_wait(&full[s], uint32_t(last_round[s]) & 1u, st, 104);
+            }
         }
-        umma_commit(accum);          // accumulator complete (also on the error path)
-    }
-
-    // ---------------- epilogue: TMEM -> registers -> H += alpha * acc
-    __syncwarp();
-    const bool acc_ready = mbar_wait(accum, 0, st, 103);
-    tc_fence_after();
-    if (acc_ready && ksteps > 0) {
-        const int m = warp * 32 + lane;  // TMEM lane == row of the tile
-        const int a = a0 + m;
-        float* hrow = H + size_t(a) * p.d;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            float v[32];
-            tmem_ld_32x32b_x32(tmem_base + (uint32_t(warp * 32) << 16) + uint32_t(c * 32), v);
-            const int b = b0 + c * 32;
-            if (b + 32 <= p.d) {
-                float4* dst = reinterpret_cast<float4*>(hrow + b);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            constexpr uint32_t idesc = idesc_bf16_mn_mn(BM, BN);
+            bool ok = true;
+            for (int c = 0; c < nchunks && ok; ++c) {
+                const int buf = c & 1;
+                const int use = c >> 1;
+                if (use > 0 && !mbar_wait(&tempty[buf], uint32_t(use - 1) & 1u, st, 105)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t dt = tmem_base + uint32_t(buf * BN);
+                const int k_end = min(ksteps, (c + 1) * CHUNK);
+                for (int ks = c * CHUNK; ks < k_end; ++ks) {
+                    const int s = ks % STAGES;
+                    const uint32_t round = ks / STAGES;
+                    if (!mbar_wait(&full[s], round & 1u, st, 102)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + size_t(s) * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    float4 h = dst[q];
-                    h.x = fmaf(p.alpha, v[4 * q + 0], h.x);
-                    h.y = fmaf(p.alpha, v[4 * q + 1], h.y);
-                    h.z = fmaf(p.alpha, v[4 * q + 2], h.z);
-                    h.w = fmaf(p.alpha, v[4 * q + 3], h.w);
-                    dst[q] = h;
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        // 16 K rows = two 8-row groups of 128 bytes each
+                        const uint64_t da = sdesc_sw128(sa + kk * 2048, CHUNK_BYTES, 1024);
+                        const uint64_t db = sdesc_sw128(sb + kk * 2048, CHUNK_BYTES, 1024);
+                        umma_f16(dt, da, db, idesc, (ks > c * CHUNK || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&empty[s]);  // frees the stage once these MMAs are done
                 }
-            } else {
+                umma_commit(&tfull[buf]);    // this chunk's sum is complete (also on the error path)
+            }
+        }
+    } else {
+        // ---------------- epilogue warps: promote each chunk into fp32 registers
+        const int e = warp - 2;
+        const int quad = warp & 3;           // TMEM lanes this warp may access
+        const int half = e >> 2;             // which 128 of the 256 columns
+        const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+        float acc[128];
 #pragma unroll
-                for (int q = 0; q < 32; ++q)
-                    if (b + q < p.d) hrow[b + q] = fmaf(p.alpha, v[q], hrow[b + q]);
+        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+        bool ok = true;
+        for (int c = 0; c < nchunks; ++c) {
+            const int buf = c & 1;
+            const int use = c >> 1;
+            if (!mbar_wait(&tfull[buf], uint32_t(use) & 1u, st, 103)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + uint32_t(buf * BN + half * 128 + cc * 32), v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[cc * 32 + i] += v[i];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+        if (ok && nchunks > 0) {
+            const int a = a0 + quad * 32 + lane;   // TMEM lane == row of the tile
+            float* hrow = H + size_t(a) * p.d;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int b = b0 + half * 128 + cc * 32;
+                if (b + 32 <= p.d) {
+                    float4* dst = reinterpret_cast<float4*>(hrow + b);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 h = dst[q];
+                        h.x = fmaf(p.alpha, acc[cc * 32 + 4 * q + 0], h.x);
+                        h.y = fmaf(p.alpha, acc[cc * 32 + 4 * q + 1], h.y);
+                        h.z = fmaf(p.alpha, acc[cc * 32 + 4 * q + 2], h.z);
+                        h.w = fmaf(p.alpha, acc[cc * 32 + 4 * q + 3], h.w);
+                        dst[q] = h;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q)
+                        if (b + q < p.d) hrow[b + q] = fmaf(p.alpha, acc[cc * 32 + q], hrow[b + q]);
+                }
             }
         }
     }

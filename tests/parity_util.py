@@ -3,9 +3,18 @@
 Tolerances (stated once, used by every parity test):
   H        relative Frobenius error <= 1e-5   (upper triangle)
   U        relative Frobenius error <= 1e-4
-  codes    >= 99.9% identical; every differing code off by exactly one level
+  codes    >= 99.9% identical.  In every row the codes agree exactly up to
+           the row's first difference (its "initiating flip"), and that
+           first difference is off by exactly one level at a near-tie: the
+           oracle's value w/s + z lies within TIE_TOL of a rounding boundary.
+           After an initiating flip the row's later weights are compensated
+           differently, so its later codes follow another valid trajectory;
+           those are bounded by the fraction and the loss criteria.  (An fp32
+           restatement of the sweep on the CPU shows the same cascades,
+           including later codes two levels apart.)
   loss     ||W X^T - W^ X^T||^2 within 0.5% (relative) of the oracle's
-  grid     per-row scales/zeros (from the original W) and RTN: bit-exact
+  grid     per-row scales/zeros (from the original W) and RTN: bit-exact;
+           group scales/zeros: bit-exact given the GPU's own group min/max
 """
 import numpy as np
 import torch
@@ -17,6 +26,7 @@ H_TOL = 1e-5
 U_TOL = 1e-4
 CODE_MATCH = 0.999
 LOSS_TOL = 0.005
+TIE_TOL = 5e-3
 
 
 def rel_fro(a, b):
@@ -44,13 +54,33 @@ def fp16_values(t):
     return t.cpu().float().numpy().astype(np.float32)
 
 
-def check_codes(got, ref, what=""):
+def check_codes(got, ref, what="", match=CODE_MATCH, bits=None, groupsize=-1, gpu_scales=None,
+                gpu_zeros=None):
+    """`ref` is the oracle's output dict (with the trace when available)."""
     got = np.asarray(got)
-    ref = np.asarray(ref)
-    diff = np.abs(got - ref)
+    rc = np.asarray(ref["codes"])
+    diff = np.abs(got - rc)
     frac = float(np.mean(diff == 0))
-    assert frac >= CODE_MATCH, f"{what}: only {frac:.6f} of codes identical"
-    assert diff.max() <= 1, f"{what}: a code differs by {diff.max()} levels"
+    assert frac >= match, f"{what}: only {frac:.6f} of codes identical"
+    if "W_at" not in ref:
+        return frac
+    d_in = rc.shape[1]
+    g = d_in if groupsize <= 0 else groupsize
+    s_full = np.repeat(np.asarray(ref["scales"], np.float64), g, axis=1)[:, :d_in]
+    z_full = np.repeat(np.asarray(ref["zeros"], np.float64), g, axis=1)[:, :d_in]
+    grid_differs = None
+    if gpu_scales is not None:
+        gs = np.asarray(gpu_scales, np.float64)
+        gz = np.asarray(gpu_zeros, np.float64)
+        grid_differs = (gs != np.asarray(ref["scales"], np.float64)) | (gz != np.asarray(ref["zeros"], np.float64))
+    for r in np.where(diff.max(axis=1) > 0)[0]:
+        j = int(np.argmax(diff[r] > 0))
+        if grid_differs is not None and grid_differs[r, : j // g + 1].any():
+            continue     # the row's grid changed first (fp16 rounding of a min/max at a boundary)
+        assert diff[r, j] == 1, f"{what}: row {r} first differs at column {j} by {diff[r, j]} levels"
+        t = ref["W_at"][r, j] / s_full[r, j] + z_full[r, j]
+        dist = abs((t - np.floor(t)) - 0.5)
+        assert dist <= TIE_TOL, f"{what}: row {r} col {j} flipped away from a tie (distance {dist:.2e})"
     return frac
 
 
@@ -71,5 +101,17 @@ def oracle_pipeline(problem, batches=None, rows=None):
     Hd, lam = oracle.damp(H, problem.percdamp)
     U = oracle.hinv_upper_factor(Hd)
     W = problem.W if rows is None else problem.W[rows]
-    out = oracle.gptq_quantize(W, U, problem.bits, problem.blocksize, problem.groupsize)
+    out = oracle.gptq_quantize(W, U, problem.bits, problem.blocksize, problem.groupsize, return_trace=True)
     return H, U, out
+
+
+def group_grid_from(W_state, bits, groupsize):
+    """Grid of each group computed by the oracle's formula from given weights."""
+    d_out, d_in = W_state.shape
+    ng = d_in // groupsize
+    s = np.zeros((d_out, ng), np.float32)
+    z = np.zeros((d_out, ng), np.float32)
+    for gi in range(ng):
+        blk = np.asarray(W_state[:, gi * groupsize:(gi + 1) * groupsize], np.float32)
+        s[:, gi], z[:, gi] = oracle.grid_params(blk.min(1), blk.max(1), bits)
+    return s, z
