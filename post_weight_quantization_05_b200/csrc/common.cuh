@@ -194,4 +194,14 @@ __device__ __forceinline__ float quant_code(float w, float s, float z, float max
     return fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w, s)), z), 0.0f), maxq);
 }
 
+// Non-tensor bulk copy global -> shared (16-byte aligned, size multiple of
+// 16), completion counted on `bar`.  No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 }  // namespace gptq

@@ -26,7 +26,7 @@ namespace factor {
 
 constexpr int NB = 128;
 constexpr int LD = NB + 1;  // padded shared-memory row
-constexpr int DIAG_THREADS = 512;
+constexpr int DIAG_THREADS = 256;
 constexpr size_t DIAG_SMEM = size_t(2) * NB * LD * sizeof(float);
 
 struct Layout {
@@ -79,65 +79,187 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const fl
     }
 }
 
+// ---------------------------------------------------------------------------
+// One 128 x 128 diagonal block: L L^T = A_kk (in place, lower) and L^-1.
+// The block is cut into 4 x 4 sub-blocks of 32.  For each sub-block column:
+// one warp factors the 32 x 32 diagonal sub-block in registers (lane = row,
+// column broadcasts by shuffles) and inverts it; all 8 warps then solve the
+// sub-blocks below against it and update the trailing sub-blocks.  Finally
+// the off-diagonal sub-blocks of L^-1 are formed from the diagonal ones.
+// ---------------------------------------------------------------------------
+constexpr int SB = 32;
+constexpr unsigned FULL = 0xffffffffu;
+
+// Warp-level Cholesky of the 32 x 32 sub-block at S[o.., o..] and its
+// inverse into Y[o.., o..].  Returns the failing column (0..31) or -1.
+__device__ __forceinline__ int warp_chol32(float* S, float* Y, int o, int lane) {
+    float a[SB];
+#pragma unroll
+    for (int j = 0; j < SB; ++j) a[j] = (j <= lane) ? S[(o + lane) * LD + o + j] : 0.0f;
+    int bad = -1;
+#pragma unroll
+    for (int c = 0; c < SB; ++c) {
+        const float piv = __shfl_sync(FULL, a[c], c);      // warp-uniform
+        if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) bad = c;
+        const float lcc = sqrtf(piv);
+        const float v = (lane == c) ? lcc : __fdiv_rn(a[c], lcc);   // lanes < c hold 0
+        a[c] = v;
+#pragma unroll
+        for (int j = c + 1; j < SB; ++j) {
+            const float ljc = __shfl_sync(FULL, v, j);     // L[j][c]
+            if (lane >= j) a[j] = fmaf(-v, ljc, a[j]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < SB; ++j)
+        if (j <= lane) S[(o + lane) * LD + o + j] = a[j];
+    // inverse: forward substitution on the identity, lane = row
+    float x[SB];
+#pragma unroll
+    for (int j = 0; j < SB; ++j) x[j] = (j == lane) ? 1.0f : 0.0f;
+#pragma unroll
+    for (int i = 0; i < SB; ++i) {
+        const float inv = __fdiv_rn(1.0f, __shfl_sync(FULL, a[i], i));
+        if (lane == i) {
+#pragma unroll
+            for (int j = 0; j <= i; ++j) x[j] *= inv;
+        }
+        const float lri = a[i];                            // L[lane][i]
+#pragma unroll
+        for (int j = 0; j <= i; ++j) {
+            const float xij = __shfl_sync(FULL, x[j], i);
+            if (lane > i) x[j] = fmaf(-lri, xij, x[j]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < SB; ++j) Y[(o + lane) * LD + o + j] = (j <= lane) ? x[j] : 0.0f;
+    return bad;
+}
+
 // Factor the diagonal block A[k0:k0+NB, k0:k0+NB] = L L^T in place (lower) and
 // write its inverse L^-1 to Dinv (NB x NB, row-major).  A non-positive or
 // non-finite pivot sets *info = k0 + c + 1 (first failure only).
 __global__ void __launch_bounds__(DIAG_THREADS)
     potrf_diag_kernel(float* __restrict__ A, int d, int k0, float* __restrict__ Dinv, int* info, DevStatus* st) {
     extern __shared__ float sm[];
-    float* S = sm;             // [NB][LD] factor
+    float* S = sm;             // [NB][LD] factor (upper part used as scratch)
     float* Y = sm + NB * LD;   // [NB][LD] inverse
     __shared__ int failed;
     if (*info != 0) return;
-    const int t = threadIdx.x, ty = t >> 5, tx = t & 31;
-    constexpr int NY = DIAG_THREADS / 32;
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     for (int idx = t; idx < NB * NB; idx += DIAG_THREADS) {
         const int r = idx / NB, c = idx % NB;
         S[r * LD + c] = (c <= r) ? A[size_t(k0 + r) * d + k0 + c] : 0.0f;
-        Y[r * LD + c] = (r == c) ? 1.0f : 0.0f;
+        Y[r * LD + c] = 0.0f;
     }
     if (t == 0) failed = 0;
     __syncthreads();
 
-    for (int c = 0; c < NB; ++c) {
-        if (t == 0) {
-            const float p = S[c * LD + c];
-            if (!(p > 0.0f) || !isfinite(p)) {
+    for (int kb = 0; kb < NB / SB; ++kb) {
+        const int o = kb * SB;
+        if (warp == 0) {
+            const int bad = warp_chol32(S, Y, o, lane);
+            if (bad >= 0 && lane == 0) {
                 failed = 1;
-                if (atomicCAS(info, 0, k0 + c + 1) == 0)
-                    record_error(st, isfinite(p) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, k0 + c + 1);
+                const float p = S[(o + bad) * LD + o + bad];
+                if (atomicCAS(info, 0, k0 + o + bad + 1) == 0)
+                    record_error(st, isfinite(p) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, k0 + o + bad + 1);
             }
-            S[c * LD + c] = sqrtf(p);
         }
         __syncthreads();
-        if (failed) break;
-        const float lcc = S[c * LD + c];
-        for (int r = c + 1 + t; r < NB; r += DIAG_THREADS) S[r * LD + c] = __fdiv_rn(S[r * LD + c], lcc);
-        __syncthreads();
-        for (int r = c + 1 + ty; r < NB; r += NY) {
-            const float lrc = S[r * LD + c];
-            for (int j = c + 1 + tx; j <= r; j += 32) S[r * LD + j] = fmaf(-lrc, S[j * LD + c], S[r * LD + j]);
+        if (failed) return;
+        const int below = NB - o - SB;
+        if (below == 0) break;
+        // solve the sub-blocks below: S[R][o..o+32) <- S[R][o..o+32) * Linv_kk^T
+        {
+            float out[2][8];
+            const int cg = t & 3;
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int r = o + SB + (t >> 2) + 64 * it;
+                if (r < NB) {
+                    float in[SB];
+#pragma unroll
+                    for (int k = 0; k < SB; ++k) in[k] = S[r * LD + o + k];
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        const int c = cg * 8 + cc;
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int k = 0; k < SB; ++k)
+                            if (k <= c) acc = fmaf(in[k], Y[(o + c) * LD + o + k], acc);
+                        out[it][cc] = acc;
+                    }
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int r = o + SB + (t >> 2) + 64 * it;
+                if (r < NB) {
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) S[r * LD + o + cg * 8 + cc] = out[it][cc];
+                }
+            }
+            __syncthreads();
+        }
+        // trailing update of the sub-blocks (bi, bj), kb < bj <= bi
+        {
+            const int i = t >> 3, j4 = (t & 7) * 4;
+            for (int bi = kb + 1; bi < NB / SB; ++bi) {
+                for (int bj = kb + 1; bj <= bi; ++bj) {
+                    const int r = bi * SB + i;
+                    float acc[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[q] = S[r * LD + bj * SB + j4 + q];
+#pragma unroll 8
+                    for (int k = 0; k < SB; ++k) {
+                        const float av = S[r * LD + o + k];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) acc[q] = fmaf(-av, S[(bj * SB + j4 + q) * LD + o + k], acc[q]);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) S[r * LD + bj * SB + j4 + q] = acc[q];
+                }
+            }
         }
         __syncthreads();
     }
-    if (failed) return;
 
-    // L^-1 by forward substitution on the identity, one pivot row at a time.
-    for (int i = 0; i < NB; ++i) {
-        const float lii = S[i * LD + i];
-        for (int j = t; j <= i; j += DIAG_THREADS) Y[i * LD + j] = __fdiv_rn(Y[i * LD + j], lii);
-        __syncthreads();
-        for (int r = i + 1 + ty; r < NB; r += NY) {
-            const float lri = S[r * LD + i];
-            for (int j = tx; j <= i; j += 32) Y[r * LD + j] = fmaf(-lri, Y[i * LD + j], Y[r * LD + j]);
+    // off-diagonal sub-blocks of L^-1:  Y[bi][bj] = -Y[bi][bi] * sum_{k=bj}^{bi-1} L[bi][k] Y[k][bj]
+    // T[bj] is kept in the (unused) strictly upper sub-blocks (0, 1 + bj) of S.
+    {
+        const int i = t >> 3, j4 = (t & 7) * 4;
+        for (int bi = 1; bi < NB / SB; ++bi) {
+            for (int bj = 0; bj < bi; ++bj) {
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                for (int k = bj * SB; k < bi * SB; ++k) {
+                    const float l = S[(bi * SB + i) * LD + k];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[q] = fmaf(l, Y[k * LD + bj * SB + j4 + q], acc[q]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) S[i * LD + (1 + bj) * SB + j4 + q] = acc[q];
+            }
+            __syncthreads();
+            for (int bj = 0; bj < bi; ++bj) {
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                for (int k = 0; k <= i; ++k) {
+                    const float y = Y[(bi * SB + i) * LD + bi * SB + k];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[q] = fmaf(y, S[k * LD + (1 + bj) * SB + j4 + q], acc[q]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) Y[(bi * SB + i) * LD + bj * SB + j4 + q] = -acc[q];
+            }
+            __syncthreads();
         }
-        __syncthreads();
     }
 
     for (int idx = t; idx < NB * NB; idx += DIAG_THREADS) {
         const int r = idx / NB, c = idx % NB;
         if (c <= r) A[size_t(k0 + r) * d + k0 + c] = S[r * LD + c];
-        Dinv[idx] = Y[r * LD + c];
+        Dinv[idx] = (c <= r) ? Y[r * LD + c] : 0.0f;
     }
 }
 

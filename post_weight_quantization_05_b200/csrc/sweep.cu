@@ -29,7 +29,8 @@ namespace sweep {
 
 constexpr int B = 128;
 constexpr int ROWS = 32;  // rows (threads) per CTA
-constexpr size_t SMEM = (size_t(B) * B + size_t(ROWS) * 33) * sizeof(float);
+// U block, 1/U[j][j], per-thread E rows; plus one mbarrier
+constexpr size_t SMEM = (size_t(B) * B + B + size_t(ROWS) * 33) * sizeof(float) + 16;
 
 // Per-row grid over columns [c0, c0 + len) of the ORIGINAL W: one warp per
 // (row, group).  Writes fp16 scale/zero bit patterns.
@@ -84,15 +85,18 @@ struct Packer {
 
 // Column J of the block: quantize, record code and E, and apply the rank-1
 // correction to the remaining columns of J's 32-column sub-block.
+struct Grid {
+    float s, inv_s, z, maxq;
+};
+
 template <int BITS, int J>
 __device__ __forceinline__ void quant_column(float (&w)[B], const float* __restrict__ Us, float* __restrict__ Erow,
-                                             float s, float z, float maxq, Packer<BITS>& pk, float* Qrow,
-                                             bool& finite) {
+                                             const Grid& gr, Packer<BITS>& pk, float* Qrow, bool& finite) {
     constexpr int SUB_END = (J / 32 + 1) * 32;
     const float wj = w[J];
-    const float c = quant_code(wj, s, z, maxq);
-    const float q = s * (c - z);
-    const float e = __fdiv_rn(wj - q, Us[J * B + J]);
+    const float c = quant_code(wj, gr.s, gr.z, gr.maxq);
+    const float q = gr.s * (c - gr.z);
+    const float e = (wj - q) * Us[B * B + J];     // 1/U[j][j] kept after the block
     finite &= isfinite(e);
     if (Qrow) Qrow[J] = q;
     pk.template put<J>(static_cast<uint32_t>(c));
@@ -105,10 +109,10 @@ __device__ __forceinline__ void quant_column(float (&w)[B], const float* __restr
 
 template <int BITS, int SB, int J>
 struct SubCols {
-    __device__ __forceinline__ static void run(float (&w)[B], const float* Us, float* Erow, float s, float z,
-                                               float maxq, Packer<BITS>& pk, float* Qrow, bool& finite) {
-        quant_column<BITS, SB * 32 + J>(w, Us, Erow, s, z, maxq, pk, Qrow, finite);
-        if constexpr (J + 1 < 32) SubCols<BITS, SB, J + 1>::run(w, Us, Erow, s, z, maxq, pk, Qrow, finite);
+    __device__ __forceinline__ static void run(float (&w)[B], const float* Us, float* Erow, const Grid& gr,
+                                               Packer<BITS>& pk, float* Qrow, bool& finite) {
+        quant_column<BITS, SB * 32 + J>(w, Us, Erow, gr, pk, Qrow, finite);
+        if constexpr (J + 1 < 32) SubCols<BITS, SB, J + 1>::run(w, Us, Erow, gr, pk, Qrow, finite);
     }
 };
 
@@ -134,14 +138,14 @@ __device__ __forceinline__ void cross_update(float (&w)[B], const float* __restr
 }
 
 template <int BITS, int SB>
-__device__ __forceinline__ void sub_block(float (&w)[B], const float* Us, float* Erow, float s, float z, float maxq,
+__device__ __forceinline__ void sub_block(float (&w)[B], const float* Us, float* Erow, const Grid& gr,
                                           Packer<BITS>& pk, float* Qrow, bool& finite) {
     // Erow is private to this thread: no synchronization needed around it.
-    SubCols<BITS, SB, 0>::run(w, Us, Erow, s, z, maxq, pk, Qrow, finite);
+    SubCols<BITS, SB, 0>::run(w, Us, Erow, gr, pk, Qrow, finite);
     if constexpr (SB < 1) cross_update<SB, 1>(w, Us, Erow);
     if constexpr (SB < 2) cross_update<SB, 2>(w, Us, Erow);
     if constexpr (SB < 3) cross_update<SB, 3>(w, Us, Erow);
-    if constexpr (SB + 1 < B / 32) sub_block<BITS, SB + 1>(w, Us, Erow, s, z, maxq, pk, Qrow, finite);
+    if constexpr (SB + 1 < B / 32) sub_block<BITS, SB + 1>(w, Us, Erow, gr, pk, Qrow, finite);
 }
 
 struct SweepArgs {
@@ -159,14 +163,24 @@ struct SweepArgs {
 
 template <int BITS>
 __global__ void __launch_bounds__(ROWS) sweep_block_kernel(const SweepArgs a, int i0) {
-    extern __shared__ float Us[];  // U[i0:i0+B, i0:i0+B], row-major, then E of one sub-block per thread
-    float* Erow = Us + B * B + threadIdx.x * 33;   // stride 33: conflict-free per-thread rows
-    const float* ub = a.U + size_t(i0) * a.d_in + i0;
-    for (int idx = threadIdx.x * 4; idx < B * B; idx += ROWS * 4) {
-        const int r = idx / B, c = idx % B;
-        *reinterpret_cast<float4*>(Us + idx) = *reinterpret_cast<const float4*>(ub + size_t(r) * a.d_in + c);
+    // U[i0:i0+B, i0:i0+B] row-major, then 1/U[j][j], then one E row per thread
+    extern __shared__ float Us[];
+    float* Erow = Us + B * B + B + threadIdx.x * 33;   // stride 33: conflict-free per-thread rows
+    uint64_t* bar = reinterpret_cast<uint64_t*>(Us + B * B + B + ROWS * 33);  // even float offset: 8-byte aligned
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
     }
     __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(bar, B * B * sizeof(float));
+        const float* ub = a.U + size_t(i0) * a.d_in + i0;
+        for (int j = 0; j < B; ++j) bulk_load(Us + j * B, ub + size_t(j) * a.d_in, B * sizeof(float), bar);
+    }
+    const bool loaded = mbar_wait(bar, 0, a.st, 201);
+    for (int j = threadIdx.x; j < B; j += ROWS) Us[B * B + j] = 1.0f / Us[j * B + j];
+    __syncthreads();
+    if (!loaded) return;
     const int r = blockIdx.x * ROWS + threadIdx.x;
     if (r >= a.d_out) return;
 
@@ -209,7 +223,8 @@ __global__ void __launch_bounds__(ROWS) sweep_block_kernel(const SweepArgs a, in
 
     Packer<BITS> pk;
     float* Qrow = a.Q ? a.Q + size_t(r) * a.d_in + i0 : nullptr;
-    sub_block<BITS, 0>(w, Us, Erow, s, z, a.maxq, pk, Qrow, finite);
+    const Grid gr{s, 1.0f / s, z, a.maxq};
+    sub_block<BITS, 0>(w, Us, Erow, gr, pk, Qrow, finite);
     if (!finite) record_error(a.st, GPTQ_ERR_NONFINITE, r);
 
     pk.store(a.codes + size_t(r) * (size_t(a.d_in) * BITS / 32) + size_t(i0) * BITS / 32);
