@@ -47,6 +47,7 @@ int encode_fn(PFN_encodeTiled* out) {
             q != cudaDriverEntryPointSuccess || fn == nullptr)
             return GPTQ_ERR_CUDA;
         g_encode = reinterpret_cast<PFN_encodeTiled>(fn);
+        set_tensor_map_encoder(g_encode);
     }
     *out = g_encode;
     return GPTQ_OK;
@@ -116,7 +117,8 @@ int gptq_prepare_hinv(const float* H, int64_t d_in, float percdamp, float* U, in
     if (ws_bytes < factor_workspace_bytes(d_in)) return GPTQ_ERR_INVALID_ARG;
     if (info_dev && (reinterpret_cast<uintptr_t>(info_dev) & 3u)) return GPTQ_ERR_INVALID_ARG;
     DevStatus* st = nullptr;
-    if (status_ptr(&st)) return GPTQ_ERR_CUDA;
+    PFN_encodeTiled enc = nullptr;
+    if (status_ptr(&st) || encode_fn(&enc)) return GPTQ_ERR_CUDA;
     return launch_prepare_hinv(H, d_in, percdamp, U, info_dev, ws, static_cast<cudaStream_t>(stream), st);
 }
 
@@ -137,7 +139,8 @@ int gptq_quantize_layer(float* W, int64_t d_out, int64_t d_in, const float* U, i
         return GPTQ_ERR_INVALID_ARG;
     if (ws_bytes < sweep_workspace_bytes(d_out, d_in)) return GPTQ_ERR_INVALID_ARG;
     DevStatus* st = nullptr;
-    if (status_ptr(&st)) return GPTQ_ERR_CUDA;
+    PFN_encodeTiled enc = nullptr;
+    if (status_ptr(&st) || encode_fn(&enc)) return GPTQ_ERR_CUDA;
     return launch_quantize(W, d_out, d_in, U, bits, groupsize, codes, scales, zeros, Q, ws,
                            static_cast<cudaStream_t>(stream), st);
 }

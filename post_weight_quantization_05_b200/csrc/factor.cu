@@ -90,51 +90,62 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const fl
 constexpr int SB = 32;
 constexpr unsigned FULL = 0xffffffffu;
 
-// Warp-level Cholesky of the 32 x 32 sub-block at S[o.., o..] and its
-// inverse into Y[o.., o..].  Returns the failing column (0..31) or -1.
-__device__ __forceinline__ int warp_chol32(float* S, float* Y, int o, int lane) {
-    float a[SB];
-#pragma unroll
-    for (int j = 0; j < SB; ++j) a[j] = (j <= lane) ? S[(o + lane) * LD + o + j] : 0.0f;
-    int bad = -1;
-#pragma unroll
-    for (int c = 0; c < SB; ++c) {
-        const float piv = __shfl_sync(FULL, a[c], c);      // warp-uniform
-        if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) bad = c;
+// The 32 x 32 pieces are written as template recursions so that every
+// register index is a compile-time constant (a rolled or partly unrolled loop
+// would put the row in local memory).
+
+// Cholesky of a 32 x 32 block, one row per lane in a[] (a[j] = 0 for j > lane).
+// `bad` gets the first column whose pivot is not positive and finite.
+template <int C>
+struct Chol32 {
+    __device__ __forceinline__ static void run(float (&a)[SB], int lane, int& bad) {
+        const float piv = __shfl_sync(FULL, a[C], C);    // warp-uniform
+        if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) bad = C;
         const float lcc = sqrtf(piv);
-        const float v = (lane == c) ? lcc : __fdiv_rn(a[c], lcc);   // lanes < c hold 0
-        a[c] = v;
+        const float inv = 1.0f / lcc;
+        const float v = (lane == C) ? lcc : a[C] * inv;  // lanes < C hold 0
+        a[C] = v;
 #pragma unroll
-        for (int j = c + 1; j < SB; ++j) {
-            const float ljc = __shfl_sync(FULL, v, j);     // L[j][c]
-            if (lane >= j) a[j] = fmaf(-v, ljc, a[j]);
+        for (int j = C + 1; j < SB; ++j) {
+            const float ljc = __shfl_sync(FULL, v, j);   // L[j][C]
+            const float upd = fmaf(-v, ljc, a[j]);
+            a[j] = (lane >= j) ? upd : a[j];
         }
+        if constexpr (C + 1 < SB) Chol32<C + 1>::run(a, lane, bad);
     }
+};
+
+// Inverse of a 32 x 32 lower-triangular L (row `lane` in a[]): forward
+// substitution on the identity, row `lane` of L^-1 into x[].
+template <int I>
+struct Inv32 {
+    __device__ __forceinline__ static void run(const float (&a)[SB], float (&x)[SB], int lane) {
+        const float inv = 1.0f / __shfl_sync(FULL, a[I], I);
+        const float lri = a[I];
 #pragma unroll
-    for (int j = 0; j < SB; ++j)
-        if (j <= lane) S[(o + lane) * LD + o + j] = a[j];
-    // inverse: forward substitution on the identity, lane = row
-    float x[SB];
-#pragma unroll
-    for (int j = 0; j < SB; ++j) x[j] = (j == lane) ? 1.0f : 0.0f;
-#pragma unroll
-    for (int i = 0; i < SB; ++i) {
-        const float inv = __fdiv_rn(1.0f, __shfl_sync(FULL, a[i], i));
-        if (lane == i) {
-#pragma unroll
-            for (int j = 0; j <= i; ++j) x[j] *= inv;
+        for (int j = 0; j <= I; ++j) {
+            const float xi = (lane == I) ? x[j] * inv : x[j];
+            const float xij = __shfl_sync(FULL, xi, I);
+            const float upd = fmaf(-lri, xij, xi);
+            x[j] = (lane > I) ? upd : xi;
         }
-        const float lri = a[i];                            // L[lane][i]
-#pragma unroll
-        for (int j = 0; j <= i; ++j) {
-            const float xij = __shfl_sync(FULL, x[j], i);
-            if (lane > i) x[j] = fmaf(-lri, xij, x[j]);
-        }
+        if constexpr (I + 1 < SB) Inv32<I + 1>::run(a, x, lane);
     }
+};
+
+// One row a[] (32 values) solved against L (32 x 32 lower, in shared memory
+// with row stride LD):  a <- a L^-T  (right-looking, invd[c] = 1/L[c][c]).
+template <int C>
+struct Trsm32 {
+    __device__ __forceinline__ static void run(float (&a)[SB], const float* __restrict__ L,
+                                               const float* __restrict__ invd) {
+        const float xc = a[C] * invd[C];
+        a[C] = xc;
 #pragma unroll
-    for (int j = 0; j < SB; ++j) Y[(o + lane) * LD + o + j] = (j <= lane) ? x[j] : 0.0f;
-    return bad;
-}
+        for (int j = C + 1; j < SB; ++j) a[j] = fmaf(-xc, L[j * LD + C], a[j]);
+        if constexpr (C + 1 < SB) Trsm32<C + 1>::run(a, L, invd);
+    }
+};
 
 // Factor the diagonal block A[k0:k0+NB, k0:k0+NB] = L L^T in place (lower) and
 // write its inverse L^-1 to Dinv (NB x NB, row-major).  A non-positive or
@@ -144,6 +155,7 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     extern __shared__ float sm[];
     float* S = sm;             // [NB][LD] factor (upper part used as scratch)
     float* Y = sm + NB * LD;   // [NB][LD] inverse
+    __shared__ float invd[NB];
     __shared__ int failed;
     if (*info != 0) return;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -158,7 +170,16 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     for (int kb = 0; kb < NB / SB; ++kb) {
         const int o = kb * SB;
         if (warp == 0) {
-            const int bad = warp_chol32(S, Y, o, lane);
+            float a[SB];
+#pragma unroll
+            for (int j = 0; j < SB; ++j) a[j] = (j <= lane) ? S[(o + lane) * LD + o + j] : 0.0f;
+            int bad = -1;
+            Chol32<0>::run(a, lane, bad);
+#pragma unroll
+            for (int j = 0; j < SB; ++j)
+                if (j <= lane) S[(o + lane) * LD + o + j] = a[j];
+            __syncwarp();
+            invd[o + lane] = 1.0f / S[(o + lane) * LD + o + lane];
             if (bad >= 0 && lane == 0) {
                 failed = 1;
                 const float p = S[(o + bad) * LD + o + bad];
@@ -170,39 +191,17 @@ __global__ void __launch_bounds__(DIAG_THREADS)
         if (failed) return;
         const int below = NB - o - SB;
         if (below == 0) break;
-        // solve the sub-blocks below: S[R][o..o+32) <- S[R][o..o+32) * Linv_kk^T
-        {
-            float out[2][8];
-            const int cg = t & 3;
+        // solve the rows below against this sub-block: S[r][o..o+32) <- S[r][o..o+32) L_kk^-T
+        if (t < below) {
+            const int r = o + SB + t;
+            float a[SB];
 #pragma unroll
-            for (int it = 0; it < 2; ++it) {
-                const int r = o + SB + (t >> 2) + 64 * it;
-                if (r < NB) {
-                    float in[SB];
+            for (int k = 0; k < SB; ++k) a[k] = S[r * LD + o + k];
+            Trsm32<0>::run(a, S + o * LD + o, invd + o);
 #pragma unroll
-                    for (int k = 0; k < SB; ++k) in[k] = S[r * LD + o + k];
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        const int c = cg * 8 + cc;
-                        float acc = 0.0f;
-#pragma unroll
-                        for (int k = 0; k < SB; ++k)
-                            if (k <= c) acc = fmaf(in[k], Y[(o + c) * LD + o + k], acc);
-                        out[it][cc] = acc;
-                    }
-                }
-            }
-            __syncthreads();
-#pragma unroll
-            for (int it = 0; it < 2; ++it) {
-                const int r = o + SB + (t >> 2) + 64 * it;
-                if (r < NB) {
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) S[r * LD + o + cg * 8 + cc] = out[it][cc];
-                }
-            }
-            __syncthreads();
+            for (int k = 0; k < SB; ++k) S[r * LD + o + k] = a[k];
         }
+        __syncthreads();
         // trailing update of the sub-blocks (bi, bj), kb < bj <= bi
         {
             const int i = t >> 3, j4 = (t & 7) * 4;
@@ -226,7 +225,22 @@ __global__ void __launch_bounds__(DIAG_THREADS)
         __syncthreads();
     }
 
-    // off-diagonal sub-blocks of L^-1:  Y[bi][bj] = -Y[bi][bi] * sum_{k=bj}^{bi-1} L[bi][k] Y[k][bj]
+    // inverse: the four diagonal sub-blocks in parallel (warps 0..3) ...
+    if (warp < NB / SB) {
+        const int o = warp * SB;
+        float a[SB], x[SB];
+#pragma unroll
+        for (int j = 0; j < SB; ++j) {
+            a[j] = (j <= lane) ? S[(o + lane) * LD + o + j] : 0.0f;
+            x[j] = (j == lane) ? 1.0f : 0.0f;
+        }
+        Inv32<0>::run(a, x, lane);
+#pragma unroll
+        for (int j = 0; j < SB; ++j) Y[(o + lane) * LD + o + j] = (j <= lane) ? x[j] : 0.0f;
+    }
+    __syncthreads();
+
+    // ... then the off-diagonal ones:  Y[bi][bj] = -Y[bi][bi] * sum_{k=bj}^{bi-1} L[bi][k] Y[k][bj]
     // T[bj] is kept in the (unused) strictly upper sub-blocks (0, 1 + bj) of S.
     {
         const int i = t >> 3, j4 = (t & 7) * 4;
@@ -263,26 +277,34 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     }
 }
 
-// Y[k*NB + r][k*NB + c] = Dinv_k[r][c] for every diagonal block k.
-__global__ void place_diag_inverses_kernel(const float* __restrict__ Dinv, int d, float* __restrict__ Y) {
+// Z[k*NB + c][k*NB + r] = Dinv_k[r][c]: the diagonal blocks of Z = L^-T.
+__global__ void place_diag_inverses_t_kernel(const float* __restrict__ Dinv, int d, float* __restrict__ Z) {
     const int k = blockIdx.x;
     for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
         const int r = idx / NB, c = idx % NB;
-        Y[size_t(k * NB + r) * d + k * NB + c] = Dinv[size_t(k) * NB * NB + idx];
+        Z[size_t(k * NB + c) * d + k * NB + r] = Dinv[size_t(k) * NB * NB + idx];
     }
 }
 
-// U[r][c] = Y[d-1-r][d-1-c] for r <= c, 0 below the diagonal; NaN everywhere
-// if the factorization failed.
-__global__ void write_u_kernel(const float* __restrict__ Y, int d, const int* __restrict__ info, float* __restrict__ U) {
+// U[r][c] = Z[d-1-c][d-1-r] for r <= c (U = P L'^-1 P = P Z^T P), 0 below the
+// diagonal; NaN everywhere if the factorization failed.  32 x 32 tiles are
+// transposed through shared memory so that both sides stay coalesced.
+__global__ void write_u_kernel(const float* __restrict__ Z, int d, const int* __restrict__ info,
+                               float* __restrict__ U) {
+    __shared__ float tile[32][33];
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
     const bool bad = *info != 0;
-    const size_t total = size_t(d) * d;
-    for (size_t idx = size_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += size_t(gridDim.x) * blockDim.x) {
-        const int r = int(idx / d), c = int(idx % d);
-        float v = (c >= r) ? Y[size_t(d - 1 - r) * d + (d - 1 - c)] : 0.0f;
+    const bool below = c0 + 31 < r0;    // tile entirely in the strict lower triangle
+    if (!below && !bad) {
+        for (int cc = threadIdx.y; cc < 32; cc += blockDim.y)
+            tile[cc][threadIdx.x] = Z[size_t(d - 1 - (c0 + cc)) * d + (d - 1 - (r0 + threadIdx.x))];
+    }
+    __syncthreads();
+    for (int rr = threadIdx.y; rr < 32; rr += blockDim.y) {
+        const int r = r0 + rr, c = c0 + threadIdx.x;
+        float v = (!below && c >= r) ? tile[threadIdx.x][rr] : 0.0f;
         if (bad) v = __int_as_float(0x7fc00000);
-        U[idx] = v;
+        U[size_t(r) * d + c] = v;
     }
 }
 
@@ -297,7 +319,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     const Layout L = layout(d64);
     uint8_t* base = static_cast<uint8_t*>(ws);
     float* A = reinterpret_cast<float*>(base + L.a_off);
-    float* Y = reinterpret_cast<float*>(base + L.y_off);
+    float* Z = reinterpret_cast<float*>(base + L.y_off);
     float* Dinv = reinterpret_cast<float*>(base + L.dinv_off);
     float* lam = reinterpret_cast<float*>(base + L.scal_off);
     int* info = info_user ? info_user : reinterpret_cast<int*>(base + L.scal_off + 64);
@@ -317,7 +339,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     damp_lambda_kernel<<<1, 1024, 0, stream>>>(H, d, percdamp, lam, info, st); count_launch();
     reverse_damp_kernel<<<ew_blocks, 256, 0, stream>>>(H, d, lam, A); count_launch();
 
-    // Cholesky of A (lower), blocked right-looking.
+    // Cholesky of A (lower), blocked right-looking; products on the tensor cores.
     for (int k = 0; k < nblk; ++k) {
         const int k0 = k * NB;
         potrf_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, stream>>>(A, d, k0, Dinv + size_t(k) * NB * NB, info, st); count_launch();
@@ -325,42 +347,44 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         if (rest <= 0) break;
         float* panel = A + size_t(k0 + NB) * d + k0;
         // panel <- panel * Dinv_k^T.  In place is safe: N = NB is one output
-        // tile column, so each CTA reads only the rows it writes.
-        int rc = launch_sgemm(rest, NB, NB, 1.0f, panel, d, Dinv + size_t(k) * NB * NB, NB, true, 0.0f, panel,
-                              panel, d, false, stream);
+        // tile column, so each CTA reads only the rows it writes, all before
+        // its epilogue.
+        int rc = launch_tgemm(rest, NB, NB, 1.0f, panel, d, Dinv + size_t(k) * NB * NB, NB, true, 0.0f, panel,
+                              panel, d, false, stream, st);
         if (rc) return rc;
         float* trail = A + size_t(k0 + NB) * d + k0 + NB;
-        rc = launch_sgemm(rest, rest, NB, -1.0f, panel, d, panel, d, true, 1.0f, trail, trail, d, true, stream);
+        rc = launch_tgemm(rest, rest, NB, -1.0f, panel, d, panel, d, true, 1.0f, trail, trail, d, true, stream, st);
         if (rc) return rc;
     }
 
-    // Y = L^-1, right-looking block forward substitution on the identity.
+    // Z = L^-T (upper), i.e. the transpose of the block forward substitution
+    // Y = L^-1: for each block i,  Z[0:i0, i] <- Z[0:i0, i] Dinv_i^T,  then
+    // Z[0:i0+NB, i0+NB:] -= Z[0:i0+NB, i] L[i0+NB:, i]^T.  Working on Z keeps
+    // every tensor-core operand K-major.
     {
-        const int rc = launch_fill(Y, int64_t(d) * d, 0.0f, stream);
+        const int rc = launch_fill(Z, int64_t(d) * d, 0.0f, stream);
         if (rc) return rc;
     }
-    place_diag_inverses_kernel<<<nblk, 256, 0, stream>>>(Dinv, d, Y); count_launch();
+    place_diag_inverses_t_kernel<<<nblk, 256, 0, stream>>>(Dinv, d, Z); count_launch();
     for (int i = 0; i < nblk; ++i) {
         const int i0 = i * NB;
         int rc;
         if (i > 0) {
-            // Y[i, 0:i0] <- Dinv_i * Y[i, 0:i0].  In place is safe: M = NB is one
-            // output tile row, so each CTA reads only the columns it writes.
-            float* yi = Y + size_t(i0) * d;
-            rc = launch_sgemm(NB, i0, NB, 1.0f, Dinv + size_t(i) * NB * NB, NB, yi, d, false, 0.0f, yi, yi, d,
-                              false, stream);
+            // in place is safe for the same reason as the panel above
+            float* zi = Z + i0;
+            rc = launch_tgemm(i0, NB, NB, 1.0f, zi, d, Dinv + size_t(i) * NB * NB, NB, true, 0.0f, zi, zi, d,
+                              false, stream, st);
             if (rc) return rc;
         }
         const int below = d - i0 - NB;
         if (below > 0) {
-            // Y[i0+NB:, 0:i0+NB] -= L[i0+NB:, i0:i0+NB] * Y[i0:i0+NB, 0:i0+NB]
-            float* yb = Y + size_t(i0 + NB) * d;
-            rc = launch_sgemm(below, i0 + NB, NB, -1.0f, A + size_t(i0 + NB) * d + i0, d, Y + size_t(i0) * d, d,
-                              false, 1.0f, yb, yb, d, false, stream);
+            float* zc = Z + i0 + NB;
+            rc = launch_tgemm(i0 + NB, below, NB, -1.0f, Z + i0, d, A + size_t(i0 + NB) * d + i0, d, true, 1.0f,
+                              zc, zc, d, false, stream, st);
             if (rc) return rc;
         }
     }
-    write_u_kernel<<<ew_blocks, 256, 0, stream>>>(Y, d, info, U); count_launch();
+    write_u_kernel<<<dim3(d / 32, d / 32), dim3(32, 8), 0, stream>>>(Z, d, info, U); count_launch();
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 

@@ -22,13 +22,16 @@ typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_
 int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, void* ws, cudaStream_t stream,
                    DevStatus* st, PFN_encodeTiled encode);
 
-// gemm.cu: C[M,N] = alpha * A[M,K] * op(B)[K,N] + beta * C, fp32, row-major.
-// trans_b = false: B(k, n) = B[k * ldb + n];  true: B(k, n) = B[n * ldb + k].
-// lower_only: skip 128x128 output tiles whose rows all lie above the diagonal
-// (tile entirely in the strict upper triangle: n0 > m0 + 127).
-// C_out may differ from C_in (beta applies to C_in); they may also alias.
-int launch_sgemm(int M, int N, int K, float alpha, const float* A, int lda, const float* B, int ldb, bool trans_b,
-                 float beta, const float* C_in, float* C_out, int ldc, bool lower_only, cudaStream_t stream);
+// tgemm.cu: C[M,N] = alpha * A[M,K] * B + beta * C_in with B(k, n) =
+// Bt[n * ldb + k] (trans_b must be true), fp32 row-major, on the tensor cores
+// (kind::tf32, hi/lo split, three passes; fp32-class accuracy).  K must be a
+// multiple of 32; pointers and leading dimensions must satisfy TMA's 16-byte
+// rules.  lower_only skips 128 x 128 output tiles entirely above the
+// diagonal.  C_out may alias C_in.
+void set_tensor_map_encoder(PFN_encodeTiled f);
+int launch_tgemm(int M, int N, int K, float alpha, const float* A, int lda, const float* B, int ldb, bool trans_b,
+                 float beta, const float* C_in, float* C_out, int ldc, bool lower_only, cudaStream_t stream,
+                 DevStatus* st);
 
 // factor.cu
 size_t factor_workspace_bytes(int64_t d);

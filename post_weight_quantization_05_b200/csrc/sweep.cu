@@ -277,8 +277,21 @@ __global__ void fill_kernel(float* __restrict__ p, size_t n, float v) {
         p[i] = v;
 }
 
+// Ut[c][r] = U[r][c] for the tiles of U that reach the upper triangle (the
+// trailing products read U's rows as K-major operands through Ut).
+__global__ void transpose_upper_kernel(const float* __restrict__ U, int d, float* __restrict__ Ut) {
+    __shared__ float tile[32][33];
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    if (c0 + 31 < r0) return;
+    for (int rr = threadIdx.y; rr < 32; rr += blockDim.y)
+        tile[rr][threadIdx.x] = U[size_t(r0 + rr) * d + c0 + threadIdx.x];
+    __syncthreads();
+    for (int cc = threadIdx.y; cc < 32; cc += blockDim.y)
+        Ut[size_t(c0 + cc) * d + r0 + threadIdx.x] = tile[threadIdx.x][cc];
+}
+
 template <int BITS>
-int run_sweep(const SweepArgs& a, cudaStream_t stream) {
+int run_sweep(const SweepArgs& a, const float* Ut, cudaStream_t stream) {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -293,10 +306,10 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
         sweep_block_kernel<BITS><<<blocks, ROWS, SMEM, stream>>>(a, i0); count_launch();
         const int tail = a.d_in - i0 - B;
         if (tail > 0) {
-            // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]
+            // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]   (U[i0+k][i0+B+n] = Ut[i0+B+n][i0+k])
             float* c = a.W + i0 + B;
-            const int rc = launch_sgemm(a.d_out, tail, B, -1.0f, a.E, B, a.U + size_t(i0) * a.d_in + i0 + B, a.d_in,
-                                        false, 1.0f, c, c, a.d_in, false, stream);
+            const int rc = launch_tgemm(a.d_out, tail, B, -1.0f, a.E, B, Ut + size_t(i0 + B) * a.d_in + i0, a.d_in,
+                                        true, 1.0f, c, c, a.d_in, false, stream, a.st);
             if (rc) return rc;
         }
     }
@@ -305,9 +318,10 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
 
 }  // namespace sweep
 
+// E [d_out, B] fp32, then U^T [d_in, d_in] fp32 (256-byte aligned)
 size_t sweep_workspace_bytes(int64_t d_out, int64_t d_in) {
-    (void)d_in;
-    return size_t(d_out) * sweep::B * sizeof(float);
+    const size_t e = (size_t(d_out) * sweep::B * sizeof(float) + 255) & ~size_t(255);
+    return e + size_t(d_in) * size_t(d_in) * sizeof(float);
 }
 
 int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int bits, int groupsize,
@@ -333,11 +347,15 @@ int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int b
         grid_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(W, a.d_out, a.d_in, a.d_in, 1, a.maxq, scales,
                                                                   zeros, st); count_launch();
     }
+    float* Ut = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                         ((size_t(d_out) * B * sizeof(float) + 255) & ~size_t(255)));
+    transpose_upper_kernel<<<dim3(unsigned(d_in / 32), unsigned(d_in / 32)), dim3(32, 8), 0, stream>>>(U, int(d_in), Ut);
+    count_launch();
     switch (bits) {
-        case 2: return run_sweep<2>(a, stream);
-        case 3: return run_sweep<3>(a, stream);
-        case 4: return run_sweep<4>(a, stream);
-        case 8: return run_sweep<8>(a, stream);
+        case 2: return run_sweep<2>(a, Ut, stream);
+        case 3: return run_sweep<3>(a, Ut, stream);
+        case 4: return run_sweep<4>(a, Ut, stream);
+        case 8: return run_sweep<8>(a, Ut, stream);
         default: return GPTQ_ERR_UNSUPPORTED;
     }
 }
