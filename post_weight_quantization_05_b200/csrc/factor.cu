@@ -18,6 +18,8 @@
 //   SGEMM.  The inverse L'^-1 is then built block row by block row
 //   (right-looking forward substitution on the identity), and U is written
 //   by reversing both indices.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -94,45 +96,6 @@ constexpr unsigned FULL = 0xffffffffu;
 // register index is a compile-time constant (a rolled or partly unrolled loop
 // would put the row in local memory).
 
-// Cholesky of a 32 x 32 block, one row per lane in a[] (a[j] = 0 for j > lane).
-// `bad` gets the first column whose pivot is not positive and finite.
-template <int C>
-struct Chol32 {
-    __device__ __forceinline__ static void run(float (&a)[SB], int lane, int& bad) {
-        const float piv = __shfl_sync(FULL, a[C], C);    // warp-uniform
-        if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) bad = C;
-        const float lcc = sqrtf(piv);
-        const float inv = 1.0f / lcc;
-        const float v = (lane == C) ? lcc : a[C] * inv;  // lanes < C hold 0
-        a[C] = v;
-#pragma unroll
-        for (int j = C + 1; j < SB; ++j) {
-            const float ljc = __shfl_sync(FULL, v, j);   // L[j][C]
-            const float upd = fmaf(-v, ljc, a[j]);
-            a[j] = (lane >= j) ? upd : a[j];
-        }
-        if constexpr (C + 1 < SB) Chol32<C + 1>::run(a, lane, bad);
-    }
-};
-
-// Inverse of a 32 x 32 lower-triangular L (row `lane` in a[]): forward
-// substitution on the identity, row `lane` of L^-1 into x[].
-template <int I>
-struct Inv32 {
-    __device__ __forceinline__ static void run(const float (&a)[SB], float (&x)[SB], int lane) {
-        const float inv = 1.0f / __shfl_sync(FULL, a[I], I);
-        const float lri = a[I];
-#pragma unroll
-        for (int j = 0; j <= I; ++j) {
-            const float xi = (lane == I) ? x[j] * inv : x[j];
-            const float xij = __shfl_sync(FULL, xi, I);
-            const float upd = fmaf(-lri, xij, xi);
-            x[j] = (lane > I) ? upd : xi;
-        }
-        if constexpr (I + 1 < SB) Inv32<I + 1>::run(a, x, lane);
-    }
-};
-
 // One row a[] (32 values) solved against L (32 x 32 lower, in shared memory
 // with row stride LD):  a <- a L^-T  (right-looking, invd[c] = 1/L[c][c]).
 template <int C>
@@ -147,6 +110,53 @@ struct Trsm32 {
     }
 };
 
+// Column-oriented Cholesky of a 32 x 32 block by one warp: lane j holds
+// column j (col[r] = A[r][j]; entries above the diagonal are ignored).  At
+// step C lane C finalizes its column and publishes it through `buf` (shared
+// memory); every later lane then updates its own column with one broadcast
+// read per row -- no shuffles, one short dependency chain per column.
+template <int C>
+struct ColChol32 {
+    __device__ __forceinline__ static void run(float (&col)[SB], int lane, float* __restrict__ buf, int& bad) {
+        if (lane == C) {
+            const float piv = col[C];
+            if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) bad = C;
+            const float lcc = sqrtf(piv);
+            const float inv = 1.0f / lcc;
+            col[C] = lcc;
+            buf[C] = lcc;
+#pragma unroll
+            for (int r = C + 1; r < SB; ++r) {
+                col[r] *= inv;
+                buf[r] = col[r];
+            }
+        }
+        __syncwarp();
+        if (lane > C) {
+            const float ljc = buf[lane];                  // L[lane][C]
+#pragma unroll
+            for (int r = C + 1; r < SB; ++r) col[r] = fmaf(-buf[r], ljc, col[r]);
+        }
+        __syncwarp();
+        if constexpr (C + 1 < SB) ColChol32<C + 1>::run(col, lane, buf, bad);
+    }
+};
+
+// Column-oriented inverse of a 32 x 32 lower-triangular L held in shared
+// memory (row stride LD, 1/L[i][i] in invd): lane j computes column j of
+// L^-1 (y[i] for i >= j) by forward substitution, reading L by broadcast.
+template <int I>
+struct ColInv32 {
+    __device__ __forceinline__ static void run(float (&y)[SB], const float* __restrict__ L,
+                                               const float* __restrict__ invd, int lane) {
+        const float yi = y[I] * invd[I];
+        y[I] = yi;
+#pragma unroll
+        for (int r = I + 1; r < SB; ++r) y[r] = fmaf(-L[r * LD + I], yi, y[r]);
+        if constexpr (I + 1 < SB) ColInv32<I + 1>::run(y, L, invd, lane);
+    }
+};
+
 // Factor the diagonal block A[k0:k0+NB, k0:k0+NB] = L L^T in place (lower) and
 // write its inverse L^-1 to Dinv (NB x NB, row-major).  A non-positive or
 // non-finite pivot sets *info = k0 + c + 1 (first failure only).
@@ -156,6 +166,7 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     float* S = sm;             // [NB][LD] factor (upper part used as scratch)
     float* Y = sm + NB * LD;   // [NB][LD] inverse
     __shared__ float invd[NB];
+    __shared__ float colbuf[SB];
     __shared__ int failed;
     if (*info != 0) return;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -170,17 +181,18 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     for (int kb = 0; kb < NB / SB; ++kb) {
         const int o = kb * SB;
         if (warp == 0) {
-            float a[SB];
+            float col[SB];
 #pragma unroll
-            for (int j = 0; j < SB; ++j) a[j] = (j <= lane) ? S[(o + lane) * LD + o + j] : 0.0f;
+            for (int r = 0; r < SB; ++r) col[r] = (r >= lane) ? S[(o + r) * LD + o + lane] : 0.0f;
             int bad = -1;
-            Chol32<0>::run(a, lane, bad);
+            ColChol32<0>::run(col, lane, colbuf, bad);
 #pragma unroll
-            for (int j = 0; j < SB; ++j)
-                if (j <= lane) S[(o + lane) * LD + o + j] = a[j];
+            for (int r = 0; r < SB; ++r)
+                if (r >= lane) S[(o + r) * LD + o + lane] = col[r];
             __syncwarp();
             invd[o + lane] = 1.0f / S[(o + lane) * LD + o + lane];
-            if (bad >= 0 && lane == 0) {
+            bad = __reduce_min_sync(FULL, bad < 0 ? SB : bad);
+            if (bad < SB && lane == 0) {
                 failed = 1;
                 const float p = S[(o + bad) * LD + o + bad];
                 if (atomicCAS(info, 0, k0 + o + bad + 1) == 0)
@@ -225,18 +237,16 @@ __global__ void __launch_bounds__(DIAG_THREADS)
         __syncthreads();
     }
 
-    // inverse: the four diagonal sub-blocks in parallel (warps 0..3) ...
+    // inverse: the four diagonal sub-blocks in parallel (warps 0..3), one
+    // column of L^-1 per lane ...
     if (warp < NB / SB) {
         const int o = warp * SB;
-        float a[SB], x[SB];
+        float y[SB];
 #pragma unroll
-        for (int j = 0; j < SB; ++j) {
-            a[j] = (j <= lane) ? S[(o + lane) * LD + o + j] : 0.0f;
-            x[j] = (j == lane) ? 1.0f : 0.0f;
-        }
-        Inv32<0>::run(a, x, lane);
+        for (int r = 0; r < SB; ++r) y[r] = (r == lane) ? 1.0f : 0.0f;
+        ColInv32<0>::run(y, S + o * LD + o, invd + o, lane);
 #pragma unroll
-        for (int j = 0; j < SB; ++j) Y[(o + lane) * LD + o + j] = (j <= lane) ? x[j] : 0.0f;
+        for (int r = 0; r < SB; ++r) Y[(o + r) * LD + o + lane] = (r >= lane) ? y[r] : 0.0f;
     }
     __syncthreads();
 
@@ -277,13 +287,38 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     }
 }
 
-// Z[k*NB + c][k*NB + r] = Dinv_k[r][c]: the diagonal blocks of Z = L^-T.
-__global__ void place_diag_inverses_t_kernel(const float* __restrict__ Dinv, int d, float* __restrict__ Z) {
-    const int k = blockIdx.x;
+// Z[k*NB + c][k*NB + r] = Dinv_k[r][c]: diagonal block k of Z = L^-T.
+__global__ void place_diag_inverse_t_kernel(const float* __restrict__ Dinv_k, int d, int k, float* __restrict__ Z) {
     for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
         const int r = idx / NB, c = idx % NB;
-        Z[size_t(k * NB + c) * d + k * NB + r] = Dinv[size_t(k) * NB * NB + idx];
+        Z[size_t(k * NB + c) * d + k * NB + r] = Dinv_k[idx];
     }
+}
+
+// One auxiliary stream and two events per device (created on first use):
+// the inverse's block steps run there, each as soon as the factorization has
+// finished the block column it needs, overlapping the rest of the Cholesky.
+struct AuxStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, step = nullptr, join = nullptr;
+};
+
+static int aux_stream(AuxStream** out) {
+    static std::mutex mu;
+    static AuxStream per_dev[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    AuxStream& a = per_dev[dev];
+    if (!a.s) {
+        if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.step, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+    }
+    *out = &a;
+    return GPTQ_OK;
 }
 
 // U[r][c] = Z[d-1-c][d-1-r] for r <= c (U = P L'^-1 P = P Z^T P), 0 below the
@@ -336,54 +371,68 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         attr_set[dev] = true;
     }
 
+    // One call enqueues at a time (per process): the auxiliary stream and its
+    // events are shared by every call on a device.
+    static std::mutex enqueue_mu;
+    std::lock_guard<std::mutex> enqueue_lock(enqueue_mu);
+    AuxStream* aux = nullptr;
+    if (aux_stream(&aux)) return GPTQ_ERR_CUDA;
+    const cudaStream_t as = aux->s;
+
     damp_lambda_kernel<<<1, 1024, 0, stream>>>(H, d, percdamp, lam, info, st); count_launch();
     reverse_damp_kernel<<<ew_blocks, 256, 0, stream>>>(H, d, lam, A); count_launch();
+    // fork: the inverse (stream `as`) starts from a zeroed Z
+    if (cudaEventRecord(aux->fork, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->fork, 0) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    {
+        const int rc = launch_fill(Z, int64_t(d) * d, 0.0f, as);
+        if (rc) return rc;
+    }
 
-    // Cholesky of A (lower), blocked right-looking; products on the tensor cores.
+    // Cholesky of A (lower), blocked right-looking, on `stream`; products on the
+    // tensor cores.  Z = L^-T (upper) on `as`: block step i needs only L's block
+    // column i and Dinv_i, so it runs as soon as the factorization has them:
+    //   Z[i][i] = Dinv_i^T;  Z[0:i0, i] <- Z[0:i0, i] Dinv_i^T;
+    //   Z[0:i0+NB, i0+NB:] -= Z[0:i0+NB, i] L[i0+NB:, i]^T
+    // (the transpose of the block forward substitution Y = L^-1; working on Z
+    // keeps every tensor-core operand K-major).
     for (int k = 0; k < nblk; ++k) {
         const int k0 = k * NB;
-        potrf_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, stream>>>(A, d, k0, Dinv + size_t(k) * NB * NB, info, st); count_launch();
+        float* dk = Dinv + size_t(k) * NB * NB;
+        potrf_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, stream>>>(A, d, k0, dk, info, st); count_launch();
         const int rest = d - k0 - NB;
-        if (rest <= 0) break;
         float* panel = A + size_t(k0 + NB) * d + k0;
-        // panel <- panel * Dinv_k^T.  In place is safe: N = NB is one output
-        // tile column, so each CTA reads only the rows it writes, all before
-        // its epilogue.
-        int rc = launch_tgemm(rest, NB, NB, 1.0f, panel, d, Dinv + size_t(k) * NB * NB, NB, true, 0.0f, panel,
-                              panel, d, false, stream, st);
-        if (rc) return rc;
-        float* trail = A + size_t(k0 + NB) * d + k0 + NB;
-        rc = launch_tgemm(rest, rest, NB, -1.0f, panel, d, panel, d, true, 1.0f, trail, trail, d, true, stream, st);
-        if (rc) return rc;
-    }
-
-    // Z = L^-T (upper), i.e. the transpose of the block forward substitution
-    // Y = L^-1: for each block i,  Z[0:i0, i] <- Z[0:i0, i] Dinv_i^T,  then
-    // Z[0:i0+NB, i0+NB:] -= Z[0:i0+NB, i] L[i0+NB:, i]^T.  Working on Z keeps
-    // every tensor-core operand K-major.
-    {
-        const int rc = launch_fill(Z, int64_t(d) * d, 0.0f, stream);
-        if (rc) return rc;
-    }
-    place_diag_inverses_t_kernel<<<nblk, 256, 0, stream>>>(Dinv, d, Z); count_launch();
-    for (int i = 0; i < nblk; ++i) {
-        const int i0 = i * NB;
         int rc;
-        if (i > 0) {
-            // in place is safe for the same reason as the panel above
-            float* zi = Z + i0;
-            rc = launch_tgemm(i0, NB, NB, 1.0f, zi, d, Dinv + size_t(i) * NB * NB, NB, true, 0.0f, zi, zi, d,
-                              false, stream, st);
+        if (rest > 0) {
+            // panel <- panel * Dinv_k^T.  In place is safe: N = NB is one output
+            // tile column, so each CTA reads only the rows it writes, all before
+            // its epilogue.
+            rc = launch_tgemm(rest, NB, NB, 1.0f, panel, d, dk, NB, true, 0.0f, panel, panel, d, false, stream, st);
             if (rc) return rc;
         }
-        const int below = d - i0 - NB;
-        if (below > 0) {
-            float* zc = Z + i0 + NB;
-            rc = launch_tgemm(i0 + NB, below, NB, -1.0f, Z + i0, d, A + size_t(i0 + NB) * d + i0, d, true, 1.0f,
-                              zc, zc, d, false, stream, st);
+        if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->step, 0) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        if (rest > 0) {
+            float* trail = A + size_t(k0 + NB) * d + k0 + NB;
+            rc = launch_tgemm(rest, rest, NB, -1.0f, panel, d, panel, d, true, 1.0f, trail, trail, d, true, stream, st);
+            if (rc) return rc;
+        }
+        // inverse block step k on the auxiliary stream
+        place_diag_inverse_t_kernel<<<1, 256, 0, as>>>(dk, d, k, Z); count_launch();
+        if (k > 0) {
+            float* zi = Z + k0;   // in place is safe for the same reason as the panel
+            rc = launch_tgemm(k0, NB, NB, 1.0f, zi, d, dk, NB, true, 0.0f, zi, zi, d, false, as, st);
+            if (rc) return rc;
+        }
+        if (rest > 0) {
+            float* zc = Z + k0 + NB;
+            rc = launch_tgemm(k0 + NB, rest, NB, -1.0f, Z + k0, d, panel, d, true, 1.0f, zc, zc, d, false, as, st);
             if (rc) return rc;
         }
     }
+    // join
+    if (cudaEventRecord(aux->join, as) != cudaSuccess || cudaStreamWaitEvent(stream, aux->join, 0) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
     write_u_kernel<<<dim3(d / 32, d / 32), dim3(32, 8), 0, stream>>>(Z, d, info, U); count_launch();
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }

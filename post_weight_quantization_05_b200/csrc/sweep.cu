@@ -8,17 +8,12 @@
 // (groups share a grid set from the latest updated weights); "문제 설정" (RTN).
 //
 // Sweep kernel design: rows are independent given U (the same U serves every
-// row), so one thread owns one row of the 128-column block: the block's 128
-// weights live in registers, the 128 x 128 diagonal block of U in shared
-// memory (every thread of a warp reads the same U element: broadcast).  The
-// block is walked in four 32-column sub-blocks: inside a sub-block the column
-// loop is unrolled (static register indices); the sub-block's E values are
-// then applied to the later sub-blocks in a rolled loop that reads E back from
-// shared memory -- the same additions in the same order as the plain rank-1
-// sweep, with a quarter of the code.  After column j is quantized its
-// register slot holds E[:, j], and the block's E is written once for the
-// trailing SGEMM.  The codes are packed in registers
-// (compile-time bit positions) and stored as 16-byte vectors.
+// row), so one thread owns one row of the 128-column block, 32 rows per CTA.
+// The 128 x 128 diagonal block of U (and its transpose) is brought into
+// shared memory by bulk copies; every thread of a warp reads the same U
+// element at the same time (broadcast).  The block's E is written for the
+// lazy trailing product on the tensor cores.  The codes are packed in
+// registers (compile-time bit positions) and stored as vectors.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -29,8 +24,6 @@ namespace sweep {
 
 constexpr int B = 128;
 constexpr int ROWS = 32;  // rows (threads) per CTA
-// U block, 1/U[j][j], per-thread E rows; plus one mbarrier
-constexpr size_t SMEM = (size_t(B) * B + B + size_t(ROWS) * 33) * sizeof(float) + 16;
 
 // Per-row grid over columns [c0, c0 + len) of the ORIGINAL W: one warp per
 // (row, group).  Writes fp16 scale/zero bit patterns.
@@ -60,15 +53,25 @@ __global__ void grid_kernel(const float* __restrict__ W, int d_out, int d_in, in
     }
 }
 
-// Bit-stream packer with compile-time positions: code k of the block goes to
-// stream bits [k*BITS, (k+1)*BITS).
+// The 128-column block is walked as four 32-column windows.  A thread's row
+// lives in shared memory; the current window is copied into 32 registers and
+// processed by one fully unrolled body (static register indices), which is
+// the same code for all four windows -- the kernel's hot code stays small
+// enough for the instruction cache.  After a window its E values (still in
+// the registers) update the later columns of the row in shared memory, in
+// column order j = 0..31 per element, i.e. the same additions in the same
+// order as the plain rank-1 sweep.
+constexpr int SUB = 32;
+constexpr int RLD = B + 1;   // per-thread row stride in shared memory (conflict-free columns)
+
+// Packer for one window: code j of the window goes to stream bits
+// [j*BITS, (j+1)*BITS) of the window's BITS words.
 template <int BITS>
 struct Packer {
-    static constexpr int WORDS = B * BITS / 32;
-    uint32_t w[WORDS];
+    uint32_t w[BITS];
     __device__ __forceinline__ Packer() {
 #pragma unroll
-        for (int i = 0; i < WORDS; ++i) w[i] = 0u;
+        for (int i = 0; i < BITS; ++i) w[i] = 0u;
     }
     template <int K>
     __device__ __forceinline__ void put(uint32_t c) {
@@ -77,80 +80,50 @@ struct Packer {
         if constexpr (off + BITS > 32) w[word + 1] |= c >> (32 - off);
     }
     __device__ __forceinline__ void store(uint32_t* dst) const {
+        if constexpr (BITS % 4 == 0) {
 #pragma unroll
-        for (int i = 0; i < WORDS; i += 4)
-            *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
-    }
-};
-
-// Column J of the block: quantize, record code and E, and apply the rank-1
-// correction to the remaining columns of J's 32-column sub-block.
-struct Grid {
-    float s, inv_s, z, maxq;
-};
-
-template <int BITS, int J>
-__device__ __forceinline__ void quant_column(float (&w)[B], const float* __restrict__ Us, float* __restrict__ Erow,
-                                             const Grid& gr, Packer<BITS>& pk, float* Qrow, bool& finite) {
-    constexpr int SUB_END = (J / 32 + 1) * 32;
-    const float wj = w[J];
-    const float c = quant_code(wj, gr.s, gr.z, gr.maxq);
-    const float q = gr.s * (c - gr.z);
-    const float e = (wj - q) * Us[B * B + J];     // 1/U[j][j] kept after the block
-    finite &= isfinite(e);
-    if (Qrow) Qrow[J] = q;
-    pk.template put<J>(static_cast<uint32_t>(c));
-    const float* urow = Us + J * B;
+            for (int i = 0; i < BITS; i += 4)
+                *reinterpret_cast<uint4*>(dst + i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+        } else if constexpr (BITS == 2) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+        } else {
 #pragma unroll
-    for (int k = J + 1; k < SUB_END; ++k) w[k] = fmaf(-e, urow[k], w[k]);
-    w[J] = e;
-    Erow[J % 32] = e;
-}
-
-template <int BITS, int SB, int J>
-struct SubCols {
-    __device__ __forceinline__ static void run(float (&w)[B], const float* Us, float* Erow, const Grid& gr,
-                                               Packer<BITS>& pk, float* Qrow, bool& finite) {
-        quant_column<BITS, SB * 32 + J>(w, Us, Erow, gr, pk, Qrow, finite);
-        if constexpr (J + 1 < 32) SubCols<BITS, SB, J + 1>::run(w, Us, Erow, gr, pk, Qrow, finite);
-    }
-};
-
-// Updates of sub-block SB's 32 columns to the later sub-block SBK, in column
-// order j = 0..31 (the same order in which the plain rank-1 sweep applies
-// them), with E read back from shared memory so that j can be a loop index.
-template <int SB, int SBK>
-__device__ __forceinline__ void cross_update(float (&w)[B], const float* __restrict__ Us,
-                                             const float* __restrict__ Erow) {
-#pragma unroll 1
-    for (int j = 0; j < 32; ++j) {
-        const float e = Erow[j];
-        const float* urow = Us + (SB * 32 + j) * B + SBK * 32;
-#pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-            const float4 u = *reinterpret_cast<const float4*>(urow + k);
-            w[SBK * 32 + k + 0] = fmaf(-e, u.x, w[SBK * 32 + k + 0]);
-            w[SBK * 32 + k + 1] = fmaf(-e, u.y, w[SBK * 32 + k + 1]);
-            w[SBK * 32 + k + 2] = fmaf(-e, u.z, w[SBK * 32 + k + 2]);
-            w[SBK * 32 + k + 3] = fmaf(-e, u.w, w[SBK * 32 + k + 3]);
+            for (int i = 0; i < BITS; ++i) dst[i] = w[i];
         }
     }
-}
+};
 
-template <int BITS, int SB>
-__device__ __forceinline__ void sub_block(float (&w)[B], const float* Us, float* Erow, const Grid& gr,
-                                          Packer<BITS>& pk, float* Qrow, bool& finite) {
-    // Erow is private to this thread: no synchronization needed around it.
-    SubCols<BITS, SB, 0>::run(w, Us, Erow, gr, pk, Qrow, finite);
-    if constexpr (SB < 1) cross_update<SB, 1>(w, Us, Erow);
-    if constexpr (SB < 2) cross_update<SB, 2>(w, Us, Erow);
-    if constexpr (SB < 3) cross_update<SB, 3>(w, Us, Erow);
-    if constexpr (SB + 1 < B / 32) sub_block<BITS, SB + 1>(w, Us, Erow, gr, pk, Qrow, finite);
-}
+struct Grid {
+    float s, z, maxq;
+};
+
+// Column J of the window: quantize, pack, E = (w - q) / U_jj, and the rank-1
+// correction of the window's later columns.  `urow` = U row of this column,
+// offset to the window's first column.
+template <int BITS, int J>
+struct WindowCol {
+    __device__ __forceinline__ static void run(float (&w)[SUB], const float* __restrict__ Us, int wc,
+                                               const float* __restrict__ invd, const Grid& gr, Packer<BITS>& pk,
+                                               float* Qw, bool& finite) {
+        const float wj = w[J];
+        const float c = quant_code(wj, gr.s, gr.z, gr.maxq);
+        const float q = gr.s * (c - gr.z);
+        const float e = (wj - q) * invd[wc + J];
+        finite &= isfinite(e);
+        if (Qw) Qw[J] = q;
+        pk.template put<J>(static_cast<uint32_t>(c));
+        const float* urow = Us + (wc + J) * B + wc;
+#pragma unroll
+        for (int k = J + 1; k < SUB; ++k) w[k] = fmaf(-e, urow[k], w[k]);
+        w[J] = e;
+        if constexpr (J + 1 < SUB) WindowCol<BITS, J + 1>::run(w, Us, wc, invd, gr, pk, Qw, finite);
+    }
+};
 
 struct SweepArgs {
     float* W;
     const float* U;
+    const float* Ut;
     int d_out, d_in, groupsize, n_groups;
     float maxq;
     uint32_t* codes;
@@ -161,76 +134,106 @@ struct SweepArgs {
     DevStatus* st;
 };
 
+// shared memory: U block (row-major), U block transposed, 1/U_jj, rows, mbarrier
+constexpr size_t SMEM = (size_t(2) * B * B + B + size_t(ROWS) * RLD) * sizeof(float) + 16;
+
 template <int BITS>
 __global__ void __launch_bounds__(ROWS) sweep_block_kernel(const SweepArgs a, int i0) {
-    // U[i0:i0+B, i0:i0+B] row-major, then 1/U[j][j], then one E row per thread
-    extern __shared__ float Us[];
-    float* Erow = Us + B * B + B + threadIdx.x * 33;   // stride 33: conflict-free per-thread rows
-    uint64_t* bar = reinterpret_cast<uint64_t*>(Us + B * B + B + ROWS * 33);  // even float offset: 8-byte aligned
+    extern __shared__ float sm[];
+    float* Us = sm;                          // Us[j][k]  = U[i0+j][i0+k]
+    float* UtS = sm + B * B;                 // UtS[k][j] = U[i0+j][i0+k]
+    float* invd = UtS + B * B;               // 1 / U[i0+j][i0+j]
+    float* rows = invd + B;                  // per-thread row, stride RLD
+    uint64_t* bar = reinterpret_cast<uint64_t*>(rows + ROWS * RLD);   // even float offset: 8-byte aligned
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(bar, B * B * sizeof(float));
+        mbar_arrive_expect_tx(bar, 2 * B * B * sizeof(float));
         const float* ub = a.U + size_t(i0) * a.d_in + i0;
-        for (int j = 0; j < B; ++j) bulk_load(Us + j * B, ub + size_t(j) * a.d_in, B * sizeof(float), bar);
+        const float* utb = a.Ut + size_t(i0) * a.d_in + i0;
+        for (int j = 0; j < B; ++j) {
+            bulk_load(Us + j * B, ub + size_t(j) * a.d_in, B * sizeof(float), bar);
+            bulk_load(UtS + j * B, utb + size_t(j) * a.d_in, B * sizeof(float), bar);
+        }
+    }
+    const int r = blockIdx.x * ROWS + threadIdx.x;
+    const bool active = r < a.d_out;
+    float* myrow = rows + threadIdx.x * RLD;
+    const float* wsrc = a.W + size_t(active ? r : 0) * a.d_in + i0;
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll 4
+    for (int k = 0; k < B; k += 4) {
+        const float4 v = active ? *reinterpret_cast<const float4*>(wsrc + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+        myrow[k] = v.x; myrow[k + 1] = v.y; myrow[k + 2] = v.z; myrow[k + 3] = v.w;
+        mn = fminf(fminf(mn, v.x), fminf(v.y, fminf(v.z, v.w)));
+        mx = fmaxf(fmaxf(mx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
     }
     const bool loaded = mbar_wait(bar, 0, a.st, 201);
-    for (int j = threadIdx.x; j < B; j += ROWS) Us[B * B + j] = 1.0f / Us[j * B + j];
+    for (int j = threadIdx.x; j < B; j += ROWS) invd[j] = 1.0f / Us[j * B + j];
     __syncthreads();
-    if (!loaded) return;
-    const int r = blockIdx.x * ROWS + threadIdx.x;
-    if (r >= a.d_out) return;
+    if (!loaded || !active) return;
 
-    float w[B];
-    float* wrow = a.W + size_t(r) * a.d_in + i0;
-#pragma unroll
-    for (int k = 0; k < B; k += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(wrow + k);
-        w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
-    }
-
-    float s, z;
+    Grid gr;
+    gr.maxq = a.maxq;
     bool finite = true;
     if (a.groupsize < 0) {
-        s = __half2float(__ushort_as_half(a.scales[r]));
-        z = __half2float(__ushort_as_half(a.zeros[r]));
+        gr.s = __half2float(__ushort_as_half(a.scales[r]));
+        gr.z = __half2float(__ushort_as_half(a.zeros[r]));
     } else {
-        const int g = i0 / a.groupsize;
-        const size_t gi = size_t(r) * a.n_groups + g;
+        const size_t gi = size_t(r) * a.n_groups + i0 / a.groupsize;
         if (i0 % a.groupsize == 0) {
-            // grid from the current weights of the group (this block's columns
-            // from registers, later columns from W, already lazily updated)
-            float mn = w[0], mx = w[0];
-#pragma unroll
-            for (int k = 1; k < B; ++k) { mn = fminf(mn, w[k]); mx = fmaxf(mx, w[k]); }
+            // grid from the current weights of the group: this block's columns as
+            // loaded, later columns from W (already lazily updated)
             for (int c = B; c < a.groupsize; c += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(wrow + c);
+                const float4 v = *reinterpret_cast<const float4*>(wsrc + c);
                 mn = fminf(fminf(mn, v.x), fminf(v.y, fminf(v.z, v.w)));
                 mx = fmaxf(fmaxf(mx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
             }
             __half s16, z16;
-            finite &= grid_params(mn, mx, a.maxq, s, z, s16, z16);
+            finite &= grid_params(mn, mx, a.maxq, gr.s, gr.z, s16, z16);
             a.scales[gi] = __half_as_ushort(s16);
             a.zeros[gi] = __half_as_ushort(z16);
         } else {
-            s = __half2float(__ushort_as_half(a.scales[gi]));
-            z = __half2float(__ushort_as_half(a.zeros[gi]));
+            gr.s = __half2float(__ushort_as_half(a.scales[gi]));
+            gr.z = __half2float(__ushort_as_half(a.zeros[gi]));
         }
     }
 
-    Packer<BITS> pk;
-    float* Qrow = a.Q ? a.Q + size_t(r) * a.d_in + i0 : nullptr;
-    const Grid gr{s, 1.0f / s, z, a.maxq};
-    sub_block<BITS, 0>(w, Us, Erow, gr, pk, Qrow, finite);
-    if (!finite) record_error(a.st, GPTQ_ERR_NONFINITE, r);
-
-    pk.store(a.codes + size_t(r) * (size_t(a.d_in) * BITS / 32) + size_t(i0) * BITS / 32);
+    uint32_t* crow = a.codes + size_t(r) * (size_t(a.d_in) * BITS / 32) + size_t(i0) * BITS / 32;
     float* erow = a.E + size_t(r) * B;
+    float* qrow = a.Q ? a.Q + size_t(r) * a.d_in + i0 : nullptr;
+#pragma unroll 1
+    for (int sb = 0; sb < B / SUB; ++sb) {
+        const int wc = sb * SUB;
+        float w[SUB];
 #pragma unroll
-    for (int k = 0; k < B; k += 4) *reinterpret_cast<float4*>(erow + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+        for (int j = 0; j < SUB; ++j) w[j] = myrow[wc + j];
+        Packer<BITS> pk;
+        WindowCol<BITS, 0>::run(w, Us, wc, invd, gr, pk, qrow ? qrow + wc : nullptr, finite);
+        pk.store(crow + sb * BITS);
+#pragma unroll
+        for (int j = 0; j < SUB; j += 4)
+            *reinterpret_cast<float4*>(erow + wc + j) = make_float4(w[j], w[j + 1], w[j + 2], w[j + 3]);
+        // this window's E applied to the later columns of the row
+#pragma unroll 2
+        for (int k = wc + SUB; k < B; ++k) {
+            const float4* u4 = reinterpret_cast<const float4*>(UtS + k * B + wc);
+            float acc = myrow[k];
+#pragma unroll
+            for (int jj = 0; jj < SUB / 4; ++jj) {
+                const float4 u = u4[jj];
+                acc = fmaf(-w[4 * jj + 0], u.x, acc);
+                acc = fmaf(-w[4 * jj + 1], u.y, acc);
+                acc = fmaf(-w[4 * jj + 2], u.z, acc);
+                acc = fmaf(-w[4 * jj + 3], u.w, acc);
+            }
+            myrow[k] = acc;
+        }
+    }
+    if (!finite) record_error(a.st, GPTQ_ERR_NONFINITE, r);
 }
 
 // RTN: one thread per 32 consecutive codes of a row (one packing unit for
@@ -291,7 +294,7 @@ __global__ void transpose_upper_kernel(const float* __restrict__ U, int d, float
 }
 
 template <int BITS>
-int run_sweep(const SweepArgs& a, const float* Ut, cudaStream_t stream) {
+int run_sweep(const SweepArgs& a, cudaStream_t stream) {
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -308,7 +311,7 @@ int run_sweep(const SweepArgs& a, const float* Ut, cudaStream_t stream) {
         if (tail > 0) {
             // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]   (U[i0+k][i0+B+n] = Ut[i0+B+n][i0+k])
             float* c = a.W + i0 + B;
-            const int rc = launch_tgemm(a.d_out, tail, B, -1.0f, a.E, B, Ut + size_t(i0 + B) * a.d_in + i0, a.d_in,
+            const int rc = launch_tgemm(a.d_out, tail, B, -1.0f, a.E, B, a.Ut + size_t(i0 + B) * a.d_in + i0, a.d_in,
                                         true, 1.0f, c, c, a.d_in, false, stream, a.st);
             if (rc) return rc;
         }
@@ -342,20 +345,21 @@ int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int b
     a.Q = Q;
     a.E = static_cast<float*>(ws);
     a.st = st;
+    float* Ut = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                         ((size_t(d_out) * B * sizeof(float) + 255) & ~size_t(255)));
+    a.Ut = Ut;
     if (groupsize < 0) {
         const int warps = a.d_out;
         grid_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(W, a.d_out, a.d_in, a.d_in, 1, a.maxq, scales,
                                                                   zeros, st); count_launch();
     }
-    float* Ut = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                         ((size_t(d_out) * B * sizeof(float) + 255) & ~size_t(255)));
     transpose_upper_kernel<<<dim3(unsigned(d_in / 32), unsigned(d_in / 32)), dim3(32, 8), 0, stream>>>(U, int(d_in), Ut);
     count_launch();
     switch (bits) {
-        case 2: return run_sweep<2>(a, Ut, stream);
-        case 3: return run_sweep<3>(a, Ut, stream);
-        case 4: return run_sweep<4>(a, Ut, stream);
-        case 8: return run_sweep<8>(a, Ut, stream);
+        case 2: return run_sweep<2>(a, stream);
+        case 3: return run_sweep<3>(a, stream);
+        case 4: return run_sweep<4>(a, stream);
+        case 8: return run_sweep<8>(a, stream);
         default: return GPTQ_ERR_UNSUPPORTED;
     }
 }

@@ -11,12 +11,14 @@
 // accurate to about 2^-21 relative (the dropped A_lo B_lo term and the tf32
 // reading of the lo parts), comparable to an fp32 FMA chain of length K.
 //
-// Tile 128 x 128 per CTA, K in chunks of 32 (one 128-byte swizzle row of
-// fp32).  Both operands are K-major: A[m * lda + k] and B(k, n) = Bt[n * ldb + k]
+// Tile 128 x 128 per CTA, K <= 128 in chunks of 32 (one 128-byte swizzle row
+// of fp32), all chunks loaded at once so that the tile's latency is one load,
+// not four.  Both operands are K-major: A[m * lda + k] and B(k, n) = Bt[n * ldb + k]
 // (an MN-major tf32 operand would need a different shared-memory layout, so
-// the callers arrange their data to avoid it).  A chunk travels by TMA (no
-// multicast), eight warps split it into hi / lo in place, one thread issues
-// the MMAs, and four warps drain TMEM into C.  K must be a multiple of 32.
+// the callers arrange their data to avoid it).  Chunks travel by TMA (no
+// multicast), eight warps split each into hi (in place) / lo (two rotating
+// buffers), one thread issues the MMAs, and four warps drain TMEM into C.
+// K must be a multiple of 32 and at most 128.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,15 +26,16 @@ namespace gptq {
 namespace tg {
 
 constexpr int BM = 128, BN = 128, BKC = 32;       // tile, K chunk (fp32 elements)
-constexpr int STAGES = 2;
+constexpr int MAX_CHUNKS = 4;                      // K <= 128: every chunk resident at once
+constexpr int LO_BUFS = 2;                         // lo parts, double-buffered
 constexpr int A_BYTES = BM * BKC * 4;              // 16 KB
 constexpr int B_BYTES = BN * BKC * 4;              // 16 KB
-constexpr int STAGE_BYTES = 2 * (A_BYTES + B_BYTES);   // fp32(->hi) + lo for A and B
+constexpr int CHUNK_BYTES = A_BYTES + B_BYTES;     // fp32 chunk (becomes the hi part in place)
 constexpr int CONV_WARPS = 8;                      // split hi/lo; warp 0 lane 0 issues MMAs; warps 0-3 drain TMEM
 constexpr int PRODUCER_WARP = CONV_WARPS;          // TMA only
 constexpr int THREADS = 32 * (CONV_WARPS + 1);
 constexpr int TMEM_COLS = 128;
-constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + 256;
+constexpr size_t SMEM_BYTES = 1024 + size_t(MAX_CHUNKS + LO_BUFS) * CHUNK_BYTES + 256;
 
 // instruction descriptor: tf32 x tf32 -> f32, A and B K-major, M = BM, N = BN
 __host__ __device__ constexpr uint32_t idesc_tf32() {
@@ -76,10 +79,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     tgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Args g) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(STAGES) * STAGE_BYTES);
-    uint64_t* conv = full + STAGES;    // 8 warp arrivals: stage split into hi / lo
-    uint64_t* empty = conv + STAGES;   // MMA commit: stage free
-    uint64_t* accum = empty + STAGES;
+    uint8_t* lo_base = smem + size_t(MAX_CHUNKS) * CHUNK_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(lo_base + size_t(LO_BUFS) * CHUNK_BYTES);  // [MAX_CHUNKS]
+    uint64_t* conv = full + MAX_CHUNKS;      // [MAX_CHUNKS] 8 warp arrivals: chunk split into hi / lo
+    uint64_t* lo_free = conv + MAX_CHUNKS;   // [LO_BUFS] MMA commit: lo buffer may be reused
+    uint64_t* accum = lo_free + LO_BUFS;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
 
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
@@ -89,11 +93,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&conv[s], CONV_WARPS);
-            mbar_init(&empty[s], 1);
+        for (int c = 0; c < MAX_CHUNKS; ++c) {
+            mbar_init(&full[c], 1);
+            mbar_init(&conv[c], CONV_WARPS);
         }
+        for (int b = 0; b < LO_BUFS; ++b) mbar_init(&lo_free[b], 1);
         mbar_init(accum, 1);
         fence_mbar_init();
     }
@@ -109,22 +113,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == PRODUCER_WARP) {
         if (lane == 0) {
-            int last_round[STAGES] = {-1, -1};
-            bool ok = true;
             for (int c = 0; c < nk; ++c) {
-                const int s = c % STAGES;
-                const uint32_t round = c / STAGES;
-                if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, g.st, 301)) { ok = false; break; }
-                uint8_t* base = smem + size_t(s) * STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
-                tma_load_2d(base, &tmA, c * BKC, m0, &full[s]);              // A:   {32 k, 128 rows}
-                tma_load_2d(base + 2 * A_BYTES, &tmB, c * BKC, n0, &full[s]); // B^T: {32 k, 128 rows}
-                last_round[s] = int(round);
+                uint8_t* base = smem + size_t(c) * CHUNK_BYTES;
+                mbar_arrive_expect_tx(&full[c], CHUNK_BYTES);
+                tma_load_2d(base, &tmA, c * BKC, m0, &full[c]);              // A:   {32 k, 128 rows}
+                tma_load_2d(base + A_BYTES, &tmB, c * BKC, n0, &full[c]);    // B^T: {32 k, 128 rows}
             }
-            if (!ok) {
-                for (int s = 0; s < STAGES; ++s)
-                    if (last_round[s] >= 0) (void)mbar_wait(&full[s], uint32_t(last_round[s]) & 1u, g.st, 302);
-            }
+            // every wait below is bounded; the copies are all waited for by the
+            // converters before the CTA can reach its end
         }
     } else {
         // ---------------- split each chunk into hi / lo; warp 0 lane 0 issues the MMAs
@@ -132,37 +128,30 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int ct = threadIdx.x;   // 0 .. 32*CONV_WARPS-1
         bool ok = true;
         for (int c = 0; c < nk; ++c) {
-            const int s = c % STAGES;
-            const uint32_t round = c / STAGES;
-            uint8_t* base = smem + size_t(s) * STAGE_BYTES;
-            ok = ok && mbar_wait(&full[s], round & 1u, g.st, 303);
+            uint8_t* base = smem + size_t(c) * CHUNK_BYTES;
+            uint8_t* lo = lo_base + size_t(c % LO_BUFS) * CHUNK_BYTES;
+            const bool landed = mbar_wait(&full[c], 0, g.st, 303);
+            ok = ok && landed;
+            if (c >= LO_BUFS) ok = ok && mbar_wait(&lo_free[c % LO_BUFS], uint32_t(c / LO_BUFS - 1) & 1u, g.st, 306);
             if (ok) {
-                float4* xa = reinterpret_cast<float4*>(base);
-                float4* la = reinterpret_cast<float4*>(base + A_BYTES);
-                float4* xb = reinterpret_cast<float4*>(base + 2 * A_BYTES);
-                float4* lb = reinterpret_cast<float4*>(base + 2 * A_BYTES + B_BYTES);
-                for (int i = ct; i < A_BYTES / 16; i += 32 * CONV_WARPS) {
-                    float4 v = xa[i], h, l;
-                    split_tf32(v.x, h.x, l.x); split_tf32(v.y, h.y, l.y);
-                    split_tf32(v.z, h.z, l.z); split_tf32(v.w, h.w, l.w);
-                    xa[i] = h; la[i] = l;
-                }
-                for (int i = ct; i < B_BYTES / 16; i += 32 * CONV_WARPS) {
-                    float4 v = xb[i], h, l;
-                    split_tf32(v.x, h.x, l.x); split_tf32(v.y, h.y, l.y);
-                    split_tf32(v.z, h.z, l.z); split_tf32(v.w, h.w, l.w);
-                    xb[i] = h; lb[i] = l;
+                float4* x = reinterpret_cast<float4*>(base);
+                float4* l = reinterpret_cast<float4*>(lo);
+                for (int i = ct; i < CHUNK_BYTES / 16; i += 32 * CONV_WARPS) {
+                    float4 v = x[i], h, q;
+                    split_tf32(v.x, h.x, q.x); split_tf32(v.y, h.y, q.y);
+                    split_tf32(v.z, h.z, q.z); split_tf32(v.w, h.w, q.w);
+                    x[i] = h; l[i] = q;
                 }
             }
             fence_proxy_async_smem();      // generic-proxy writes -> visible to tcgen05 reads
             __syncwarp();
-            if (lane == 0) mbar_arrive(&conv[s]);
+            if (lane == 0) mbar_arrive(&conv[c]);
             if (warp == 0 && lane == 0) {
-                const bool ready = ok && mbar_wait(&conv[s], round & 1u, g.st, 304);
+                const bool ready = ok && mbar_wait(&conv[c], 0, g.st, 304);
                 if (ready) {
                     tc_fence_after();
-                    const uint32_t a_hi = smem_u32(base), a_lo = a_hi + A_BYTES;
-                    const uint32_t b_hi = a_hi + 2 * A_BYTES, b_lo = b_hi + B_BYTES;
+                    const uint32_t a_hi = smem_u32(base), b_hi = a_hi + A_BYTES;
+                    const uint32_t a_lo = smem_u32(lo), b_lo = a_lo + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BKC / 8; ++kk) {
                         // K-major: 8 k (32 bytes) per MMA inside the 128-byte swizzled
@@ -177,7 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
                 ok = ready;
-                umma_commit(&empty[s]);    // frees the stage once these MMAs are done
+                umma_commit(&lo_free[c % LO_BUFS]);   // this chunk's lo buffer is free once these MMAs finish
             }
             __syncwarp();
         }
@@ -253,7 +242,7 @@ int launch_tgemm(int M, int N, int K, float alpha, const float* A, int lda, cons
                  DevStatus* st) {
     using namespace tg;
     if (M <= 0 || N <= 0) return GPTQ_OK;
-    if (!trans_b || K <= 0 || K % BKC != 0 || g_enc == nullptr) return GPTQ_ERR_UNSUPPORTED;
+    if (!trans_b || K <= 0 || K % BKC != 0 || K > BKC * MAX_CHUNKS || g_enc == nullptr) return GPTQ_ERR_UNSUPPORTED;
     CUtensorMap ta, tb;
     int rc = make_map_2d(&ta, A, uint64_t(K), uint64_t(M), uint64_t(lda), BKC, BM);
     if (rc) return rc;
