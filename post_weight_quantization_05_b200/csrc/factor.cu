@@ -170,11 +170,16 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     __shared__ int failed;
     if (*info != 0) return;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    for (int idx = t; idx < NB * NB; idx += DIAG_THREADS) {
+#pragma unroll 4
+    for (int idx = 4 * t; idx < NB * NB; idx += 4 * DIAG_THREADS) {
         const int r = idx / NB, c = idx % NB;
-        S[r * LD + c] = (c <= r) ? A[size_t(k0 + r) * d + k0 + c] : 0.0f;
-        Y[r * LD + c] = 0.0f;
+        const float4 v = *reinterpret_cast<const float4*>(A + size_t(k0 + r) * d + k0 + c);
+        S[r * LD + c] = (c <= r) ? v.x : 0.0f;
+        S[r * LD + c + 1] = (c + 1 <= r) ? v.y : 0.0f;
+        S[r * LD + c + 2] = (c + 2 <= r) ? v.z : 0.0f;
+        S[r * LD + c + 3] = (c + 3 <= r) ? v.w : 0.0f;
     }
+    for (int idx = t; idx < NB * LD; idx += DIAG_THREADS) Y[idx] = 0.0f;
     if (t == 0) failed = 0;
     __syncthreads();
 
@@ -280,18 +285,37 @@ __global__ void __launch_bounds__(DIAG_THREADS)
         }
     }
 
-    for (int idx = t; idx < NB * NB; idx += DIAG_THREADS) {
+#pragma unroll 4
+    for (int idx = 4 * t; idx < NB * NB; idx += 4 * DIAG_THREADS) {
         const int r = idx / NB, c = idx % NB;
-        if (c <= r) A[size_t(k0 + r) * d + k0 + c] = S[r * LD + c];
-        Dinv[idx] = (c <= r) ? Y[r * LD + c] : 0.0f;
+        float* arow = A + size_t(k0 + r) * d + k0 + c;
+        if (c + 3 <= r) {
+            *reinterpret_cast<float4*>(arow) =
+                make_float4(S[r * LD + c], S[r * LD + c + 1], S[r * LD + c + 2], S[r * LD + c + 3]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (c + q <= r) arow[q] = S[r * LD + c + q];
+        }
+        *reinterpret_cast<float4*>(Dinv + idx) =
+            make_float4((c <= r) ? Y[r * LD + c] : 0.0f, (c + 1 <= r) ? Y[r * LD + c + 1] : 0.0f,
+                        (c + 2 <= r) ? Y[r * LD + c + 2] : 0.0f, (c + 3 <= r) ? Y[r * LD + c + 3] : 0.0f);
     }
 }
 
-// Z[k*NB + c][k*NB + r] = Dinv_k[r][c]: diagonal block k of Z = L^-T.
+// Z[k*NB + c][k*NB + r] = Dinv_k[r][c]: diagonal block k of Z = L^-T,
+// transposed through shared memory (coalesced on both sides).
 __global__ void place_diag_inverse_t_kernel(const float* __restrict__ Dinv_k, int d, int k, float* __restrict__ Z) {
-    for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
+    extern __shared__ float tile[];   // [NB][LD]
+    for (int idx = 4 * threadIdx.x; idx < NB * NB; idx += 4 * blockDim.x) {
         const int r = idx / NB, c = idx % NB;
-        Z[size_t(k * NB + c) * d + k * NB + r] = Dinv_k[idx];
+        const float4 v = *reinterpret_cast<const float4*>(Dinv_k + idx);
+        tile[r * LD + c] = v.x; tile[r * LD + c + 1] = v.y; tile[r * LD + c + 2] = v.z; tile[r * LD + c + 3] = v.w;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
+        const int c = idx / NB, r = idx % NB;
+        Z[size_t(k * NB + c) * d + k * NB + r] = tile[r * LD + c];
     }
 }
 
@@ -366,7 +390,9 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
         if (cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(DIAG_SMEM)) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(place_diag_inverse_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(NB * LD * sizeof(float))) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         attr_set[dev] = true;
     }
@@ -418,7 +444,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
             if (rc) return rc;
         }
         // inverse block step k on the auxiliary stream
-        place_diag_inverse_t_kernel<<<1, 256, 0, as>>>(dk, d, k, Z); count_launch();
+        place_diag_inverse_t_kernel<<<1, 512, NB * LD * sizeof(float), as>>>(dk, d, k, Z); count_launch();
         if (k > 0) {
             float* zi = Z + k0;   // in place is safe for the same reason as the panel
             rc = launch_tgemm(k0, NB, NB, 1.0f, zi, d, dk, NB, true, 0.0f, zi, zi, d, false, as, st);

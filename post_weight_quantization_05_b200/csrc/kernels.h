@@ -29,6 +29,9 @@ int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, voi
 // rules.  lower_only skips 128 x 128 output tiles entirely above the
 // diagonal.  C_out may alias C_in.
 void set_tensor_map_encoder(PFN_encodeTiled f);
+// 2-D fp32 tensor map (row stride ld_elems), 128-byte swizzle or none.
+int make_map_2d_f32(CUtensorMap* tm, const float* base, uint64_t inner, uint64_t outer, uint64_t ld_elems,
+                    uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 int launch_tgemm(int M, int N, int K, float alpha, const float* A, int lda, const float* B, int ldb, bool trans_b,
                  float beta, const float* C_in, float* C_out, int ldc, bool lower_only, cudaStream_t stream,
                  DevStatus* st);

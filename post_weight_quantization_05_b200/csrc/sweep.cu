@@ -135,12 +135,15 @@ struct SweepArgs {
 };
 
 // shared memory: U block (row-major), U block transposed, 1/U_jj, rows, mbarrier
-constexpr size_t SMEM = (size_t(2) * B * B + B + size_t(ROWS) * RLD) * sizeof(float) + 16;
+constexpr size_t SMEM = 1024 /*align slack*/ + (size_t(2) * B * B + B + size_t(ROWS) * RLD) * sizeof(float) + 16;
 
 template <int BITS>
-__global__ void __launch_bounds__(ROWS) sweep_block_kernel(const SweepArgs a, int i0) {
-    extern __shared__ float sm[];
-    float* Us = sm;                          // Us[j][k]  = U[i0+j][i0+k]
+__global__ void __launch_bounds__(ROWS) sweep_block_kernel(const __grid_constant__ CUtensorMap tmU,
+                                                           const __grid_constant__ CUtensorMap tmUt, const SweepArgs a,
+                                                           int i0) {
+    extern __shared__ uint8_t smem_raw[];
+    float* sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* Us = sm;                          // Us[j][k]  = U[i0+j][i0+k]  (TMA destination: 1024-aligned)
     float* UtS = sm + B * B;                 // UtS[k][j] = U[i0+j][i0+k]
     float* invd = UtS + B * B;               // 1 / U[i0+j][i0+j]
     float* rows = invd + B;                  // per-thread row, stride RLD
@@ -151,13 +154,10 @@ __global__ void __launch_bounds__(ROWS) sweep_block_kernel(const SweepArgs a, in
     }
     __syncthreads();
     if (threadIdx.x == 0) {
+        // two 128 x 128 fp32 boxes (no swizzle: dense row-major in shared memory)
         mbar_arrive_expect_tx(bar, 2 * B * B * sizeof(float));
-        const float* ub = a.U + size_t(i0) * a.d_in + i0;
-        const float* utb = a.Ut + size_t(i0) * a.d_in + i0;
-        for (int j = 0; j < B; ++j) {
-            bulk_load(Us + j * B, ub + size_t(j) * a.d_in, B * sizeof(float), bar);
-            bulk_load(UtS + j * B, utb + size_t(j) * a.d_in, B * sizeof(float), bar);
-        }
+        tma_load_2d(Us, &tmU, i0, i0, bar);
+        tma_load_2d(UtS, &tmUt, i0, i0, bar);
     }
     const int r = blockIdx.x * ROWS + threadIdx.x;
     const bool active = r < a.d_out;
@@ -304,9 +304,13 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
             return GPTQ_ERR_CUDA;
         attr_set[dev] = true;
     }
+    CUtensorMap tmU, tmUt;
+    if (make_map_2d_f32(&tmU, a.U, uint64_t(a.d_in), uint64_t(a.d_in), uint64_t(a.d_in), B, B, false) ||
+        make_map_2d_f32(&tmUt, a.Ut, uint64_t(a.d_in), uint64_t(a.d_in), uint64_t(a.d_in), B, B, false))
+        return GPTQ_ERR_CUDA;
     const int blocks = (a.d_out + ROWS - 1) / ROWS;
     for (int i0 = 0; i0 < a.d_in; i0 += B) {
-        sweep_block_kernel<BITS><<<blocks, ROWS, SMEM, stream>>>(a, i0); count_launch();
+        sweep_block_kernel<BITS><<<blocks, ROWS, SMEM, stream>>>(tmU, tmUt, a, i0); count_launch();
         const int tail = a.d_in - i0 - B;
         if (tail > 0) {
             // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]   (U[i0+k][i0+B+n] = Ut[i0+B+n][i0+k])

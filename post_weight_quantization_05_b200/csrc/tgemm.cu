@@ -123,6 +123,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             // converters before the CTA can reach its end
         }
     } else {
+        // epilogue warps: fetch this thread's row of C_in now, so that its
+        // latency overlaps the loads, the split and the MMAs
+        const int m = m0 + (warp & 3) * 32 + lane;
+        const bool pre = warp < 4 && g.beta != 0.0f && m < g.M && n0 + BN <= g.N;
+        float4 cpre[BN / 4];
+        if (pre) {
+            const float4* src = reinterpret_cast<const float4*>(g.C_in + size_t(m) * g.ldc + n0);
+#pragma unroll
+            for (int q = 0; q < BN / 4; ++q) cpre[q] = src[q];
+        }
         // ---------------- split each chunk into hi / lo; warp 0 lane 0 issues the MMAs
         constexpr uint32_t idesc = idesc_tf32();
         const int ct = threadIdx.x;   // 0 .. 32*CONV_WARPS-1
@@ -178,16 +188,23 @@ __global__ void __launch_bounds__(THREADS, 1)
             const bool ready = mbar_wait(accum, 0, g.st, 305);
             tc_fence_after();
             if (ready && nk > 0) {
-                const int m = m0 + warp * 32 + lane;
-#pragma unroll 1
+#pragma unroll
                 for (int cc = 0; cc < BN / 32; ++cc) {
                     float v[32];
                     tmem_ld_32x32b_x32(tmem_base + (uint32_t(warp * 32) << 16) + uint32_t(cc * 32), v);
                     const int n = n0 + cc * 32;
                     if (m >= g.M) continue;
-                    const float* cin = g.C_in + size_t(m) * g.ldc + n;
                     float* cout = g.C_out + size_t(m) * g.ldc + n;
-                    if (n + 32 <= g.N) {
+                    if (pre) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 ci = cpre[cc * 8 + q];
+                            *reinterpret_cast<float4*>(cout + 4 * q) =
+                                make_float4(fmaf(g.alpha, v[4 * q], g.beta * ci.x), fmaf(g.alpha, v[4 * q + 1], g.beta * ci.y),
+                                            fmaf(g.alpha, v[4 * q + 2], g.beta * ci.z), fmaf(g.alpha, v[4 * q + 3], g.beta * ci.w));
+                        }
+                    } else if (n + 32 <= g.N) {
+                        const float* cin = g.C_in + size_t(m) * g.ldc + n;
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             float4 r;
@@ -204,6 +221,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                             *reinterpret_cast<float4*>(cout + 4 * q) = r;
                         }
                     } else {
+                        const float* cin = g.C_in + size_t(m) * g.ldc + n;
 #pragma unroll
                         for (int q = 0; q < 32; ++q)
                             if (n + q < g.N) cout[q] = fmaf(g.alpha, v[q], g.beta != 0.0f ? g.beta * cin[q] : 0.0f);
@@ -225,14 +243,16 @@ PFN_encodeTiled g_enc = nullptr;
 
 void set_tensor_map_encoder(PFN_encodeTiled f) { g_enc = f; }
 
-static int make_map_2d(CUtensorMap* tm, const float* base, uint64_t inner, uint64_t outer, uint64_t ld_elems,
-                       uint32_t box_inner, uint32_t box_outer) {
+int make_map_2d_f32(CUtensorMap* tm, const float* base, uint64_t inner, uint64_t outer, uint64_t ld_elems,
+                    uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+    if (g_enc == nullptr) return GPTQ_ERR_CUDA;
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {ld_elems * 4};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = g_enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box,
-                             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
@@ -244,9 +264,9 @@ int launch_tgemm(int M, int N, int K, float alpha, const float* A, int lda, cons
     if (M <= 0 || N <= 0) return GPTQ_OK;
     if (!trans_b || K <= 0 || K % BKC != 0 || K > BKC * MAX_CHUNKS || g_enc == nullptr) return GPTQ_ERR_UNSUPPORTED;
     CUtensorMap ta, tb;
-    int rc = make_map_2d(&ta, A, uint64_t(K), uint64_t(M), uint64_t(lda), BKC, BM);
+    int rc = make_map_2d_f32(&ta, A, uint64_t(K), uint64_t(M), uint64_t(lda), BKC, BM, true);
     if (rc) return rc;
-    rc = make_map_2d(&tb, B, uint64_t(K), uint64_t(N), uint64_t(ldb), BKC, BN);
+    rc = make_map_2d_f32(&tb, B, uint64_t(K), uint64_t(N), uint64_t(ldb), BKC, BN, true);
     if (rc) return rc;
     Args g{M, N, K, alpha, beta, C_in, C_out, ldc, lower_only ? 1 : 0, st};
     static bool attr_set[64] = {};
