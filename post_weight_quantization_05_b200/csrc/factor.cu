@@ -27,9 +27,10 @@ namespace gptq {
 namespace factor {
 
 constexpr int NB = 128;
-constexpr int LD = NB + 1;  // padded shared-memory row
+constexpr int LD = NB + 1;   // padded shared-memory row (column accesses conflict-free)
+constexpr int LDY = NB + 4;  // inverse rows: 16-byte aligned for vector access
 constexpr int DIAG_THREADS = 256;
-constexpr size_t DIAG_SMEM = size_t(2) * NB * LD * sizeof(float);
+constexpr size_t DIAG_SMEM = size_t(NB) * (LD + LDY) * sizeof(float);
 
 struct Layout {
     size_t a_off, y_off, dinv_off, scal_off, total;
@@ -121,21 +122,25 @@ struct ColChol32 {
         if (lane == C) {
             const float piv = col[C];
             if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) bad = C;
-            const float lcc = sqrtf(piv);
-            const float inv = 1.0f / lcc;
-            col[C] = lcc;
-            buf[C] = lcc;
+            const float inv = rsqrtf(piv);
+            col[C] = piv * inv;
 #pragma unroll
-            for (int r = C + 1; r < SB; ++r) {
-                col[r] *= inv;
-                buf[r] = col[r];
-            }
+            for (int r = C + 1; r < SB; ++r) col[r] *= inv;
+#pragma unroll
+            for (int r = (C / 4) * 4; r < SB; r += 4)      // whole 16-byte groups; entries < C unused
+                *reinterpret_cast<float4*>(buf + r) = make_float4(col[r], col[r + 1], col[r + 2], col[r + 3]);
         }
         __syncwarp();
         if (lane > C) {
             const float ljc = buf[lane];                  // L[lane][C]
 #pragma unroll
-            for (int r = C + 1; r < SB; ++r) col[r] = fmaf(-buf[r], ljc, col[r]);
+            for (int r4 = ((C + 1) / 4) * 4; r4 < SB; r4 += 4) {
+                const float4 b = *reinterpret_cast<const float4*>(buf + r4);
+                if (r4 + 0 > C) col[r4 + 0] = fmaf(-b.x, ljc, col[r4 + 0]);
+                if (r4 + 1 > C) col[r4 + 1] = fmaf(-b.y, ljc, col[r4 + 1]);
+                if (r4 + 2 > C) col[r4 + 2] = fmaf(-b.z, ljc, col[r4 + 2]);
+                if (r4 + 3 > C) col[r4 + 3] = fmaf(-b.w, ljc, col[r4 + 3]);
+            }
         }
         __syncwarp();
         if constexpr (C + 1 < SB) ColChol32<C + 1>::run(col, lane, buf, bad);
@@ -164,9 +169,9 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     potrf_diag_kernel(float* __restrict__ A, int d, int k0, float* __restrict__ Dinv, int* info, DevStatus* st) {
     extern __shared__ float sm[];
     float* S = sm;             // [NB][LD] factor (upper part used as scratch)
-    float* Y = sm + NB * LD;   // [NB][LD] inverse
+    float* Y = sm + NB * LD;   // [NB][LDY] inverse (NB * LD is a multiple of 4: 16-byte aligned)
     __shared__ float invd[NB];
-    __shared__ float colbuf[SB];
+    __shared__ __align__(16) float colbuf[SB];
     __shared__ int failed;
     if (*info != 0) return;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -179,7 +184,7 @@ __global__ void __launch_bounds__(DIAG_THREADS)
         S[r * LD + c + 2] = (c + 2 <= r) ? v.z : 0.0f;
         S[r * LD + c + 3] = (c + 3 <= r) ? v.w : 0.0f;
     }
-    for (int idx = t; idx < NB * LD; idx += DIAG_THREADS) Y[idx] = 0.0f;
+    for (int idx = t; idx < NB * LDY; idx += DIAG_THREADS) Y[idx] = 0.0f;
     if (t == 0) failed = 0;
     __syncthreads();
 
@@ -251,7 +256,7 @@ __global__ void __launch_bounds__(DIAG_THREADS)
         for (int r = 0; r < SB; ++r) y[r] = (r == lane) ? 1.0f : 0.0f;
         ColInv32<0>::run(y, S + o * LD + o, invd + o, lane);
 #pragma unroll
-        for (int r = 0; r < SB; ++r) Y[(o + r) * LD + o + lane] = (r >= lane) ? y[r] : 0.0f;
+        for (int r = 0; r < SB; ++r) Y[(o + r) * LDY + o + lane] = (r >= lane) ? y[r] : 0.0f;
     }
     __syncthreads();
 
@@ -260,26 +265,42 @@ __global__ void __launch_bounds__(DIAG_THREADS)
     {
         const int i = t >> 3, j4 = (t & 7) * 4;
         for (int bi = 1; bi < NB / SB; ++bi) {
-            for (int bj = 0; bj < bi; ++bj) {
-                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                for (int k = bj * SB; k < bi * SB; ++k) {
-                    const float l = S[(bi * SB + i) * LD + k];
+            // one pass over k serves every bj (independent accumulators)
+            float4 acc[NB / SB - 1];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[q] = fmaf(l, Y[k * LD + bj * SB + j4 + q], acc[q]);
+            for (int bj = 0; bj < NB / SB - 1; ++bj) acc[bj] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            const float* lrow = S + (bi * SB + i) * LD;
+#pragma unroll 4
+            for (int k = 0; k < bi * SB; ++k) {
+                const float l = lrow[k];
+#pragma unroll
+                for (int bj = 0; bj < NB / SB - 1; ++bj) {
+                    if (bj < bi && k >= bj * SB) {
+                        const float4 y = *reinterpret_cast<const float4*>(Y + k * LDY + bj * SB + j4);
+                        acc[bj].x = fmaf(l, y.x, acc[bj].x); acc[bj].y = fmaf(l, y.y, acc[bj].y);
+                        acc[bj].z = fmaf(l, y.z, acc[bj].z); acc[bj].w = fmaf(l, y.w, acc[bj].w);
+                    }
                 }
+            }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) S[i * LD + (1 + bj) * SB + j4 + q] = acc[q];
+            for (int bj = 0; bj < NB / SB - 1; ++bj) {
+                if (bj < bi) {
+                    float* trow = S + i * LD + (1 + bj) * SB + j4;
+                    trow[0] = acc[bj].x; trow[1] = acc[bj].y; trow[2] = acc[bj].z; trow[3] = acc[bj].w;
+                }
             }
             __syncthreads();
             for (int bj = 0; bj < bi; ++bj) {
-                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                const float* yrow = Y + (bi * SB + i) * LDY + bi * SB;
                 for (int k = 0; k <= i; ++k) {
-                    const float y = Y[(bi * SB + i) * LD + bi * SB + k];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[q] = fmaf(y, S[k * LD + (1 + bj) * SB + j4 + q], acc[q]);
+                    const float y = yrow[k];
+                    const float* trow = S + k * LD + (1 + bj) * SB + j4;
+                    acc.x = fmaf(y, trow[0], acc.x); acc.y = fmaf(y, trow[1], acc.y);
+                    acc.z = fmaf(y, trow[2], acc.z); acc.w = fmaf(y, trow[3], acc.w);
                 }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) Y[(bi * SB + i) * LD + bj * SB + j4 + q] = -acc[q];
+                *reinterpret_cast<float4*>(Y + (bi * SB + i) * LDY + bj * SB + j4) =
+                    make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
             __syncthreads();
         }
@@ -297,9 +318,10 @@ __global__ void __launch_bounds__(DIAG_THREADS)
             for (int q = 0; q < 4; ++q)
                 if (c + q <= r) arow[q] = S[r * LD + c + q];
         }
+        const float4 yv = *reinterpret_cast<const float4*>(Y + r * LDY + c);
         *reinterpret_cast<float4*>(Dinv + idx) =
-            make_float4((c <= r) ? Y[r * LD + c] : 0.0f, (c + 1 <= r) ? Y[r * LD + c + 1] : 0.0f,
-                        (c + 2 <= r) ? Y[r * LD + c + 2] : 0.0f, (c + 3 <= r) ? Y[r * LD + c + 3] : 0.0f);
+            make_float4((c <= r) ? yv.x : 0.0f, (c + 1 <= r) ? yv.y : 0.0f, (c + 2 <= r) ? yv.z : 0.0f,
+                        (c + 3 <= r) ? yv.w : 0.0f);
     }
 }
 
@@ -319,12 +341,15 @@ __global__ void place_diag_inverse_t_kernel(const float* __restrict__ Dinv_k, in
     }
 }
 
-// One auxiliary stream and two events per device (created on first use):
-// the inverse's block steps run there, each as soon as the factorization has
-// finished the block column it needs, overlapping the rest of the Cholesky.
+// Two auxiliary streams and a few events per device (created on first use):
+// the inverse's block steps run on one, each as soon as the factorization has
+// finished the block column it needs; the trailing update beyond the next
+// block column runs on the other, so that the next diagonal block can be
+// factored while it proceeds (look-ahead).
 struct AuxStream {
-    cudaStream_t s = nullptr;
-    cudaEvent_t fork = nullptr, step = nullptr, join = nullptr;
+    cudaStream_t s = nullptr;       // inverse steps
+    cudaStream_t side = nullptr;    // trailing updates beyond the next block column
+    cudaEvent_t fork = nullptr, step = nullptr, rest = nullptr, join = nullptr, join_side = nullptr;
 };
 
 static int aux_stream(AuxStream** out) {
@@ -336,9 +361,12 @@ static int aux_stream(AuxStream** out) {
     AuxStream& a = per_dev[dev];
     if (!a.s) {
         if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&a.side, cudaStreamNonBlocking) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.step, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess)
+            cudaEventCreateWithFlags(&a.rest, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.join_side, cudaEventDisableTiming) != cudaSuccess)
             return GPTQ_ERR_CUDA;
     }
     *out = &a;
@@ -407,17 +435,23 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
 
     damp_lambda_kernel<<<1, 1024, 0, stream>>>(H, d, percdamp, lam, info, st); count_launch();
     reverse_damp_kernel<<<ew_blocks, 256, 0, stream>>>(H, d, lam, A); count_launch();
-    // fork: the inverse (stream `as`) starts from a zeroed Z
-    if (cudaEventRecord(aux->fork, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->fork, 0) != cudaSuccess)
+    // fork: the inverse (stream `as`) starts from a zeroed Z; `ss` takes the
+    // trailing updates beyond the next block column
+    const cudaStream_t ss = aux->side;
+    if (cudaEventRecord(aux->fork, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->fork, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(ss, aux->fork, 0) != cudaSuccess || cudaEventRecord(aux->rest, ss) != cudaSuccess)
         return GPTQ_ERR_CUDA;
     {
         const int rc = launch_fill(Z, int64_t(d) * d, 0.0f, as);
         if (rc) return rc;
     }
 
-    // Cholesky of A (lower), blocked right-looking, on `stream`; products on the
-    // tensor cores.  Z = L^-T (upper) on `as`: block step i needs only L's block
-    // column i and Dinv_i, so it runs as soon as the factorization has them:
+    // Cholesky of A (lower), blocked right-looking, products on the tensor
+    // cores.  Step k on `stream`: factor the diagonal block, solve the panel,
+    // update the next block column (after the previous step's far update on
+    // `ss` is done); the rest of the trailing update goes to `ss`.
+    // Z = L^-T (upper) on `as`: block step i needs only L's block column i and
+    // Dinv_i, so it runs as soon as the factorization has them:
     //   Z[i][i] = Dinv_i^T;  Z[0:i0, i] <- Z[0:i0, i] Dinv_i^T;
     //   Z[0:i0+NB, i0+NB:] -= Z[0:i0+NB, i] L[i0+NB:, i]^T
     // (the transpose of the block forward substitution Y = L^-1; working on Z
@@ -439,9 +473,21 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->step, 0) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         if (rest > 0) {
-            float* trail = A + size_t(k0 + NB) * d + k0 + NB;
-            rc = launch_tgemm(rest, rest, NB, -1.0f, panel, d, panel, d, true, 1.0f, trail, trail, d, true, stream, st);
+            // next block column (it holds the next diagonal block) on `stream` ...
+            if (cudaStreamWaitEvent(stream, aux->rest, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
+            float* next = A + size_t(k0 + NB) * d + k0 + NB;
+            rc = launch_tgemm(rest, NB, NB, -1.0f, panel, d, panel, d, true, 1.0f, next, next, d, true, stream, st);
             if (rc) return rc;
+            // ... the columns after it on `ss`
+            if (rest > NB) {
+                if (cudaStreamWaitEvent(ss, aux->step, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
+                float* far = A + size_t(k0 + 2 * NB) * d + k0 + 2 * NB;
+                const float* prow = panel + size_t(NB) * d;
+                rc = launch_tgemm(rest - NB, rest - NB, NB, -1.0f, prow, d, prow, d, true, 1.0f, far, far, d, true,
+                                  ss, st);
+                if (rc) return rc;
+                if (cudaEventRecord(aux->rest, ss) != cudaSuccess) return GPTQ_ERR_CUDA;
+            }
         }
         // inverse block step k on the auxiliary stream
         place_diag_inverse_t_kernel<<<1, 512, NB * LD * sizeof(float), as>>>(dk, d, k, Z); count_launch();
@@ -456,8 +502,10 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
             if (rc) return rc;
         }
     }
-    // join
-    if (cudaEventRecord(aux->join, as) != cudaSuccess || cudaStreamWaitEvent(stream, aux->join, 0) != cudaSuccess)
+    // join both auxiliary streams
+    if (cudaEventRecord(aux->join, as) != cudaSuccess || cudaStreamWaitEvent(stream, aux->join, 0) != cudaSuccess ||
+        cudaEventRecord(aux->join_side, ss) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, aux->join_side, 0) != cudaSuccess)
         return GPTQ_ERR_CUDA;
     write_u_kernel<<<dim3(d / 32, d / 32), dim3(32, 8), 0, stream>>>(Z, d, info, U); count_launch();
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
