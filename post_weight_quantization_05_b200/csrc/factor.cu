@@ -118,10 +118,11 @@ struct Trsm32 {
 // read per row -- no shuffles, one short dependency chain per column.
 template <int C>
 struct ColChol32 {
-    __device__ __forceinline__ static void run(float (&col)[SB], int lane, float* __restrict__ buf, int& bad) {
+    __device__ __forceinline__ static void run(float (&col)[SB], int lane, float* __restrict__ buf, int& bad,
+                                               float& badpiv) {
         if (lane == C) {
             const float piv = col[C];
-            if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) bad = C;
+            if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) { bad = C; badpiv = piv; }
             const float inv = rsqrtf(piv);
             col[C] = piv * inv;
 #pragma unroll
@@ -143,7 +144,7 @@ struct ColChol32 {
             }
         }
         __syncwarp();
-        if constexpr (C + 1 < SB) ColChol32<C + 1>::run(col, lane, buf, bad);
+        if constexpr (C + 1 < SB) ColChol32<C + 1>::run(col, lane, buf, bad, badpiv);
     }
 };
 
@@ -195,16 +196,17 @@ __global__ void __launch_bounds__(DIAG_THREADS)
 #pragma unroll
             for (int r = 0; r < SB; ++r) col[r] = (r >= lane) ? S[(o + r) * LD + o + lane] : 0.0f;
             int bad = -1;
-            ColChol32<0>::run(col, lane, colbuf, bad);
+            float badpiv = 0.0f;
+            ColChol32<0>::run(col, lane, colbuf, bad, badpiv);
 #pragma unroll
             for (int r = 0; r < SB; ++r)
                 if (r >= lane) S[(o + r) * LD + o + lane] = col[r];
             __syncwarp();
             invd[o + lane] = 1.0f / S[(o + lane) * LD + o + lane];
             bad = __reduce_min_sync(FULL, bad < 0 ? SB : bad);
+            const float p = __shfl_sync(FULL, badpiv, bad < SB ? bad : 0);   // the failing pivot's value
             if (bad < SB && lane == 0) {
                 failed = 1;
-                const float p = S[(o + bad) * LD + o + bad];
                 if (atomicCAS(info, 0, k0 + o + bad + 1) == 0)
                     record_error(st, isfinite(p) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, k0 + o + bad + 1);
             }
@@ -341,12 +343,14 @@ __global__ void place_diag_inverse_t_kernel(const float* __restrict__ Dinv_k, in
     }
 }
 
-// Two auxiliary streams and a few events per device (created on first use):
-// the inverse's block steps run on one, each as soon as the factorization has
+// Three internal streams and a few events per device (created on first use).
+// The factorization's critical chain runs on a high-priority stream; the
+// inverse's block steps run on another, each as soon as the factorization has
 // finished the block column it needs; the trailing update beyond the next
-// block column runs on the other, so that the next diagonal block can be
-// factored while it proceeds (look-ahead).
+// block column runs on a low-priority stream, so that the next diagonal block
+// is factored while it proceeds (look-ahead) and gets the SMs first.
 struct AuxStream {
+    cudaStream_t main = nullptr;    // the factorization's critical chain (highest priority)
     cudaStream_t s = nullptr;       // inverse steps
     cudaStream_t side = nullptr;    // trailing updates beyond the next block column
     cudaEvent_t fork = nullptr, step = nullptr, rest = nullptr, join = nullptr, join_side = nullptr;
@@ -360,8 +364,11 @@ static int aux_stream(AuxStream** out) {
     std::lock_guard<std::mutex> lock(mu);
     AuxStream& a = per_dev[dev];
     if (!a.s) {
-        if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaStreamCreateWithFlags(&a.side, cudaStreamNonBlocking) != cudaSuccess ||
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&a.main, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&a.s, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&a.side, cudaStreamNonBlocking, least) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.step, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.rest, cudaEventDisableTiming) != cudaSuccess ||
@@ -432,6 +439,10 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     AuxStream* aux = nullptr;
     if (aux_stream(&aux)) return GPTQ_ERR_CUDA;
     const cudaStream_t as = aux->s;
+    const cudaStream_t caller = stream;
+    stream = aux->main;
+    if (cudaEventRecord(aux->fork, caller) != cudaSuccess || cudaStreamWaitEvent(stream, aux->fork, 0) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
 
     damp_lambda_kernel<<<1, 1024, 0, stream>>>(H, d, percdamp, lam, info, st); count_launch();
     reverse_damp_kernel<<<ew_blocks, 256, 0, stream>>>(H, d, lam, A); count_launch();
@@ -508,6 +519,9 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         cudaStreamWaitEvent(stream, aux->join_side, 0) != cudaSuccess)
         return GPTQ_ERR_CUDA;
     write_u_kernel<<<dim3(d / 32, d / 32), dim3(32, 8), 0, stream>>>(Z, d, info, U); count_launch();
+    // back to the caller's stream
+    if (cudaEventRecord(aux->join, stream) != cudaSuccess || cudaStreamWaitEvent(caller, aux->join, 0) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 

@@ -8,12 +8,15 @@
 // (groups share a grid set from the latest updated weights); "문제 설정" (RTN).
 //
 // Sweep kernel design: rows are independent given U (the same U serves every
-// row), so one thread owns one row of the 128-column block, 32 rows per CTA.
-// The 128 x 128 diagonal block of U (and its transpose) is brought into
-// shared memory by bulk copies; every thread of a warp reads the same U
-// element at the same time (broadcast).  The block's E is written for the
-// lazy trailing product on the tensor cores.  The codes are packed in
-// registers (compile-time bit positions) and stored as vectors.
+// row).  A CTA takes 32 rows (lane = row) and four warps, one per 32-column
+// window of the 128-column block.  Warp q holds its window of every row in
+// registers; it first applies the E of windows p < q (handed over through
+// shared memory, signalled by an mbarrier per window) to its columns, then
+// quantizes its window column by column.  The 128 x 128 diagonal block of U
+// arrives by one TMA copy; every lane of a warp reads the same U element at
+// the same time (broadcast).  The block's E is written for the lazy trailing
+// product on the tensor cores.  The codes are packed in registers
+// (compile-time bit positions) and stored as vectors.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -23,7 +26,6 @@ namespace gptq {
 namespace sweep {
 
 constexpr int B = 128;
-constexpr int ROWS = 32;  // rows (threads) per CTA
 
 // Per-row grid over columns [c0, c0 + len) of the ORIGINAL W: one warp per
 // (row, group).  Writes fp16 scale/zero bit patterns.
@@ -53,16 +55,9 @@ __global__ void grid_kernel(const float* __restrict__ W, int d_out, int d_in, in
     }
 }
 
-// The 128-column block is walked as four 32-column windows.  A thread's row
-// lives in shared memory; the current window is copied into 32 registers and
-// processed by one fully unrolled body (static register indices), which is
-// the same code for all four windows -- the kernel's hot code stays small
-// enough for the instruction cache.  After a window its E values (still in
-// the registers) update the later columns of the row in shared memory, in
-// column order j = 0..31 per element, i.e. the same additions in the same
-// order as the plain rank-1 sweep.
-constexpr int SUB = 32;
-constexpr int RLD = B + 1;   // per-thread row stride in shared memory (conflict-free columns)
+constexpr int SUB = 32;          // window width = rows per CTA
+constexpr int NWIN = B / SUB;    // windows per block = warps per CTA
+constexpr int ELD = SUB + 1;     // E hand-over rows (conflict-free)
 
 // Packer for one window: code j of the window goes to stream bits
 // [j*BITS, (j+1)*BITS) of the window's BITS words.
@@ -98,8 +93,7 @@ struct Grid {
 };
 
 // Column J of the window: quantize, pack, E = (w - q) / U_jj, and the rank-1
-// correction of the window's later columns.  `urow` = U row of this column,
-// offset to the window's first column.
+// correction of the window's later columns (U row from shared memory).
 template <int BITS, int J>
 struct WindowCol {
     __device__ __forceinline__ static void run(float (&w)[SUB], const float* __restrict__ Us, int wc,
@@ -108,7 +102,7 @@ struct WindowCol {
         const float wj = w[J];
         const float c = quant_code(wj, gr.s, gr.z, gr.maxq);
         const float q = gr.s * (c - gr.z);
-        const float e = (wj - q) * invd[wc + J];
+        const float e = (wj - q) * invd[J];
         finite &= isfinite(e);
         if (Qw) Qw[J] = q;
         pk.template put<J>(static_cast<uint32_t>(c));
@@ -134,106 +128,134 @@ struct SweepArgs {
     DevStatus* st;
 };
 
-// shared memory: U block (row-major), U block transposed, 1/U_jj, rows, mbarrier
-constexpr size_t SMEM = 1024 /*align slack*/ + (size_t(2) * B * B + B + size_t(ROWS) * RLD) * sizeof(float) + 16;
+// shared memory: U block, E hand-over (one [32][ELD] per window), 1/U_jj per
+// window, reduction and grid scratch, mbarriers
+constexpr size_t SMEM = 1024 /*align slack*/ +
+                        (size_t(B) * B + size_t(NWIN) * SUB * ELD + B + 4 * NWIN * SUB) * sizeof(float) + 64;
 
 template <int BITS>
-__global__ void __launch_bounds__(ROWS) sweep_block_kernel(const __grid_constant__ CUtensorMap tmU,
-                                                           const __grid_constant__ CUtensorMap tmUt, const SweepArgs a,
-                                                           int i0) {
+__global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_constant__ CUtensorMap tmU,
+                                                                 const SweepArgs a, int i0) {
     extern __shared__ uint8_t smem_raw[];
     float* sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* Us = sm;                          // Us[j][k]  = U[i0+j][i0+k]  (TMA destination: 1024-aligned)
-    float* UtS = sm + B * B;                 // UtS[k][j] = U[i0+j][i0+k]
-    float* invd = UtS + B * B;               // 1 / U[i0+j][i0+j]
-    float* rows = invd + B;                  // per-thread row, stride RLD
-    uint64_t* bar = reinterpret_cast<uint64_t*>(rows + ROWS * RLD);   // even float offset: 8-byte aligned
+    float* Us = sm;                            // Us[j][k] = U[i0+j][i0+k]  (TMA destination: 1024-aligned)
+    float* Eh = Us + B * B;                    // Eh[p][row][j]: E of window p
+    float* invd = Eh + NWIN * SUB * ELD;       // 1 / U[i0+j][i0+j]
+    float* red = invd + B;                     // [2][NWIN][SUB] min / max, then [2][SUB] grid
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + 4 * NWIN * SUB);   // [0] U landed, [1+p] window p's E
+    const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wc = q * SUB;
+    const int r = blockIdx.x * SUB + lane;
+    const bool active = r < a.d_out;
+
     if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
+        mbar_init(&bars[0], 1);
+        for (int p = 0; p < NWIN; ++p) mbar_init(&bars[1 + p], SUB);
         fence_mbar_init();
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        // two 128 x 128 fp32 boxes (no swizzle: dense row-major in shared memory)
-        mbar_arrive_expect_tx(bar, 2 * B * B * sizeof(float));
-        tma_load_2d(Us, &tmU, i0, i0, bar);
-        tma_load_2d(UtS, &tmUt, i0, i0, bar);
+        mbar_arrive_expect_tx(&bars[0], B * B * sizeof(float));
+        tma_load_2d(Us, &tmU, i0, i0, &bars[0]);   // one 128 x 128 fp32 box, no swizzle
     }
-    const int r = blockIdx.x * ROWS + threadIdx.x;
-    const bool active = r < a.d_out;
-    float* myrow = rows + threadIdx.x * RLD;
-    const float* wsrc = a.W + size_t(active ? r : 0) * a.d_in + i0;
+
+    // this warp's window of this lane's row, and its min / max
+    float w[SUB];
+    const float* wsrc = a.W + size_t(active ? r : 0) * a.d_in + i0 + wc;
     float mn = INFINITY, mx = -INFINITY;
-#pragma unroll 4
-    for (int k = 0; k < B; k += 4) {
+#pragma unroll
+    for (int k = 0; k < SUB; k += 4) {
         const float4 v = active ? *reinterpret_cast<const float4*>(wsrc + k) : make_float4(0.f, 0.f, 0.f, 0.f);
-        myrow[k] = v.x; myrow[k + 1] = v.y; myrow[k + 2] = v.z; myrow[k + 3] = v.w;
+        w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
         mn = fminf(fminf(mn, v.x), fminf(v.y, fminf(v.z, v.w)));
         mx = fmaxf(fmaxf(mx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
     }
-    const bool loaded = mbar_wait(bar, 0, a.st, 201);
-    for (int j = threadIdx.x; j < B; j += ROWS) invd[j] = 1.0f / Us[j * B + j];
+    red[q * SUB + lane] = mn;
+    red[(NWIN + q) * SUB + lane] = mx;
     __syncthreads();
-    if (!loaded || !active) return;
 
-    Grid gr;
-    gr.maxq = a.maxq;
+    // grid of each row (warp 0), handed to the other warps through shared memory
+    float* gsh = red + 2 * NWIN * SUB;
     bool finite = true;
-    if (a.groupsize < 0) {
-        gr.s = __half2float(__ushort_as_half(a.scales[r]));
-        gr.z = __half2float(__ushort_as_half(a.zeros[r]));
-    } else {
-        const size_t gi = size_t(r) * a.n_groups + i0 / a.groupsize;
-        if (i0 % a.groupsize == 0) {
-            // grid from the current weights of the group: this block's columns as
-            // loaded, later columns from W (already lazily updated)
-            for (int c = B; c < a.groupsize; c += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(wsrc + c);
-                mn = fminf(fminf(mn, v.x), fminf(v.y, fminf(v.z, v.w)));
-                mx = fmaxf(fmaxf(mx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
-            }
-            __half s16, z16;
-            finite &= grid_params(mn, mx, a.maxq, gr.s, gr.z, s16, z16);
-            a.scales[gi] = __half_as_ushort(s16);
-            a.zeros[gi] = __half_as_ushort(z16);
+    if (q == 0 && active) {
+        float s, z;
+        if (a.groupsize < 0) {
+            s = __half2float(__ushort_as_half(a.scales[r]));
+            z = __half2float(__ushort_as_half(a.zeros[r]));
         } else {
-            gr.s = __half2float(__ushort_as_half(a.scales[gi]));
-            gr.z = __half2float(__ushort_as_half(a.zeros[gi]));
+            const size_t gi = size_t(r) * a.n_groups + i0 / a.groupsize;
+            if (i0 % a.groupsize == 0) {
+                // grid from the current weights of the group: this block as loaded,
+                // later columns of the group from W (already lazily updated)
+                float gmn = red[lane], gmx = red[NWIN * SUB + lane];
+#pragma unroll
+                for (int p = 1; p < NWIN; ++p) {
+                    gmn = fminf(gmn, red[p * SUB + lane]);
+                    gmx = fmaxf(gmx, red[(NWIN + p) * SUB + lane]);
+                }
+                const float* rowp = a.W + size_t(r) * a.d_in + i0;
+                for (int c = B; c < a.groupsize; c += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(rowp + c);
+                    gmn = fminf(fminf(gmn, v.x), fminf(v.y, fminf(v.z, v.w)));
+                    gmx = fmaxf(fmaxf(gmx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
+                }
+                __half s16, z16;
+                finite &= grid_params(gmn, gmx, a.maxq, s, z, s16, z16);
+                a.scales[gi] = __half_as_ushort(s16);
+                a.zeros[gi] = __half_as_ushort(z16);
+            } else {
+                s = __half2float(__ushort_as_half(a.scales[gi]));
+                z = __half2float(__ushort_as_half(a.zeros[gi]));
+            }
+        }
+        gsh[lane] = s;
+        gsh[SUB + lane] = z;
+    }
+    const bool loaded = mbar_wait(&bars[0], 0, a.st, 201);
+    invd[wc + lane] = loaded ? 1.0f / Us[(wc + lane) * B + wc + lane] : 0.0f;
+    __syncthreads();
+    Grid gr{gsh[lane], gsh[SUB + lane], a.maxq};
+
+    // E of the earlier windows, applied to this window (in window order)
+    for (int p = 0; p < q; ++p) {
+        const bool ready = mbar_wait(&bars[1 + p], 0, a.st, 202);
+        if (!ready) break;
+        const float* eh = Eh + (p * SUB + lane) * ELD;
+#pragma unroll 4
+        for (int j = 0; j < SUB; ++j) {
+            const float e = eh[j];
+            const float4* u4 = reinterpret_cast<const float4*>(Us + (p * SUB + j) * B + wc);
+#pragma unroll
+            for (int k4 = 0; k4 < SUB / 4; ++k4) {
+                const float4 u = u4[k4];
+                w[4 * k4 + 0] = fmaf(-e, u.x, w[4 * k4 + 0]);
+                w[4 * k4 + 1] = fmaf(-e, u.y, w[4 * k4 + 1]);
+                w[4 * k4 + 2] = fmaf(-e, u.z, w[4 * k4 + 2]);
+                w[4 * k4 + 3] = fmaf(-e, u.w, w[4 * k4 + 3]);
+            }
         }
     }
 
-    uint32_t* crow = a.codes + size_t(r) * (size_t(a.d_in) * BITS / 32) + size_t(i0) * BITS / 32;
-    float* erow = a.E + size_t(r) * B;
-    float* qrow = a.Q ? a.Q + size_t(r) * a.d_in + i0 : nullptr;
-#pragma unroll 1
-    for (int sb = 0; sb < B / SUB; ++sb) {
-        const int wc = sb * SUB;
-        float w[SUB];
+    // this window, column by column
+    Packer<BITS> pk;
+    float* qrow = (a.Q && active) ? a.Q + size_t(r) * a.d_in + i0 + wc : nullptr;
+    WindowCol<BITS, 0>::run(w, Us, wc, invd + wc, gr, pk, qrow, finite);
+
+    // hand E to the later windows, then write E and the codes
+    if (q + 1 < NWIN) {
+        float* eh = Eh + (q * SUB + lane) * ELD;
 #pragma unroll
-        for (int j = 0; j < SUB; ++j) w[j] = myrow[wc + j];
-        Packer<BITS> pk;
-        WindowCol<BITS, 0>::run(w, Us, wc, invd, gr, pk, qrow ? qrow + wc : nullptr, finite);
-        pk.store(crow + sb * BITS);
+        for (int j = 0; j < SUB; ++j) eh[j] = w[j];
+        mbar_arrive(&bars[1 + q]);
+    }
+    if (active) {
+        float* erow = a.E + size_t(r) * B + wc;
 #pragma unroll
         for (int j = 0; j < SUB; j += 4)
-            *reinterpret_cast<float4*>(erow + wc + j) = make_float4(w[j], w[j + 1], w[j + 2], w[j + 3]);
-        // this window's E applied to the later columns of the row
-#pragma unroll 2
-        for (int k = wc + SUB; k < B; ++k) {
-            const float4* u4 = reinterpret_cast<const float4*>(UtS + k * B + wc);
-            float acc = myrow[k];
-#pragma unroll
-            for (int jj = 0; jj < SUB / 4; ++jj) {
-                const float4 u = u4[jj];
-                acc = fmaf(-w[4 * jj + 0], u.x, acc);
-                acc = fmaf(-w[4 * jj + 1], u.y, acc);
-                acc = fmaf(-w[4 * jj + 2], u.z, acc);
-                acc = fmaf(-w[4 * jj + 3], u.w, acc);
-            }
-            myrow[k] = acc;
-        }
+            *reinterpret_cast<float4*>(erow + j) = make_float4(w[j], w[j + 1], w[j + 2], w[j + 3]);
+        pk.store(a.codes + size_t(r) * (size_t(a.d_in) * BITS / 32) + size_t(i0 + wc) * BITS / 32);
+        if (!finite) record_error(a.st, GPTQ_ERR_NONFINITE, r);
     }
-    if (!finite) record_error(a.st, GPTQ_ERR_NONFINITE, r);
 }
 
 // RTN: one thread per 32 consecutive codes of a row (one packing unit for
@@ -304,13 +326,12 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
             return GPTQ_ERR_CUDA;
         attr_set[dev] = true;
     }
-    CUtensorMap tmU, tmUt;
-    if (make_map_2d_f32(&tmU, a.U, uint64_t(a.d_in), uint64_t(a.d_in), uint64_t(a.d_in), B, B, false) ||
-        make_map_2d_f32(&tmUt, a.Ut, uint64_t(a.d_in), uint64_t(a.d_in), uint64_t(a.d_in), B, B, false))
+    CUtensorMap tmU;
+    if (make_map_2d_f32(&tmU, a.U, uint64_t(a.d_in), uint64_t(a.d_in), uint64_t(a.d_in), B, B, false))
         return GPTQ_ERR_CUDA;
-    const int blocks = (a.d_out + ROWS - 1) / ROWS;
+    const int blocks = (a.d_out + SUB - 1) / SUB;
     for (int i0 = 0; i0 < a.d_in; i0 += B) {
-        sweep_block_kernel<BITS><<<blocks, ROWS, SMEM, stream>>>(tmU, tmUt, a, i0); count_launch();
+        sweep_block_kernel<BITS><<<blocks, SUB * NWIN, SMEM, stream>>>(tmU, a, i0); count_launch();
         const int tail = a.d_in - i0 - B;
         if (tail > 0) {
             // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]   (U[i0+k][i0+B+n] = Ut[i0+B+n][i0+k])
