@@ -158,6 +158,35 @@ int gptq_quantize_layer(float* W, int64_t d_out, int64_t d_in, const float* U,
                         float* Q, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Stages 3-5 without a caller workspace.  The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory where
+ * they quantize -- code recording into a CUDA stream capture (cudaMalloc is
+ * not allowed there) or a host framework whose memory pool owns every device
+ * buffer and hands out only inputs and outputs.
+ *
+ * Same arguments, results and errors as gptq_quantize_layer, minus ws and
+ * ws_bytes.  The scratch it needs (E [d_out, 128] fp32 and U^T [d_in, d_in]
+ * fp32, each part rounded up to 256 bytes) lives in one 40 MiB device array
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits.  Sizes that need more than 40 MiB (about
+ * d_out * 512 + d_in * d_in * 4 bytes) return GPTQ_ERR_UNSUPPORTED and
+ * launch nothing: e.g. d_in = 3072 works for d_out up to 3072, d_in = 4096
+ * does not fit.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress with that device current); make that first call
+ *    before any stream capture begins.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - All calls on a device share the one array, which keeps the last call's
+ *    contents (nothing in it needs to start at zero).  Calls whose work
+ *    overlaps on the GPU (different streams, not ordered) race on it: order
+ *    them on one stream or with events.
+ * ---------------------------------------------------------------------- */
+int gptq_quantize_layer_noalloc(float* W, int64_t d_out, int64_t d_in, const float* U,
+                                int bits, int blocksize, int groupsize,
+                                uint32_t* codes, uint16_t* scales, uint16_t* zeros,
+                                float* Q, void* stream);
+
+/* ------------------------------------------------------------------------
  * Baseline -- round to nearest on the same grid, no compensation.
  * Source: itwiki "GPTQ", "문제 설정" (RTN moves each weight to its nearest
  * grid point without looking at the inputs).  Group grids come from the

@@ -29,6 +29,8 @@ SIGNATURES = {
     "gptq_quantize_workspace_size": (c_size, [c_i64, c_i64, c_int]),
     "gptq_quantize_layer": (c_int, [c_vp, c_i64, c_i64, c_vp, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp,
                                     c_vp, c_size, c_vp]),
+    "gptq_quantize_layer_noalloc": (c_int, [c_vp, c_i64, c_i64, c_vp, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp,
+                                            c_vp]),
     "gptq_rtn_layer": (c_int, [c_vp, c_i64, c_i64, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "gptq_widen_bf16": (c_int, [c_vp, c_vp, c_i64, c_vp]),
     "gptq_fill_f32": (c_int, [c_vp, c_i64, c_float, c_vp]),

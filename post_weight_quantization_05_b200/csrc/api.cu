@@ -23,6 +23,8 @@ std::atomic<unsigned long long> g_launches{0};
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
 // Device address of this device's status word (looked up once per device,
 // with that device current).
 int status_ptr(DevStatus** out) {
@@ -53,6 +55,7 @@ int encode_fn(PFN_encodeTiled* out) {
     return GPTQ_OK;
 }
 
+namespace {
 inline bool valid_d_in(int64_t d_in) { return d_in >= 128 && d_in <= 32768 && d_in % 128 == 0; }
 inline bool valid_bits(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 8; }
 inline bool valid_group(int g, int64_t d_in) { return g == -1 || (g > 0 && g % 128 == 0 && d_in % g == 0); }
@@ -60,6 +63,19 @@ inline bool valid_group(int g, int64_t d_in) { return g == -1 || (g > 0 && g % 1
 }  // namespace
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int validate_quantize_args(const float* W, int64_t d_out, int64_t d_in, const float* U, int bits, int blocksize,
+                           int groupsize, const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                           const float* Q) {
+    if (d_out <= 0 || d_out > (int64_t(1) << 24) || !valid_d_in(d_in)) return GPTQ_ERR_INVALID_ARG;
+    if (!valid_bits(bits) || !valid_group(groupsize, d_in)) return GPTQ_ERR_INVALID_ARG;
+    if (blocksize != 128) return GPTQ_ERR_UNSUPPORTED;
+    if (!W || !U || !codes || !scales || !zeros) return GPTQ_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(U) || !aligned16(codes) || (Q && !aligned16(Q)) ||
+        (reinterpret_cast<uintptr_t>(scales) & 1u) || (reinterpret_cast<uintptr_t>(zeros) & 1u))
+        return GPTQ_ERR_INVALID_ARG;
+    return GPTQ_OK;
+}
 
 }  // namespace gptq
 
@@ -130,14 +146,9 @@ size_t gptq_quantize_workspace_size(int64_t d_out, int64_t d_in, int blocksize) 
 int gptq_quantize_layer(float* W, int64_t d_out, int64_t d_in, const float* U, int bits, int blocksize,
                         int groupsize, uint32_t* codes, uint16_t* scales, uint16_t* zeros, float* Q, void* ws,
                         size_t ws_bytes, void* stream) {
-    if (d_out <= 0 || d_out > (int64_t(1) << 24) || !valid_d_in(d_in)) return GPTQ_ERR_INVALID_ARG;
-    if (!valid_bits(bits) || !valid_group(groupsize, d_in)) return GPTQ_ERR_INVALID_ARG;
-    if (blocksize != 128) return GPTQ_ERR_UNSUPPORTED;
-    if (!W || !U || !codes || !scales || !zeros || !ws) return GPTQ_ERR_INVALID_ARG;
-    if (!aligned16(W) || !aligned16(U) || !aligned16(codes) || !aligned16(ws) || (Q && !aligned16(Q)) ||
-        (reinterpret_cast<uintptr_t>(scales) & 1u) || (reinterpret_cast<uintptr_t>(zeros) & 1u))
-        return GPTQ_ERR_INVALID_ARG;
-    if (ws_bytes < sweep_workspace_bytes(d_out, d_in)) return GPTQ_ERR_INVALID_ARG;
+    const int v = validate_quantize_args(W, d_out, d_in, U, bits, blocksize, groupsize, codes, scales, zeros, Q);
+    if (v) return v;
+    if (!ws || !aligned16(ws) || ws_bytes < sweep_workspace_bytes(d_out, d_in)) return GPTQ_ERR_INVALID_ARG;
     DevStatus* st = nullptr;
     PFN_encodeTiled enc = nullptr;
     if (status_ptr(&st) || encode_fn(&enc)) return GPTQ_ERR_CUDA;

@@ -14,9 +14,18 @@ struct DevStatus;
 // Host-side count of kernels enqueued by this library (gptq_launch_count).
 void count_launch();
 
+
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                     const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// api.cu: this device's status word, the driver's tensor-map encoder, and
+// the host-side checks of gptq_quantize_layer's arguments (all but ws).
+int status_ptr(DevStatus** out);
+int encode_fn(PFN_encodeTiled* out);
+int validate_quantize_args(const float* W, int64_t d_out, int64_t d_in, const float* U, int bits, int blocksize,
+                           int groupsize, const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                           const float* Q);
 
 // hessian.cu
 int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, void* ws, cudaStream_t stream,
