@@ -163,6 +163,29 @@ def run_reference(args):
     return 0
 
 
+# --------------------------------------------------------------------------- profiling case
+def run_profile_case():
+    """The per-launch shape of the benchmark (one 16384 x 4096 bf16 batch, the
+    same 4096 x 4096 layer) run three times end to end, for ncu captures of
+    single kernels (a few hundred MB on the device)."""
+    import torch
+
+    from post_weight_quantization_05_b200 import api, build_lib, synth
+    build_lib.build()
+    torch.cuda.set_device(0)
+    p = synth.attn4096(n_batches=1)
+    x = torch.from_numpy(p.x_batch(0).view(np.int16)).cuda().view(torch.bfloat16)
+    w = torch.from_numpy(synth.f32_to_bf16_bits(p.W).view(np.int16)).cuda().view(torch.bfloat16)
+    lq = api.LayerQuantizer(p.d_out, p.d_in, p.bits, p.groupsize, p.blocksize, p.percdamp)
+    for _ in range(3):
+        lq.begin(w)
+        lq.add_batch(x)
+        lq.finish()
+    api.get_status()
+    print("profile case done")
+    return 0
+
+
 # --------------------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -172,9 +195,13 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="small case for ncu captures: one 16384-row batch of the same layer, 3 passes, no timing")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_case:
+        return run_profile_case()
 
     import torch
     import torch.distributed as dist

@@ -285,3 +285,49 @@ def test_attn4096_full_size_sampled_rows():
     lg = oracle.layer_loss_hessian(p.W[rows], Qg, H)
     lo = oracle.layer_loss_hessian(p.W[rows], ref["Q"], H)
     assert abs(lg / lo - 1.0) <= LOSS_TOL
+
+
+def _oracle_h_syrk(p, xs):
+    """H = sum 2 X^T X in fp64 (upper triangle by dsyrk, then mirrored)."""
+    d = p.d_in
+    Hu = np.zeros((d, d), dtype=np.float64, order="F")
+    for x in xs:
+        xf = np.asfortranarray(synth.x_as_f32(p, x).astype(np.float64))
+        Hu = blas.dsyrk(2.0, xf, beta=1.0, c=Hu, trans=1, lower=0, overwrite_c=1)
+        del xf
+    return np.triu(Hu) + np.triu(Hu, 1).T
+
+
+def _full_size_check(p, n_rows_sample=48, seed=0):
+    xs = synth.x_batches_threaded(p, 8)
+    lq = _gpu_pipeline(p, [to_dev_x(p, x) for x in xs], want_q=False)
+    H = _oracle_h_syrk(p, xs)
+    del xs
+    assert rel_fro(upper(lq.H.cpu().numpy()), upper(H)) <= H_TOL
+    Hd, _ = oracle.damp(H, p.percdamp)
+    U = oracle.hinv_upper_factor_ul(Hd)
+    assert rel_fro(lq.U.cpu().numpy(), U) <= U_TOL
+    rows = np.random.default_rng(seed).choice(p.d_out, size=n_rows_sample, replace=False)
+    ref = oracle.gptq_quantize(p.W[rows], U, p.bits, 128, p.groupsize, return_trace=True)
+    got = unpack_gpu_codes(lq.codes, p.bits, p.d_in)[rows]
+    s = fp16_values(lq.scales)[rows]
+    z = fp16_values(lq.zeros)[rows]
+    check_codes(got, ref, p.name, groupsize=p.groupsize, gpu_scales=s, gpu_zeros=z)
+    Qg = dequant_rows(got, s, z, p.groupsize)
+    lg = oracle.layer_loss_hessian(p.W[rows], Qg, H)
+    lo = oracle.layer_loss_hessian(p.W[rows], ref["Q"], H)
+    assert abs(lg / lo - 1.0) <= LOSS_TOL, (lg, lo)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("which,bits", [("up", 4), ("down", 3)])
+def test_mlp11008_full_size_sampled_rows(which, bits):
+    """The Llama-7B MLP pair with heavy-tailed (Student-t) activations and 1%
+    outlier channels x20, 65536 calibration rows."""
+    _full_size_check(synth.mlp11008(which, bits))
+
+
+@pytest.mark.slow
+def test_mlp28672_full_size_sampled_rows():
+    """The 8192 x 28672 layer (H and U of 3.3 GB each), 65536 rows in 8 batches."""
+    _full_size_check(synth.mlp28672(), n_rows_sample=16)
