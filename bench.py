@@ -44,6 +44,25 @@ WORKLOAD = ("attn4096: W [4096,4096] bf16 ~N(0,0.02^2), X [262144,4096] bf16 AR(
             "in 16 batches of 16384, 4-bit, groupsize 128, B=128, percdamp 0.01")
 
 
+def syrk_traffic_per_launch():
+    """DRAM bytes (read + write) of one X^T X launch from the committed ncu
+    summary, or None if the kernel's sources changed since that capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "syrk_kernel_attn4096.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = dict(line.split(": ", 1) for line in text.splitlines() if line.startswith(("traffic_", "kernel_source")))
+    h = hashlib.sha256()
+    for f in ("hessian.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "post_weight_quantization_05_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if vals.get("kernel_source_hash") != h.hexdigest()[:16]:
+        return None
+    return int(vals["traffic_bytes_per_launch"])
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -302,7 +321,8 @@ def main():
     achieved = flops_per_launch / (h_launch_avg / 1e3) / 1e12
     roof = {"kernel": "hessian syrk_kernel (tcgen05)", "bound": "tensor", "achieved": achieved,
             "peak": sustained, "unit": "TFLOP/s", "frac": achieved / sustained,
-            "peak_kind": f"bf16 dense sustained ({src})", "traffic": None,
+            "peak_kind": f"bf16 dense sustained ({src})", "traffic": syrk_traffic_per_launch(),
+            "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             "algorithmic_per_launch": f"{flops_per_launch:.4e} flop ({n_b}x{p.d_in}x{p.d_in + 1})",
             "avg_launch_ms": h_launch_avg}
 
