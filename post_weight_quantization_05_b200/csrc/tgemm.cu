@@ -17,8 +17,8 @@
 // and MMAs run while tile i's epilogue drains.  Both operands are K-major: A[m * lda + k] and B(k, n) = Bt[n * ldb + k]
 // (an MN-major tf32 operand would need a different shared-memory layout, so
 // the callers arrange their data to avoid it).  Warp roles: one TMA producer
-// (no multicast), eight warps that split each chunk into hi (in place) / lo
-// (two rotating buffers), one MMA issuer, eight epilogue warps.  K must be a
+// (no multicast), six warps that split each chunk into hi (in place) / lo
+// (two rotating buffers), one MMA issuer, four epilogue warps.  K must be a
 // multiple of 32 and at most 128.
 #include "common.cuh"
 #include "kernels.h"
@@ -33,15 +33,14 @@ constexpr int LO_BUFS = 2;                         // lo parts, rotating
 constexpr int A_BYTES = BM * BKC * 4;              // 16 KB
 constexpr int B_BYTES = BN * BKC * 4;              // 16 KB
 constexpr int CHUNK_BYTES = A_BYTES + B_BYTES;
-constexpr int CONV_WARPS = 8;                      // warps 0-7 split chunks into hi / lo
-constexpr int MMA_WARP = CONV_WARPS;               // warp 8 issues the MMAs
-constexpr int PRODUCER_WARP = CONV_WARPS + 1;      // warp 9 issues TMA
-constexpr int EPI_WARP0 = CONV_WARPS + 2;          // warps 10-17 drain TMEM: lane quadrant warp % 4,
-constexpr int EPI_WARPS = 8;                       // column half (warp - 10) / 4
+constexpr int CONV_WARPS = 6;                      // warps 0-5 split chunks into hi / lo
+constexpr int MMA_WARP = CONV_WARPS;               // warp 6 issues the MMAs
+constexpr int PRODUCER_WARP = CONV_WARPS + 1;      // warp 7 issues TMA
+constexpr int EPI_WARP0 = 8;                       // warps 8-15 drain TMEM: lane quadrant warp % 4,
+constexpr int EPI_WARPS = 8;                       // column half (warp - 8) / 4
 constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
 constexpr int TMEM_COLS = 2 * BN;                  // two accumulators: tile i+1 runs while tile i drains
-constexpr int XLD = 33;                            // epilogue transpose buffer row (conflict-free)
-constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES + LO_BUFS) * CHUNK_BYTES + size_t(EPI_WARPS) * 32 * XLD * 4 + 256;
+constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES + LO_BUFS) * CHUNK_BYTES + 512;
 
 // instruction descriptor: tf32 x tf32 -> f32, A and B K-major, M = BM, N = BN
 __host__ __device__ constexpr uint32_t idesc_tf32() {
@@ -106,8 +105,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* lo_base = smem + size_t(STAGES) * CHUNK_BYTES;
-    float* xbuf = reinterpret_cast<float*>(lo_base + size_t(LO_BUFS) * CHUNK_BYTES);          // [EPI_WARPS][32][XLD]
-    uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + EPI_WARPS * 32 * XLD);               // [STAGES] TMA landed
+    uint64_t* full = reinterpret_cast<uint64_t*>(lo_base + size_t(LO_BUFS) * CHUNK_BYTES);  // [STAGES] TMA landed
     uint64_t* conv = full + STAGES;          // [STAGES] one arrival per split warp: chunk split into hi / lo
     uint64_t* empty = conv + STAGES;         // [STAGES] MMA commit: stage may be reloaded
     uint64_t* lo_free = empty + STAGES;      // [LO_BUFS] MMA commit: lo buffer may be rewritten
@@ -221,41 +219,53 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ---------------- epilogue warps: TMEM lanes (warp % 4) * 32 .. + 31 = tile rows,
-        // columns half * 64 .. + 63.  Each 32 x 32 piece goes through a small
-        // shared-memory transpose so that every global load / store of C is one
-        // 128-byte row segment per warp (coalesced).
+        // columns half * 64 .. + 63
         const int quad = warp & 3;
         const int half = (warp - EPI_WARP0) >> 2;
-        constexpr int HC = BN / 2;   // columns per epilogue warp
-        float* xb = xbuf + (warp - EPI_WARP0) * 32 * XLD;
+        constexpr int HC = BN / 2;   // columns per epilogue thread
         for (int lt = 0; lt < my_tiles; ++lt) {
             const int acc = lt & 1;
             const uint32_t use = uint32_t(lt >> 1);
             int tm, tn;
             tile_coords(int(blockIdx.x) + lt * int(gridDim.x), g, tm, tn);
-            const int row0 = tm * BM + quad * 32;
+            const int m = tm * BM + quad * 32 + lane;
+            const int n0 = tn * BN + half * HC;
+            const bool in_range = m < g.M;
+            const bool full_row = in_range && n0 + HC <= g.N;
+            // C_in for this tile now, so that the loads overlap the tile's MMAs
+            float4 ci[HC / 4];
+            if (full_row && g.beta != 0.0f) {
+                const float4* src = reinterpret_cast<const float4*>(g.C_in + size_t(m) * g.ldc + n0);
+#pragma unroll
+                for (int q = 0; q < HC / 4; ++q) ci[q] = src[q];
+            } else {
+#pragma unroll
+                for (int q = 0; q < HC / 4; ++q) ci[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+            __syncwarp();
             if (!mbar_wait(&tfull[acc], use & 1u, g.st, 305)) break;
             tc_fence_after();
-#pragma unroll 1
+#pragma unroll
             for (int cc = 0; cc < HC / 32; ++cc) {
-                const int n = tn * BN + half * HC + cc * 32;
+                const int n = n0 + cc * 32;
                 float v[32];
                 tmem_ld_32x32b_x32(tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + half * HC + cc * 32), v);
+                if (!in_range) continue;
+                float* cout = g.C_out + size_t(m) * g.ldc + n;
+                if (full_row) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) xb[lane * XLD + j] = v[j];     // row = lane
-                __syncwarp();
-                const int col = n + lane;
-                const bool col_ok = col < g.N;
-#pragma unroll 8
-                for (int r = 0; r < 32; ++r) {
-                    const int row = row0 + r;
-                    if (col_ok && row < g.M) {
-                        const size_t off = size_t(row) * g.ldc + col;
-                        const float c = g.beta != 0.0f ? g.beta * g.C_in[off] : 0.0f;
-                        g.C_out[off] = fmaf(g.alpha, xb[r * XLD + lane], c);
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 c4 = ci[cc * 8 + q];
+                        *reinterpret_cast<float4*>(cout + 4 * q) =
+                            make_float4(fmaf(g.alpha, v[4 * q], g.beta * c4.x), fmaf(g.alpha, v[4 * q + 1], g.beta * c4.y),
+                                        fmaf(g.alpha, v[4 * q + 2], g.beta * c4.z), fmaf(g.alpha, v[4 * q + 3], g.beta * c4.w));
                     }
+                } else {
+                    const float* cin = g.C_in + size_t(m) * g.ldc + n;
+#pragma unroll
+                    for (int q = 0; q < 32; ++q)
+                        if (n + q < g.N) cout[q] = fmaf(g.alpha, v[q], g.beta != 0.0f ? g.beta * cin[q] : 0.0f);
                 }
-                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
