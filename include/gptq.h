@@ -165,13 +165,14 @@ int gptq_quantize_layer(float* W, int64_t d_out, int64_t d_in, const float* U,
  * buffer and hands out only inputs and outputs.
  *
  * Same arguments, results and errors as gptq_quantize_layer, minus ws and
- * ws_bytes.  The scratch it needs (E [d_out, 128] fp32 and U^T [d_in, d_in]
- * fp32, each part rounded up to 256 bytes) lives in one 40 MiB device array
- * inside the library, which every GPU that loads the library holds until the
- * process exits.  Sizes that need more than 40 MiB (about
- * d_out * 512 + d_in * d_in * 4 bytes) return GPTQ_ERR_UNSUPPORTED and
- * launch nothing: e.g. d_in = 3072 works for d_out up to 3072, d_in = 4096
- * does not fit.
+ * ws_bytes.  The scratch it needs (E [d_out, 128] and U^T [d_in, d_in], each
+ * kept as two fp32 arrays -- the tf32-rounded part and the remainder -- for
+ * the tensor-core trailing product, each array rounded up to 256 bytes)
+ * lives in one 40 MiB device array inside the library, which every GPU that
+ * loads the library holds until the process exits.  Sizes that need more than
+ * 40 MiB (about d_out * 1024 + d_in * d_in * 8 bytes) return
+ * GPTQ_ERR_UNSUPPORTED and launch nothing: e.g. d_in = 2048 works for d_out
+ * up to 8192, d_in = 3072 does not fit.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress with that device current); make that first call
  *    before any stream capture begins.

@@ -478,7 +478,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
             // panel <- panel * Dinv_k^T.  In place is safe: N = NB is one output
             // tile column, so each CTA reads only the rows it writes, all before
             // its epilogue.
-            rc = launch_tgemm(rest, NB, NB, 1.0f, panel, d, dk, NB, true, 0.0f, panel, panel, d, false, stream, st);
+            rc = launch_tgemm(rest, NB, NB, 1.0f, panel, nullptr, d, dk, nullptr, NB, false, panel, d, false, stream, st);
             if (rc) return rc;
         }
         if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->step, 0) != cudaSuccess)
@@ -487,14 +487,14 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
             // next block column (it holds the next diagonal block) on `stream` ...
             if (cudaStreamWaitEvent(stream, aux->rest, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
             float* next = A + size_t(k0 + NB) * d + k0 + NB;
-            rc = launch_tgemm(rest, NB, NB, -1.0f, panel, d, panel, d, true, 1.0f, next, next, d, true, stream, st);
+            rc = launch_tgemm(rest, NB, NB, -1.0f, panel, nullptr, d, panel, nullptr, d, true, next, d, true, stream, st);
             if (rc) return rc;
             // ... the columns after it on `ss`
             if (rest > NB) {
                 if (cudaStreamWaitEvent(ss, aux->step, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
                 float* far = A + size_t(k0 + 2 * NB) * d + k0 + 2 * NB;
                 const float* prow = panel + size_t(NB) * d;
-                rc = launch_tgemm(rest - NB, rest - NB, NB, -1.0f, prow, d, prow, d, true, 1.0f, far, far, d, true,
+                rc = launch_tgemm(rest - NB, rest - NB, NB, -1.0f, prow, nullptr, d, prow, nullptr, d, true, far, d, true,
                                   ss, st);
                 if (rc) return rc;
                 if (cudaEventRecord(aux->rest, ss) != cudaSuccess) return GPTQ_ERR_CUDA;
@@ -504,12 +504,12 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         place_diag_inverse_t_kernel<<<1, 512, NB * LD * sizeof(float), as>>>(dk, d, k, Z); count_launch();
         if (k > 0) {
             float* zi = Z + k0;   // in place is safe for the same reason as the panel
-            rc = launch_tgemm(k0, NB, NB, 1.0f, zi, d, dk, NB, true, 0.0f, zi, zi, d, false, as, st);
+            rc = launch_tgemm(k0, NB, NB, 1.0f, zi, nullptr, d, dk, nullptr, NB, false, zi, d, false, as, st);
             if (rc) return rc;
         }
         if (rest > 0) {
             float* zc = Z + k0 + NB;
-            rc = launch_tgemm(k0 + NB, rest, NB, -1.0f, Z + k0, d, panel, d, true, 1.0f, zc, zc, d, false, as, st);
+            rc = launch_tgemm(k0 + NB, rest, NB, -1.0f, Z + k0, nullptr, d, panel, nullptr, d, true, zc, d, false, as, st);
             if (rc) return rc;
         }
     }

@@ -31,19 +31,22 @@ int validate_quantize_args(const float* W, int64_t d_out, int64_t d_in, const fl
 int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, void* ws, cudaStream_t stream,
                    DevStatus* st, PFN_encodeTiled encode);
 
-// tgemm.cu: C[M,N] = alpha * A[M,K] * B + beta * C_in with B(k, n) =
-// Bt[n * ldb + k] (trans_b must be true), fp32 row-major, on the tensor cores
-// (kind::tf32, hi/lo split, three passes; fp32-class accuracy).  K must be a
-// multiple of 32; pointers and leading dimensions must satisfy TMA's 16-byte
-// rules.  lower_only skips 128 x 128 output tiles entirely above the
-// diagonal.  C_out may alias C_in.
+// tgemm.cu: C[M,N] = alpha * A[M,K] * B (accumulate = false) or
+// C[M,N] += alpha * A[M,K] * B (accumulate = true), B(k, n) = Bt[n * ldb + k],
+// fp32 row-major, on the tensor cores (kind::tf32, hi/lo split, three passes;
+// fp32-class accuracy).  A_lo / Bt_lo null: the kernel splits A and Bt itself;
+// both non-null: A and Bt hold the tf32-rounded hi parts and A_lo / Bt_lo the
+// remainders (split_tf32).  K must be a multiple of 32; pointers and leading
+// dimensions must satisfy TMA's 16-byte rules.  lower_only skips 128 x 128
+// output tiles entirely above the diagonal.  C may be one of the operands when
+// N <= 128 (each CTA then reads only the rows it writes, before writing them).
 void set_tensor_map_encoder(PFN_encodeTiled f);
 // 2-D fp32 tensor map (row stride ld_elems), 128-byte swizzle or none.
 int make_map_2d_f32(CUtensorMap* tm, const float* base, uint64_t inner, uint64_t outer, uint64_t ld_elems,
                     uint32_t box_inner, uint32_t box_outer, bool swizzle128);
-int launch_tgemm(int M, int N, int K, float alpha, const float* A, int lda, const float* B, int ldb, bool trans_b,
-                 float beta, const float* C_in, float* C_out, int ldc, bool lower_only, cudaStream_t stream,
-                 DevStatus* st);
+int launch_tgemm(int M, int N, int K, float alpha, const float* A, const float* A_lo, int lda, const float* Bt,
+                 const float* Bt_lo, int ldb, bool accumulate, float* C, int ldc, bool lower_only,
+                 cudaStream_t stream, DevStatus* st);
 
 // factor.cu
 size_t factor_workspace_bytes(int64_t d);

@@ -117,14 +117,16 @@ struct WindowCol {
 struct SweepArgs {
     float* W;
     const float* U;
-    const float* Ut;
+    const float* Ut;     // [d_in, d_in] tf32-rounded hi parts of U^T (lazy trailing update)
+    const float* Ut_lo;  // and their remainders
     int d_out, d_in, groupsize, n_groups;
     float maxq;
     uint32_t* codes;
     uint16_t* scales;
     uint16_t* zeros;
     float* Q;
-    float* E;  // [d_out, B]
+    float* E;     // [d_out, B] hi parts of the block's E (tf32-rounded)
+    float* E_lo;  // [d_out, B] remainders
     DevStatus* st;
 };
 
@@ -249,10 +251,17 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
         mbar_arrive(&bars[1 + q]);
     }
     if (active) {
+        // E leaves pre-split for the trailing product's tensor cores
         float* erow = a.E + size_t(r) * B + wc;
+        float* elo = a.E_lo + size_t(r) * B + wc;
 #pragma unroll
-        for (int j = 0; j < SUB; j += 4)
-            *reinterpret_cast<float4*>(erow + j) = make_float4(w[j], w[j + 1], w[j + 2], w[j + 3]);
+        for (int j = 0; j < SUB; j += 4) {
+            float4 h, l;
+            split_tf32(w[j], h.x, l.x); split_tf32(w[j + 1], h.y, l.y);
+            split_tf32(w[j + 2], h.z, l.z); split_tf32(w[j + 3], h.w, l.w);
+            *reinterpret_cast<float4*>(erow + j) = h;
+            *reinterpret_cast<float4*>(elo + j) = l;
+        }
         pk.store(a.codes + size_t(r) * (size_t(a.d_in) * BITS / 32) + size_t(i0 + wc) * BITS / 32);
         if (!finite) record_error(a.st, GPTQ_ERR_NONFINITE, r);
     }
@@ -302,17 +311,23 @@ __global__ void fill_kernel(float* __restrict__ p, size_t n, float v) {
         p[i] = v;
 }
 
-// Ut[c][r] = U[r][c] for the tiles of U that reach the upper triangle (the
-// trailing products read U's rows as K-major operands through Ut).
-__global__ void transpose_upper_kernel(const float* __restrict__ U, int d, float* __restrict__ Ut) {
+// Ut[c][r] + Ut_lo[c][r] = U[r][c] (hi / lo split) for the tiles of U that
+// reach the upper triangle (the trailing products read U's rows as K-major
+// operands through Ut).
+__global__ void transpose_upper_kernel(const float* __restrict__ U, int d, float* __restrict__ Ut,
+                                       float* __restrict__ Ut_lo) {
     __shared__ float tile[32][33];
     const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
     if (c0 + 31 < r0) return;
     for (int rr = threadIdx.y; rr < 32; rr += blockDim.y)
         tile[rr][threadIdx.x] = U[size_t(r0 + rr) * d + c0 + threadIdx.x];
     __syncthreads();
-    for (int cc = threadIdx.y; cc < 32; cc += blockDim.y)
-        Ut[size_t(c0 + cc) * d + r0 + threadIdx.x] = tile[threadIdx.x][cc];
+    for (int cc = threadIdx.y; cc < 32; cc += blockDim.y) {
+        float h, l;
+        split_tf32(tile[threadIdx.x][cc], h, l);
+        Ut[size_t(c0 + cc) * d + r0 + threadIdx.x] = h;
+        Ut_lo[size_t(c0 + cc) * d + r0 + threadIdx.x] = l;
+    }
 }
 
 template <int BITS>
@@ -336,8 +351,9 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
         if (tail > 0) {
             // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]   (U[i0+k][i0+B+n] = Ut[i0+B+n][i0+k])
             float* c = a.W + i0 + B;
-            const int rc = launch_tgemm(a.d_out, tail, B, -1.0f, a.E, B, a.Ut + size_t(i0 + B) * a.d_in + i0, a.d_in,
-                                        true, 1.0f, c, c, a.d_in, false, stream, a.st);
+            const size_t ut = size_t(i0 + B) * a.d_in + i0;
+            const int rc = launch_tgemm(a.d_out, tail, B, -1.0f, a.E, a.E_lo, B, a.Ut + ut, a.Ut_lo + ut, a.d_in,
+                                        true, c, a.d_in, false, stream, a.st);
             if (rc) return rc;
         }
     }
@@ -346,10 +362,13 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
 
 }  // namespace sweep
 
-// E [d_out, B] fp32, then U^T [d_in, d_in] fp32 (256-byte aligned)
+// E hi, E lo [d_out, B] fp32, then U^T hi, U^T lo [d_in, d_in] fp32 (each 256-byte aligned)
+namespace {
+size_t e_bytes(int64_t d_out) { return (size_t(d_out) * sweep::B * sizeof(float) + 255) & ~size_t(255); }
+}  // namespace
+
 size_t sweep_workspace_bytes(int64_t d_out, int64_t d_in) {
-    const size_t e = (size_t(d_out) * sweep::B * sizeof(float) + 255) & ~size_t(255);
-    return e + size_t(d_in) * size_t(d_in) * sizeof(float);
+    return 2 * e_bytes(d_out) + 2 * size_t(d_in) * size_t(d_in) * sizeof(float);
 }
 
 int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int bits, int groupsize,
@@ -368,17 +387,20 @@ int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int b
     a.scales = scales;
     a.zeros = zeros;
     a.Q = Q;
-    a.E = static_cast<float*>(ws);
-    a.st = st;
-    float* Ut = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                         ((size_t(d_out) * B * sizeof(float) + 255) & ~size_t(255)));
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    a.E = reinterpret_cast<float*>(wsb);
+    a.E_lo = reinterpret_cast<float*>(wsb + e_bytes(d_out));
+    float* Ut = reinterpret_cast<float*>(wsb + 2 * e_bytes(d_out));
+    float* Ut_lo = Ut + size_t(d_in) * size_t(d_in);
     a.Ut = Ut;
+    a.Ut_lo = Ut_lo;
+    a.st = st;
     if (groupsize < 0) {
         const int warps = a.d_out;
         grid_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(W, a.d_out, a.d_in, a.d_in, 1, a.maxq, scales,
                                                                   zeros, st); count_launch();
     }
-    transpose_upper_kernel<<<dim3(unsigned(d_in / 32), unsigned(d_in / 32)), dim3(32, 8), 0, stream>>>(U, int(d_in), Ut);
+    transpose_upper_kernel<<<dim3(unsigned(d_in / 32), unsigned(d_in / 32)), dim3(32, 8), 0, stream>>>(U, int(d_in), Ut, Ut_lo);
     count_launch();
     switch (bits) {
         case 2: return run_sweep<2>(a, stream);

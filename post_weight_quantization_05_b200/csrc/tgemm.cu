@@ -1,46 +1,71 @@
 // fp32-accurate GEMM on the tcgen05 tensor cores (kind::tf32, three passes).
 //
-// C[M,N] = beta * C_in + alpha * A[M,K] * op(B)[K,N]   (row-major, fp32)
+// C[M,N] = alpha * A[M,K] * op(B)[K,N]        (accumulate = false)
+// C[M,N] += alpha * A[M,K] * op(B)[K,N]       (accumulate = true)
+// row-major fp32, op(B)(k, n) = Bt[n * ldb + k].
 //
 // Every product in the factorization and in the sweep's lazy trailing update
 // ([wiki] "알고리즘": W[:, i+B:] -= E U[i:i+B, i+B:]) needs about fp32
 // accuracy: a single bf16 or tf32 product changes GPTQ codes.  Each operand x
-// is split in shared memory into hi = x rounded to tf32 and lo = x - hi
-// (exact in fp32; the MMA reads its leading 19 bits), and the product is
-// accumulated as  A_hi B_hi + A_hi B_lo + A_lo B_hi  in fp32 TMEM, which is
-// accurate to about 2^-21 relative (the dropped A_lo B_lo term and the tf32
-// reading of the lo parts), comparable to an fp32 FMA chain of length K.
+// is split into hi = x rounded to tf32 and lo = x - hi (exact in fp32; the MMA
+// reads its leading 19 bits), and the product is accumulated as
+// A_hi B_hi + A_hi B_lo + A_lo B_hi  in fp32 TMEM, which is accurate to about
+// 2^-21 relative (the dropped A_lo B_lo term and the tf32 reading of the lo
+// parts), comparable to an fp32 FMA chain of length K.
+//
+// Two ways to get the split:
+//  - pre-split: the caller stores hi and lo in global memory (the sweep writes
+//    E that way and transposes U that way); TMA brings all four operand parts
+//    and no thread touches them, which keeps shared memory free for the MMAs
+//    (at M = N = 128 the tf32 MMAs alone need most of its bandwidth);
+//  - in-kernel: six warps split each TMA-loaded chunk into hi (in place) and lo
+//    (two rotating buffers), for operands that other kernels produce as plain
+//    fp32 (the factorization).
 //
 // Persistent kernel: one CTA per SM walks its share of the 128 x 128 output
-// tiles; K <= 128 in chunks of 32 (one 128-byte swizzle row of fp32) flows
-// through a 4-stage ring, and two TMEM accumulators let tile i+1's loads, split
-// and MMAs run while tile i's epilogue drains.  Both operands are K-major: A[m * lda + k] and B(k, n) = Bt[n * ldb + k]
-// (an MN-major tf32 operand would need a different shared-memory layout, so
-// the callers arrange their data to avoid it).  Warp roles: one TMA producer
-// (no multicast), six warps that split each chunk into hi (in place) / lo
-// (two rotating buffers), one MMA issuer, four epilogue warps.  K must be a
-// multiple of 32 and at most 128.
+// tiles; K in chunks of 32 (one 128-byte swizzle row of fp32) flows through a
+// ring of stages, and two TMEM accumulators let tile i+1's loads and MMAs run
+// while tile i's epilogue drains.  Both operands are K-major (an MN-major tf32
+// operand would need a different shared-memory layout, so the callers arrange
+// their data to avoid it).  The epilogue moves the accumulator to shared memory
+// 32 columns at a time (128-byte swizzle, conflict-free) and writes it with one
+// TMA store, or one TMA reduce-add when accumulating, so C leaves the SM as
+// whole lines and is never read by the SM.  No TMA load uses multicast.
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace gptq {
 namespace tg {
 
-constexpr int BM = 128, BN = 128, BKC = 32;       // tile, K chunk (fp32 elements)
-constexpr int MAX_K = 128;                         // K <= 128 (every caller uses 128)
-constexpr int STAGES = 4;                          // ring of fp32 chunks (each becomes its hi part in place)
-constexpr int LO_BUFS = 2;                         // lo parts, rotating
-constexpr int A_BYTES = BM * BKC * 4;              // 16 KB
-constexpr int B_BYTES = BN * BKC * 4;              // 16 KB
-constexpr int CHUNK_BYTES = A_BYTES + B_BYTES;
-constexpr int CONV_WARPS = 6;                      // warps 0-5 split chunks into hi / lo
-constexpr int MMA_WARP = CONV_WARPS;               // warp 6 issues the MMAs
-constexpr int PRODUCER_WARP = CONV_WARPS + 1;      // warp 7 issues TMA
-constexpr int EPI_WARP0 = 8;                       // warps 8-15 drain TMEM: lane quadrant warp % 4,
-constexpr int EPI_WARPS = 8;                       // column half (warp - 8) / 4
-constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
+constexpr int BM = 128, BN = 128, BKC = 32;        // tile, K chunk (fp32 elements)
+constexpr int MAX_K = 8192;
+constexpr int PART_BYTES = BM * BKC * 4;           // one 128 x 32 fp32 operand part: 16 KB
+constexpr int EPI_WARPS = 4;                       // one per TMEM lane quadrant
+constexpr int SLAB = 32;                           // epilogue columns per TMA store
+constexpr int SLAB_BYTES = BM * SLAB * 4;          // 16 KB
+constexpr int SLAB_BUFS = 2;
 constexpr int TMEM_COLS = 2 * BN;                  // two accumulators: tile i+1 runs while tile i drains
-constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES + LO_BUFS) * CHUNK_BYTES + 512;
+constexpr int EPI_BARRIER = 1;                     // named barrier of the epilogue warps
+
+// Shared-memory and warp layout of the two variants.
+template <bool PRESPLIT>
+struct Cfg {
+    // pre-split: a stage holds A_hi, B_hi, A_lo, B_lo of one chunk.
+    // in-kernel: a stage holds A, B (split to hi in place); lo goes to LO_BUFS buffers.
+    static constexpr int STAGE_BYTES = PRESPLIT ? 4 * PART_BYTES : 2 * PART_BYTES;
+    static constexpr int STAGES = PRESPLIT ? 3 : 4;
+    static constexpr int LO_BUFS = PRESPLIT ? 0 : 2;
+    static constexpr int CONV_WARPS = PRESPLIT ? 0 : 6;
+    static constexpr int MMA_WARP = CONV_WARPS;
+    static constexpr int PRODUCER_WARP = CONV_WARPS + 1;
+    static constexpr int EPI_WARP0 = PRESPLIT ? 4 : 8;   // multiple of 4: warp % 4 = TMEM lane quadrant
+    static constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
+    static constexpr size_t SMEM_BYTES =
+        1024 + size_t(STAGES) * STAGE_BYTES + size_t(LO_BUFS) * 2 * PART_BYTES + size_t(SLAB_BUFS) * SLAB_BYTES + 256;
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
 
 // instruction descriptor: tf32 x tf32 -> f32, A and B K-major, M = BM, N = BN
 __host__ __device__ constexpr uint32_t idesc_tf32() {
@@ -58,24 +83,10 @@ __device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// x -> (hi, lo): hi = x rounded to the nearest tf32 value (ties away), lo = x - hi.
-__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
-    const uint32_t u = __float_as_uint(x);
-    const uint32_t h = (u + 0x1000u) & 0xFFFFE000u;
-    hi = isfinite(x) ? __uint_as_float(h) : x;
-    lo = isfinite(x) ? x - hi : 0.0f;
-}
-
 struct Args {
     int M, N, K;
-    float alpha, beta;
-    const float* C_in;
-    float* C_out;
-    int ldc;
+    float alpha;
+    int accumulate;
     int lower_only;
     int tiles_m, tiles_n, tiles;
     DevStatus* st;
@@ -100,36 +111,51 @@ __device__ __forceinline__ void tile_coords(int t, const Args& g, int& tm, int& 
     tn = 0;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    tgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Args g) {
+// The operand tensor maps: A_hi, B_hi, A_lo, B_lo (pre-split) or A, B.
+struct Maps {
+    CUtensorMap a, b, a_lo, b_lo, c;
+};
+
+template <bool PRESPLIT>
+__global__ void __launch_bounds__(Cfg<PRESPLIT>::THREADS, 1)
+    tgemm_kernel(const __grid_constant__ Maps maps, const Args g) {
+    using C = Cfg<PRESPLIT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* lo_base = smem + size_t(STAGES) * CHUNK_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(lo_base + size_t(LO_BUFS) * CHUNK_BYTES);  // [STAGES] TMA landed
-    uint64_t* conv = full + STAGES;          // [STAGES] one arrival per split warp: chunk split into hi / lo
-    uint64_t* empty = conv + STAGES;         // [STAGES] MMA commit: stage may be reloaded
-    uint64_t* lo_free = empty + STAGES;      // [LO_BUFS] MMA commit: lo buffer may be rewritten
-    uint64_t* tfull = lo_free + LO_BUFS;     // [2] MMA commit: accumulator complete
+    uint8_t* lo_base = smem + size_t(C::STAGES) * C::STAGE_BYTES;
+    uint8_t* cbuf = lo_base + size_t(C::LO_BUFS) * 2 * PART_BYTES;                 // [SLAB_BUFS][128 rows][128 B]
+    uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + size_t(SLAB_BUFS) * SLAB_BYTES);  // [STAGES] TMA landed
+    uint64_t* conv = full + C::STAGES;       // [STAGES] one arrival per split warp (in-kernel split)
+    uint64_t* empty = conv + C::STAGES;      // [STAGES] MMA commit: stage may be reloaded
+    uint64_t* lo_free = empty + C::STAGES;   // [2] MMA commit: lo buffer may be rewritten (in-kernel split)
+    uint64_t* tfull = lo_free + 2;           // [2] MMA commit: accumulator complete
     uint64_t* tempty = tfull + 2;            // [2] epilogue arrivals: accumulator drained
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    int* epi_abort = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nk = g.K / BKC;
     const int my_tiles = g.tiles > int(blockIdx.x) ? (g.tiles - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
 
     if (threadIdx.x == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
-        for (int s = 0; s < STAGES; ++s) {
+        tma_prefetch_desc(&maps.a);
+        tma_prefetch_desc(&maps.b);
+        tma_prefetch_desc(&maps.c);
+        if (PRESPLIT) {
+            tma_prefetch_desc(&maps.a_lo);
+            tma_prefetch_desc(&maps.b_lo);
+        }
+        for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&conv[s], CONV_WARPS);
+            mbar_init(&conv[s], C::CONV_WARPS > 0 ? C::CONV_WARPS : 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < LO_BUFS; ++b) mbar_init(&lo_free[b], 1);
         for (int b = 0; b < 2; ++b) {
+            mbar_init(&lo_free[b], 1);
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], EPI_WARPS);
         }
+        *epi_abort = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -141,7 +167,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == PRODUCER_WARP) {
+    if (warp == C::PRODUCER_WARP) {
         if (lane == 0) {
             int gc = 0;
             bool ok = true;
@@ -149,29 +175,34 @@ __global__ void __launch_bounds__(THREADS, 1)
                 int tm, tn;
                 tile_coords(int(blockIdx.x) + lt * int(gridDim.x), g, tm, tn);
                 for (int c = 0; c < nk; ++c, ++gc) {
-                    const int s = gc % STAGES;
-                    const uint32_t round = uint32_t(gc / STAGES);
+                    const int s = gc % C::STAGES;
+                    const uint32_t round = uint32_t(gc / C::STAGES);
                     if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, g.st, 301)) { ok = false; break; }
-                    uint8_t* base = smem + size_t(s) * CHUNK_BYTES;
-                    mbar_arrive_expect_tx(&full[s], CHUNK_BYTES);
-                    tma_load_2d(base, &tmA, c * BKC, tm * BM, &full[s]);             // A:   {32 k, 128 rows}
-                    tma_load_2d(base + A_BYTES, &tmB, c * BKC, tn * BN, &full[s]);   // B^T: {32 k, 128 rows}
+                    uint8_t* base = smem + size_t(s) * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                    tma_load_2d(base, &maps.a, c * BKC, tm * BM, &full[s]);                  // {32 k, 128 rows}
+                    tma_load_2d(base + PART_BYTES, &maps.b, c * BKC, tn * BN, &full[s]);
+                    if (PRESPLIT) {
+                        tma_load_2d(base + 2 * PART_BYTES, &maps.a_lo, c * BKC, tm * BM, &full[s]);
+                        tma_load_2d(base + 3 * PART_BYTES, &maps.b_lo, c * BKC, tn * BN, &full[s]);
+                    }
                 }
             }
         }
-    } else if (warp < CONV_WARPS) {
-        // ---------------- split chunks into hi (in place) / lo
+    } else if (warp < C::CONV_WARPS) {
+        // ---------------- in-kernel split: chunk -> hi (in place) / lo
         const int ct = threadIdx.x;   // 0 .. 32*CONV_WARPS-1
         const int total = my_tiles * nk;
         for (int gc = 0; gc < total; ++gc) {
-            const int s = gc % STAGES, l = gc % LO_BUFS;
-            const uint32_t round = uint32_t(gc / STAGES), lround = uint32_t(gc / LO_BUFS);
+            constexpr int LB = C::LO_BUFS > 0 ? C::LO_BUFS : 1;   // (this branch runs only when LO_BUFS > 0)
+            const int s = gc % C::STAGES, l = gc % LB;
+            const uint32_t round = uint32_t(gc / C::STAGES), lround = uint32_t(gc / LB);
             if (!mbar_wait(&full[s], round & 1u, g.st, 303)) break;
             if (!mbar_wait(&lo_free[l], (lround & 1u) ^ 1u, g.st, 306)) break;
-            float4* x = reinterpret_cast<float4*>(smem + size_t(s) * CHUNK_BYTES);
-            float4* lo = reinterpret_cast<float4*>(lo_base + size_t(l) * CHUNK_BYTES);
+            float4* x = reinterpret_cast<float4*>(smem + size_t(s) * C::STAGE_BYTES);
+            float4* lo = reinterpret_cast<float4*>(lo_base + size_t(l) * 2 * PART_BYTES);
 #pragma unroll 4
-            for (int i = ct; i < CHUNK_BYTES / 16; i += 32 * CONV_WARPS) {
+            for (int i = ct; i < 2 * PART_BYTES / 16; i += 32 * C::CONV_WARPS) {
                 float4 v = x[i], h, q;
                 split_tf32(v.x, h.x, q.x); split_tf32(v.y, h.y, q.y);
                 split_tf32(v.z, h.z, q.z); split_tf32(v.w, h.w, q.w);
@@ -181,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&conv[s]);
         }
-    } else if (warp == MMA_WARP) {
+    } else if (warp == C::MMA_WARP) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_tf32();
             int gc = 0;
@@ -193,12 +224,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc_fence_after();
                 const uint32_t dt = tmem_base + uint32_t(acc * BN);
                 for (int c = 0; c < nk; ++c, ++gc) {
-                    const int s = gc % STAGES, l = gc % LO_BUFS;
-                    const uint32_t round = uint32_t(gc / STAGES);
-                    if (!mbar_wait(&conv[s], round & 1u, g.st, 304)) { ok = false; break; }
+                    const int s = gc % C::STAGES;
+                    const int l = PRESPLIT ? 0 : gc % 2;
+                    const uint32_t round = uint32_t(gc / C::STAGES);
+                    if (!mbar_wait(PRESPLIT ? &full[s] : &conv[s], round & 1u, g.st, 304)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_hi = smem_u32(smem + size_t(s) * CHUNK_BYTES), b_hi = a_hi + A_BYTES;
-                    const uint32_t a_lo = smem_u32(lo_base + size_t(l) * CHUNK_BYTES), b_lo = a_lo + A_BYTES;
+                    const uint32_t a_hi = smem_u32(smem + size_t(s) * C::STAGE_BYTES), b_hi = a_hi + PART_BYTES;
+                    const uint32_t a_lo = PRESPLIT ? a_hi + 2 * PART_BYTES
+                                                   : smem_u32(lo_base + size_t(l) * 2 * PART_BYTES);
+                    const uint32_t b_lo = a_lo + PART_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BKC / 8; ++kk) {
                         // K-major: 8 k (32 bytes) per MMA inside the 128-byte swizzled
@@ -211,66 +245,62 @@ __global__ void __launch_bounds__(THREADS, 1)
                         umma_tf32(dt, dal, dbh, idesc, 1u);
                         umma_tf32(dt, dah, dbh, idesc, 1u);
                     }
-                    umma_commit(&empty[s]);      // stage may be reloaded once these MMAs finish
-                    umma_commit(&lo_free[l]);    // and its lo buffer rewritten
+                    umma_commit(&empty[s]);                  // stage may be reloaded once these MMAs finish
+                    if (!PRESPLIT) umma_commit(&lo_free[l]); // and its lo buffer rewritten
                 }
                 umma_commit(&tfull[acc]);        // tile complete (also on the error path)
             }
         }
-    } else {
-        // ---------------- epilogue warps: TMEM lanes (warp % 4) * 32 .. + 31 = tile rows,
-        // columns half * 64 .. + 63
-        const int quad = warp & 3;
-        const int half = (warp - EPI_WARP0) >> 2;
-        constexpr int HC = BN / 2;   // columns per epilogue thread
+    } else if (warp >= C::EPI_WARP0) {
+        // ---------------- epilogue: thread et owns tile row et (TMEM lane et)
+        const int quad = warp - C::EPI_WARP0;
+        const int et = threadIdx.x - 32 * C::EPI_WARP0;
+        volatile int* abort_flag = epi_abort;
+        int gs = 0;   // slabs issued so far (selects the staging buffer)
         for (int lt = 0; lt < my_tiles; ++lt) {
             const int acc = lt & 1;
             const uint32_t use = uint32_t(lt >> 1);
             int tm, tn;
             tile_coords(int(blockIdx.x) + lt * int(gridDim.x), g, tm, tn);
-            const int m = tm * BM + quad * 32 + lane;
-            const int n0 = tn * BN + half * HC;
-            const bool in_range = m < g.M;
-            const bool full_row = in_range && n0 + HC <= g.N;
-            // C_in for this tile now, so that the loads overlap the tile's MMAs
-            float4 ci[HC / 4];
-            if (full_row && g.beta != 0.0f) {
-                const float4* src = reinterpret_cast<const float4*>(g.C_in + size_t(m) * g.ldc + n0);
-#pragma unroll
-                for (int q = 0; q < HC / 4; ++q) ci[q] = src[q];
-            } else {
-#pragma unroll
-                for (int q = 0; q < HC / 4; ++q) ci[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            }
-            __syncwarp();
-            if (!mbar_wait(&tfull[acc], use & 1u, g.st, 305)) break;
+            if (!mbar_wait(&tfull[acc], use & 1u, g.st, 305)) *abort_flag = 1;
+            named_barrier_sync(EPI_BARRIER, 32 * EPI_WARPS);   // all four warps leave together on a timeout
+            if (*abort_flag) break;
             tc_fence_after();
-#pragma unroll
-            for (int cc = 0; cc < HC / 32; ++cc) {
-                const int n = n0 + cc * 32;
+#pragma unroll 1
+            for (int j = 0; j < BN / SLAB; ++j, ++gs) {
                 float v[32];
-                tmem_ld_32x32b_x32(tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + half * HC + cc * 32), v);
-                if (!in_range) continue;
-                float* cout = g.C_out + size_t(m) * g.ldc + n;
-                if (full_row) {
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + j * SLAB), v);
+                if (j == BN / SLAB - 1) {   // accumulator drained: the MMAs of tile lt + 2 may start
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[acc]);
+                }
+                uint8_t* buf = cbuf + size_t(gs & 1) * SLAB_BYTES;
+                if (et == 0) bulk_wait_group_read<1>();   // the store that last used this buffer has read it
+                named_barrier_sync(EPI_BARRIER, 32 * EPI_WARPS);
+                // row et, 16-byte chunk q at position q ^ (et % 8): TMA's 128-byte swizzle,
+                // and eight consecutive rows cover all 32 banks
+                uint8_t* row = buf + size_t(et) * (SLAB * 4);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 c4 = ci[cc * 8 + q];
-                        *reinterpret_cast<float4*>(cout + 4 * q) =
-                            make_float4(fmaf(g.alpha, v[4 * q], g.beta * c4.x), fmaf(g.alpha, v[4 * q + 1], g.beta * c4.y),
-                                        fmaf(g.alpha, v[4 * q + 2], g.beta * c4.z), fmaf(g.alpha, v[4 * q + 3], g.beta * c4.w));
+                for (int q = 0; q < SLAB / 4; ++q)
+                    *reinterpret_cast<float4*>(row + ((q ^ (et & 7)) << 4)) =
+                        make_float4(g.alpha * v[4 * q], g.alpha * v[4 * q + 1], g.alpha * v[4 * q + 2],
+                                    g.alpha * v[4 * q + 3]);
+                fence_proxy_async_smem();
+                named_barrier_sync(EPI_BARRIER, 32 * EPI_WARPS);
+                if (et == 0) {
+                    const int x = tn * BN + j * SLAB;
+                    if (x < g.N) {
+                        if (g.accumulate)
+                            tma_reduce_add_2d(&maps.c, buf, x, tm * BM);
+                        else
+                            tma_store_2d(&maps.c, buf, x, tm * BM);
                     }
-                } else {
-                    const float* cin = g.C_in + size_t(m) * g.ldc + n;
-#pragma unroll
-                    for (int q = 0; q < 32; ++q)
-                        if (n + q < g.N) cout[q] = fmaf(g.alpha, v[q], g.beta != 0.0f ? g.beta * cin[q] : 0.0f);
+                    bulk_commit_group();
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
         }
+        if (et == 0) bulk_wait_group<0>();   // every store has reached global memory
     }
     tc_fence_before();
     __syncthreads();
@@ -281,7 +311,27 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 namespace {
 PFN_encodeTiled g_enc = nullptr;
+
+template <bool PRESPLIT>
+int launch_variant(const tg::Maps& maps, const tg::Args& g, cudaStream_t stream) {
+    using C = tg::Cfg<PRESPLIT>;
+    static bool attr_set[64] = {};
+    static int sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(tg::tgemm_kernel<PRESPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(C::SMEM_BYTES)) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    const int grid = std::max(1, std::min(g.tiles, dev < 64 && sms[dev] > 0 ? sms[dev] : 148));
+    tg::tgemm_kernel<PRESPLIT><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(maps, g);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
+}  // namespace
 
 void set_tensor_map_encoder(PFN_encodeTiled f) { g_enc = f; }
 
@@ -299,19 +349,25 @@ int make_map_2d_f32(CUtensorMap* tm, const float* base, uint64_t inner, uint64_t
     return r == CUDA_SUCCESS ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
-int launch_tgemm(int M, int N, int K, float alpha, const float* A, int lda, const float* B, int ldb, bool trans_b,
-                 float beta, const float* C_in, float* C_out, int ldc, bool lower_only, cudaStream_t stream,
-                 DevStatus* st) {
+int launch_tgemm(int M, int N, int K, float alpha, const float* A, const float* A_lo, int lda, const float* Bt,
+                 const float* Bt_lo, int ldb, bool accumulate, float* C, int ldc, bool lower_only,
+                 cudaStream_t stream, DevStatus* st) {
     using namespace tg;
     if (M <= 0 || N <= 0) return GPTQ_OK;
-    if (!trans_b || K <= 0 || K % BKC != 0 || K > MAX_K || g_enc == nullptr) return GPTQ_ERR_UNSUPPORTED;
-    CUtensorMap ta, tb;
-    int rc = make_map_2d_f32(&ta, A, uint64_t(K), uint64_t(M), uint64_t(lda), BKC, BM, true);
-    if (rc) return rc;
-    rc = make_map_2d_f32(&tb, B, uint64_t(K), uint64_t(N), uint64_t(ldb), BKC, BN, true);
+    const bool presplit = A_lo != nullptr;
+    if (K <= 0 || K % BKC != 0 || K > MAX_K || (Bt_lo != nullptr) != presplit || g_enc == nullptr)
+        return GPTQ_ERR_UNSUPPORTED;
+    Maps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    int rc = make_map_2d_f32(&maps.a, A, uint64_t(K), uint64_t(M), uint64_t(lda), BKC, BM, true);
+    if (!rc) rc = make_map_2d_f32(&maps.b, Bt, uint64_t(K), uint64_t(N), uint64_t(ldb), BKC, BN, true);
+    if (!rc && presplit) rc = make_map_2d_f32(&maps.a_lo, A_lo, uint64_t(K), uint64_t(M), uint64_t(lda), BKC, BM, true);
+    if (!rc && presplit) rc = make_map_2d_f32(&maps.b_lo, Bt_lo, uint64_t(K), uint64_t(N), uint64_t(ldb), BKC, BN, true);
+    if (!rc) rc = make_map_2d_f32(&maps.c, C, uint64_t(N), uint64_t(M), uint64_t(ldc), SLAB, BM, true);
     if (rc) return rc;
     Args g{};
-    g.M = M; g.N = N; g.K = K; g.alpha = alpha; g.beta = beta; g.C_in = C_in; g.C_out = C_out; g.ldc = ldc;
+    g.M = M; g.N = N; g.K = K; g.alpha = alpha;
+    g.accumulate = accumulate ? 1 : 0;
     g.lower_only = lower_only ? 1 : 0;
     g.tiles_m = (M + BM - 1) / BM;
     g.tiles_n = (N + BN - 1) / BN;
@@ -322,21 +378,7 @@ int launch_tgemm(int M, int N, int K, float alpha, const float* A, int lda, cons
         g.tiles = g.tiles_m * g.tiles_n;
     }
     g.st = st;
-    static bool attr_set[64] = {};
-    static int sms[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(tgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES)) !=
-                cudaSuccess ||
-            cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return GPTQ_ERR_CUDA;
-        attr_set[dev] = true;
-    }
-    const int grid = std::max(1, std::min(g.tiles, dev < 64 && sms[dev] > 0 ? sms[dev] : 148));
-    tgemm_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, g);
-    count_launch();
-    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+    return presplit ? launch_variant<true>(maps, g, stream) : launch_variant<false>(maps, g, stream);
 }
 
 }  // namespace gptq

@@ -87,7 +87,7 @@ def test_noalloc_matches_workspace_entry_point(lib, d_out, d_in, bits, groupsize
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
-    """4096 x 4096 needs 64 MiB of U^T: over the 40 MiB array, refused before launching."""
+    """4096 x 4096 needs 128 MiB for the split U^T: over the 40 MiB array, refused before launching."""
     d = 4096
     W = torch.zeros((8, d), dtype=torch.float32, device="cuda")
     U = torch.zeros((d, d), dtype=torch.float32, device="cuda")
