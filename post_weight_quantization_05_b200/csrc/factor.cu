@@ -13,11 +13,11 @@
 //
 // All arithmetic is fp32.  Blocked right-looking, block nb = 128:
 //   per diagonal block: one CTA factors it in shared memory and inverts the
-//   factor (potrf_diag_kernel); the panel below is solved against it with an
-//   SGEMM by the inverse; the trailing lower triangle gets a SYRK-shaped
-//   SGEMM.  The inverse L'^-1 is then built block row by block row
-//   (right-looking forward substitution on the identity), and U is written
-//   by reversing both indices.
+//   factor (potrf_diag_kernel); the panel below is solved against it with a
+//   GEMM by the inverse; the trailing lower triangle gets a SYRK-shaped GEMM
+//   (both on the tensor cores, tgemm).  Z = L'^-T is built block column by
+//   block column alongside (right-looking forward substitution on the
+//   identity, transposed), and U is written by reversing both indices.
 #include <mutex>
 
 #include "common.cuh"
@@ -27,10 +27,6 @@ namespace gptq {
 namespace factor {
 
 constexpr int NB = 128;
-constexpr int LD = NB + 1;   // padded shared-memory row (column accesses conflict-free)
-constexpr int LDY = NB + 4;  // inverse rows: 16-byte aligned for vector access
-constexpr int DIAG_THREADS = 256;
-constexpr size_t DIAG_SMEM = size_t(NB) * (LD + LDY) * sizeof(float);
 
 struct Layout {
     size_t a_off, y_off, dinv_off, scal_off, total;
@@ -83,263 +79,283 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const fl
 }
 
 // ---------------------------------------------------------------------------
-// One 128 x 128 diagonal block: L L^T = A_kk (in place, lower) and L^-1.
-// The block is cut into 4 x 4 sub-blocks of 32.  For each sub-block column:
-// one warp factors the 32 x 32 diagonal sub-block in registers (lane = row,
-// column broadcasts by shuffles) and inverts it; all 8 warps then solve the
-// sub-blocks below against it and update the trailing sub-blocks.  Finally
-// the off-diagonal sub-blocks of L^-1 are formed from the diagonal ones.
+// One 128 x 128 diagonal block: L L^T = A_kk and L^-1, in one CTA of 12 warps.
+// The block is cut into 4 x 4 sub-blocks of 32.  Step kb (o = 32 kb):
+//   A: warp 0 factors the diagonal sub-block (kb, kb) in registers; the other
+//      warps meanwhile apply step kb-1 of the inverse's trailing update;
+//   B: warp 0 inverts the diagonal sub-block; warps 1-3 solve the sub-blocks
+//      below against it (one row per thread);
+//   C: the trailing update of the factorization (sub-blocks (bi, bj),
+//      kb < bj <= bi) and step kb of the inverse's block solve.
+// The inverse Y = L^-1 is built right-looking on the identity (Y = X after
+//   X_k <- L_kk^-1 X_k;  X_i -= L_ik X_k  (i > k)  for k = 0..3)
+// and kept transposed (Yt = Y^T = L^-T) so that every product reads both of
+// its operands along rows, four at a time.  Row strides of 132 floats make
+// those float4 reads and the scattered scalar writes free of bank conflicts.
 // ---------------------------------------------------------------------------
 constexpr int SB = 32;
-constexpr unsigned FULL = 0xffffffffu;
+constexpr int LDS = NB + 4;              // S and Yt row stride (floats)
+constexpr int LDI = SB + 4;              // Lr row stride
+constexpr int DIAG_THREADS = 384;           // 12 warps: the most any phase below uses
+constexpr size_t DIAG_SMEM = (size_t(2) * NB * LDS + size_t(SB) * LDI + 2 * SB + NB) * sizeof(float);
 
-// The 32 x 32 pieces are written as template recursions so that every
-// register index is a compile-time constant (a rolled or partly unrolled loop
-// would put the row in local memory).
+// The 32 x 32 pieces are template recursions so that every register index is
+// a compile-time constant (a rolled loop would put the row in local memory).
 
-// One row a[] (32 values) solved against L (32 x 32 lower, in shared memory
-// with row stride LD):  a <- a L^-T  (right-looking, invd[c] = 1/L[c][c]).
+// Right-looking Cholesky of a 32 x 32 block by one warp, lane = row: a[] holds
+// row `lane` (entries j > lane are don't-care).  Step C reads column C of the
+// current matrix from cb[C & 1] (each lane published its own entry), and every
+// lane applies  a[j] -= a[lane][C] a[j][C] / a[C][C]  with the unscaled column,
+// so the only serial work per step is one rsqrt; a[C] is then scaled to
+// L[lane][C] and entry C+1 is published for the next step.
+template <int C>
+struct RowChol32 {
+    __device__ __forceinline__ static void run(float (&a)[SB], int lane, float* __restrict__ cb,
+                                               float* __restrict__ invd, uint32_t& bad, uint32_t& nonfinite) {
+        const float* cin = cb + (C & 1) * SB;
+        const float piv = cin[C];
+        bad |= uint32_t(!(piv > 0.0f && isfinite(piv))) << C;   // bit C: pivot C failed
+        nonfinite |= uint32_t(!isfinite(piv)) << C;
+        const float inv = rsqrtf(piv);
+        const float lm = a[C] * (inv * inv);
+#pragma unroll
+        for (int j4 = ((C + 1) / 4) * 4; j4 < SB; j4 += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(cin + j4);
+            if (j4 + 0 > C) a[j4 + 0] = fmaf(-lm, v.x, a[j4 + 0]);
+            if (j4 + 1 > C) a[j4 + 1] = fmaf(-lm, v.y, a[j4 + 1]);
+            if (j4 + 2 > C) a[j4 + 2] = fmaf(-lm, v.z, a[j4 + 2]);
+            if (j4 + 3 > C) a[j4 + 3] = fmaf(-lm, v.w, a[j4 + 3]);
+        }
+        a[C] *= inv;
+        invd[C] = inv;
+        if constexpr (C + 1 < SB) {
+            cb[((C + 1) & 1) * SB + lane] = a[C + 1];
+            __syncwarp();
+            RowChol32<C + 1>::run(a, lane, cb, invd, bad, nonfinite);
+        }
+    }
+};
+
+// One row x[] (32 values) solved against L (32 x 32 lower, shared memory,
+// row stride LDS):  x <- x L^-T  (right-looking, invd[c] = 1/L[c][c]).
 template <int C>
 struct Trsm32 {
-    __device__ __forceinline__ static void run(float (&a)[SB], const float* __restrict__ L,
+    __device__ __forceinline__ static void run(float (&x)[SB], const float* __restrict__ L,
                                                const float* __restrict__ invd) {
-        const float xc = a[C] * invd[C];
-        a[C] = xc;
+        const float xc = x[C] * invd[C];
+        x[C] = xc;
 #pragma unroll
-        for (int j = C + 1; j < SB; ++j) a[j] = fmaf(-xc, L[j * LD + C], a[j]);
-        if constexpr (C + 1 < SB) Trsm32<C + 1>::run(a, L, invd);
+        for (int j = C + 1; j < SB; ++j) x[j] = fmaf(-xc, L[j * LDS + C], x[j]);
+        if constexpr (C + 1 < SB) Trsm32<C + 1>::run(x, L, invd);
     }
 };
 
-// Column-oriented Cholesky of a 32 x 32 block by one warp: lane j holds
-// column j (col[r] = A[r][j]; entries above the diagonal are ignored).  At
-// step C lane C finalizes its column and publishes it through `buf` (shared
-// memory); every later lane then updates its own column with one broadcast
-// read per row -- no shuffles, one short dependency chain per column.
-template <int C>
-struct ColChol32 {
-    __device__ __forceinline__ static void run(float (&col)[SB], int lane, float* __restrict__ buf, int& bad,
-                                               float& badpiv) {
-        if (lane == C) {
-            const float piv = col[C];
-            if (bad < 0 && (!(piv > 0.0f) || !isfinite(piv))) { bad = C; badpiv = piv; }
-            const float inv = rsqrtf(piv);
-            col[C] = piv * inv;
-#pragma unroll
-            for (int r = C + 1; r < SB; ++r) col[r] *= inv;
-#pragma unroll
-            for (int r = (C / 4) * 4; r < SB; r += 4)      // whole 16-byte groups; entries < C unused
-                *reinterpret_cast<float4*>(buf + r) = make_float4(col[r], col[r + 1], col[r + 2], col[r + 3]);
-        }
-        __syncwarp();
-        if (lane > C) {
-            const float ljc = buf[lane];                  // L[lane][C]
-#pragma unroll
-            for (int r4 = ((C + 1) / 4) * 4; r4 < SB; r4 += 4) {
-                const float4 b = *reinterpret_cast<const float4*>(buf + r4);
-                if (r4 + 0 > C) col[r4 + 0] = fmaf(-b.x, ljc, col[r4 + 0]);
-                if (r4 + 1 > C) col[r4 + 1] = fmaf(-b.y, ljc, col[r4 + 1]);
-                if (r4 + 2 > C) col[r4 + 2] = fmaf(-b.z, ljc, col[r4 + 2]);
-                if (r4 + 3 > C) col[r4 + 3] = fmaf(-b.w, ljc, col[r4 + 3]);
-            }
-        }
-        __syncwarp();
-        if constexpr (C + 1 < SB) ColChol32<C + 1>::run(col, lane, buf, bad, badpiv);
-    }
-};
-
-// Column-oriented inverse of a 32 x 32 lower-triangular L held in shared
-// memory (row stride LD, 1/L[i][i] in invd): lane j computes column j of
-// L^-1 (y[i] for i >= j) by forward substitution, reading L by broadcast.
+// Column `lane` of L^-1 for a 32 x 32 lower L (shared memory, row stride LDS)
+// by forward substitution on e_lane; reads of L are broadcasts.
 template <int I>
 struct ColInv32 {
     __device__ __forceinline__ static void run(float (&y)[SB], const float* __restrict__ L,
-                                               const float* __restrict__ invd, int lane) {
+                                               const float* __restrict__ invd) {
         const float yi = y[I] * invd[I];
         y[I] = yi;
 #pragma unroll
-        for (int r = I + 1; r < SB; ++r) y[r] = fmaf(-L[r * LD + I], yi, y[r]);
-        if constexpr (I + 1 < SB) ColInv32<I + 1>::run(y, L, invd, lane);
+        for (int r = I + 1; r < SB; ++r) y[r] = fmaf(-L[r * LDS + I], yi, y[r]);
+        if constexpr (I + 1 < SB) ColInv32<I + 1>::run(y, L, invd);
     }
 };
 
-// Factor the diagonal block A[k0:k0+NB, k0:k0+NB] = L L^T in place (lower) and
-// write its inverse L^-1 to Dinv (NB x NB, row-major).  A non-positive or
-// non-finite pivot sets *info = k0 + c + 1 (first failure only).
-__global__ void __launch_bounds__(DIAG_THREADS)
-    potrf_diag_kernel(float* __restrict__ A, int d, int k0, float* __restrict__ Dinv, int* info, DevStatus* st) {
-    extern __shared__ float sm[];
-    float* S = sm;             // [NB][LD] factor (upper part used as scratch)
-    float* Y = sm + NB * LD;   // [NB][LDY] inverse (NB * LD is a multiple of 4: 16-byte aligned)
-    __shared__ float invd[NB];
-    __shared__ __align__(16) float colbuf[SB];
+// Out[R_a][C_b] -= sum_m P[R_a][m] Q[C_b][m] over one 32-wide sub-block of m,
+// for the 4 x 4 outputs of lane (g, h) = (lane / 4, lane % 4) in one half
+// (columns 16 s .. 16 s + 15) of a 32 x 32 output sub-block:
+// R_a = r0 + g + 8a, C_b = c0 + 16 s + h + 4b.  P, Q and Out have row stride
+// LDS and P, Q point at the first m column.
+__device__ __forceinline__ void sub_block_update(const float* __restrict__ P, const float* __restrict__ Q,
+                                                 float* __restrict__ Out, int r0, int c0, int s, int lane) {
+    const int g = lane >> 2, h = lane & 3;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+#pragma unroll 1
+    for (int m = 0; m < SB; m += 4) {
+        float4 p[4], q[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) p[a] = *reinterpret_cast<const float4*>(P + (r0 + g + 8 * a) * LDS + m);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) q[b] = *reinterpret_cast<const float4*>(Q + (c0 + 16 * s + h + 4 * b) * LDS + m);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                acc[a][b] = fmaf(p[a].x, q[b].x, acc[a][b]);
+                acc[a][b] = fmaf(p[a].y, q[b].y, acc[a][b]);
+                acc[a][b] = fmaf(p[a].z, q[b].z, acc[a][b]);
+                acc[a][b] = fmaf(p[a].w, q[b].w, acc[a][b]);
+            }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) Out[(r0 + g + 8 * a) * LDS + c0 + 16 * s + h + 4 * b] -= acc[a][b];
+}
+
+// Factor the diagonal block A[k0:k0+NB, k0:k0+NB] = L L^T and write
+//   Dinv = L^-1 (NB x NB row-major, zeros above the diagonal) and
+//   Z[k0 + c][k0 + r] = L^-1[r][c]  (the diagonal block of Z = L'^-T).
+// A's block itself is left as it was (nothing reads L_kk afterwards).  A
+// non-positive or non-finite pivot sets *info = k0 + c + 1 (first failure only).
+__global__ void __launch_bounds__(DIAG_THREADS, 1)
+    potrf_diag_kernel(const float* __restrict__ A, int d, int k0, float* __restrict__ Dinv, float* __restrict__ Z,
+                      int* info, DevStatus* st) {
+    extern __shared__ __align__(16) float sm[];
+    float* S = sm;                     // [NB][LDS] the block, factored in place (lower)
+    float* Yt = S + NB * LDS;          // [NB][LDS] X, then Y, transposed (upper)
+    float* Lr = Yt + NB * LDS;         // [SB][LDI] L_kk^-1 of the current step, row-major
+    float* cb = Lr + SB * LDI;         // [2][SB] published column (Cholesky steps)
+    float* invd = cb + 2 * SB;         // [NB] 1 / L[c][c]
     __shared__ int failed;
     if (*info != 0) return;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-#pragma unroll 4
-    for (int idx = 4 * t; idx < NB * NB; idx += 4 * DIAG_THREADS) {
-        const int r = idx / NB, c = idx % NB;
-        const float4 v = *reinterpret_cast<const float4*>(A + size_t(k0 + r) * d + k0 + c);
-        S[r * LD + c] = (c <= r) ? v.x : 0.0f;
-        S[r * LD + c + 1] = (c + 1 <= r) ? v.y : 0.0f;
-        S[r * LD + c + 2] = (c + 2 <= r) ? v.z : 0.0f;
-        S[r * LD + c + 3] = (c + 3 <= r) ? v.w : 0.0f;
+
+    // lower triangle of the block (zeros above), Yt = 0
+    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
+        const int r = idx / (NB / 4), c = (idx % (NB / 4)) * 4;
+        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (c <= r) {
+            v = *reinterpret_cast<const float4*>(A + size_t(k0 + r) * d + k0 + c);
+            if (c + 1 > r) v.y = 0.0f;
+            if (c + 2 > r) v.z = 0.0f;
+            if (c + 3 > r) v.w = 0.0f;
+        }
+        *reinterpret_cast<float4*>(S + r * LDS + c) = v;
+        *reinterpret_cast<float4*>(Yt + r * LDS + c) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
-    for (int idx = t; idx < NB * LDY; idx += DIAG_THREADS) Y[idx] = 0.0f;
     if (t == 0) failed = 0;
     __syncthreads();
 
     for (int kb = 0; kb < NB / SB; ++kb) {
         const int o = kb * SB;
+        // ---- A: factor the diagonal sub-block (warp 0) || inverse update of step kb-1
         if (warp == 0) {
-            float col[SB];
+            float a[SB];
 #pragma unroll
-            for (int r = 0; r < SB; ++r) col[r] = (r >= lane) ? S[(o + r) * LD + o + lane] : 0.0f;
-            int bad = -1;
-            float badpiv = 0.0f;
-            ColChol32<0>::run(col, lane, colbuf, bad, badpiv);
-#pragma unroll
-            for (int r = 0; r < SB; ++r)
-                if (r >= lane) S[(o + r) * LD + o + lane] = col[r];
+            for (int j = 0; j < SB; j += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(S + (o + lane) * LDS + o + j);
+                a[j] = v.x; a[j + 1] = v.y; a[j + 2] = v.z; a[j + 3] = v.w;
+            }
+            cb[lane] = a[0];
             __syncwarp();
-            invd[o + lane] = 1.0f / S[(o + lane) * LD + o + lane];
-            bad = __reduce_min_sync(FULL, bad < 0 ? SB : bad);
-            const float p = __shfl_sync(FULL, badpiv, bad < SB ? bad : 0);   // the failing pivot's value
-            if (bad < SB && lane == 0) {
+            uint32_t badmask = 0, nonfinite = 0;   // the same in every lane
+            RowChol32<0>::run(a, lane, cb, invd + o, badmask, nonfinite);
+#pragma unroll
+            for (int j = 0; j < SB; j += 4)
+                *reinterpret_cast<float4*>(S + (o + lane) * LDS + o + j) =
+                    make_float4(j <= lane ? a[j] : 0.0f, j + 1 <= lane ? a[j + 1] : 0.0f,
+                                j + 2 <= lane ? a[j + 2] : 0.0f, j + 3 <= lane ? a[j + 3] : 0.0f);
+            if (badmask != 0 && lane == 0) {   // the first failing pivot of this sub-block
+                const int bad = __ffs(int(badmask)) - 1;
                 failed = 1;
                 if (atomicCAS(info, 0, k0 + o + bad + 1) == 0)
-                    record_error(st, isfinite(p) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE, k0 + o + bad + 1);
+                    record_error(st, (nonfinite >> bad) & 1u ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_PD, k0 + o + bad + 1);
+            }
+        } else if (kb > 0) {
+            // X_ij -= L_{i,kb-1} Y_{kb-1,j} for i >= kb, j < kb, transposed:
+            // Yt[j-block][i-block] -= Yt[j-block][(kb-1)-block] S[i-block][(kb-1)-block]^T
+            const int w = warp - 1;                  // 0..14
+            const int nj = kb, ni = NB / SB - kb;    // sub-blocks j < kb, i >= kb
+            if (w < 2 * ni * nj) {
+                const int blk = w >> 1, s = w & 1;
+                const int j = blk % nj, i = kb + blk / nj;
+                sub_block_update(Yt + (kb - 1) * SB, S + (kb - 1) * SB, Yt, j * SB, i * SB, s, lane);
             }
         }
         __syncthreads();
         if (failed) return;
+
+        // ---- B: invert the diagonal sub-block (warp 0) || solve the rows below (warps 1-3)
         const int below = NB - o - SB;
-        if (below == 0) break;
-        // solve the rows below against this sub-block: S[r][o..o+32) <- S[r][o..o+32) L_kk^-T
-        if (t < below) {
-            const int r = o + SB + t;
-            float a[SB];
+        if (warp == 0) {
+            float y[SB];
 #pragma unroll
-            for (int k = 0; k < SB; ++k) a[k] = S[r * LD + o + k];
-            Trsm32<0>::run(a, S + o * LD + o, invd + o);
+            for (int r = 0; r < SB; ++r) y[r] = (r == lane) ? 1.0f : 0.0f;
+            ColInv32<0>::run(y, S + o * LDS + o, invd + o);
+            // Yt rows o + lane (= column lane of L_kk^-1) and Lr (row-major copy)
 #pragma unroll
-            for (int k = 0; k < SB; ++k) S[r * LD + o + k] = a[k];
+            for (int r = 0; r < SB; r += 4)
+                *reinterpret_cast<float4*>(Yt + (o + lane) * LDS + o + r) = make_float4(y[r], y[r + 1], y[r + 2], y[r + 3]);
+#pragma unroll
+            for (int r = 0; r < SB; ++r) Lr[r * LDI + lane] = y[r];
+        } else if (t - 32 < below) {
+            const int r = o + SB + (t - 32);
+            float x[SB];
+#pragma unroll
+            for (int k = 0; k < SB; k += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(S + r * LDS + o + k);
+                x[k] = v.x; x[k + 1] = v.y; x[k + 2] = v.z; x[k + 3] = v.w;
+            }
+            Trsm32<0>::run(x, S + o * LDS + o, invd + o);
+#pragma unroll
+            for (int k = 0; k < SB; k += 4)
+                *reinterpret_cast<float4*>(S + r * LDS + o + k) = make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
         }
         __syncthreads();
-        // trailing update of the sub-blocks (bi, bj), kb < bj <= bi
+
+        // ---- C: trailing update of the factorization || inverse solve of step kb
         {
-            const int i = t >> 3, j4 = (t & 7) * 4;
-            for (int bi = kb + 1; bi < NB / SB; ++bi) {
-                for (int bj = kb + 1; bj <= bi; ++bj) {
-                    const int r = bi * SB + i;
-                    float acc[4];
+            const int nrest = NB / SB - kb - 1;            // sub-block rows / columns after kb
+            const int pair_warps = nrest * (nrest + 1);    // two warps per lower sub-block pair
+            if (warp < pair_warps) {
+                // pair p = warp / 2 over (bi, bj), kb < bj <= bi, row-major
+                int p = warp >> 1, bi = kb + 1, bj = kb + 1;
+                while (p > bi - (kb + 1)) { p -= bi - kb; ++bi; }
+                bj = kb + 1 + p;
+                sub_block_update(S + o, S + o, S, bi * SB, bj * SB, warp & 1, lane);
+            } else if (warp < pair_warps + kb) {
+                // Y_{kb,j} = L_kk^-1 X_{kb,j} for j < kb: thread = column c of block j,
+                // reading X_{kb,j}[., c] as row (j*SB + c) of Yt
+                const int u = t - 32 * pair_warps;             // 0 .. 32 kb - 1
+                float* row = Yt + (size_t(u)) * LDS + o;       // j = u / SB, c = u % SB: row j*SB + c = u
+                float x[SB];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[q] = S[r * LD + bj * SB + j4 + q];
-#pragma unroll 8
-                    for (int k = 0; k < SB; ++k) {
-                        const float av = S[r * LD + o + k];
+                for (int m = 0; m < SB; m += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(row + m);
+                    x[m] = v.x; x[m + 1] = v.y; x[m + 2] = v.z; x[m + 3] = v.w;
+                }
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) acc[q] = fmaf(-av, S[(bj * SB + j4 + q) * LD + o + k], acc[q]);
+                for (int r = 0; r < SB; r += 4) {
+                    float y4[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int m = 0; m < SB; m += 4) {
+                            if (m <= r + q) {
+                                const float4 l = *reinterpret_cast<const float4*>(Lr + (r + q) * LDI + m);
+                                acc = fmaf(l.x, x[m], acc);
+                                acc = fmaf(l.y, x[m + 1], acc);
+                                acc = fmaf(l.z, x[m + 2], acc);
+                                acc = fmaf(l.w, x[m + 3], acc);
+                            }
+                        }
+                        y4[q] = acc;
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) S[r * LD + bj * SB + j4 + q] = acc[q];
+                    *reinterpret_cast<float4*>(row + r) = make_float4(y4[0], y4[1], y4[2], y4[3]);
                 }
             }
         }
         __syncthreads();
     }
 
-    // inverse: the four diagonal sub-blocks in parallel (warps 0..3), one
-    // column of L^-1 per lane ...
-    if (warp < NB / SB) {
-        const int o = warp * SB;
-        float y[SB];
-#pragma unroll
-        for (int r = 0; r < SB; ++r) y[r] = (r == lane) ? 1.0f : 0.0f;
-        ColInv32<0>::run(y, S + o * LD + o, invd + o, lane);
-#pragma unroll
-        for (int r = 0; r < SB; ++r) Y[(o + r) * LDY + o + lane] = (r >= lane) ? y[r] : 0.0f;
+    // Z's diagonal block = Yt (rows), and Dinv = Yt^T
+    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
+        const int c = idx / (NB / 4), r = (idx % (NB / 4)) * 4;
+        *reinterpret_cast<float4*>(Z + size_t(k0 + c) * d + k0 + r) = *reinterpret_cast<const float4*>(Yt + c * LDS + r);
     }
-    __syncthreads();
-
-    // ... then the off-diagonal ones:  Y[bi][bj] = -Y[bi][bi] * sum_{k=bj}^{bi-1} L[bi][k] Y[k][bj]
-    // T[bj] is kept in the (unused) strictly upper sub-blocks (0, 1 + bj) of S.
-    {
-        const int i = t >> 3, j4 = (t & 7) * 4;
-        for (int bi = 1; bi < NB / SB; ++bi) {
-            // one pass over k serves every bj (independent accumulators)
-            float4 acc[NB / SB - 1];
-#pragma unroll
-            for (int bj = 0; bj < NB / SB - 1; ++bj) acc[bj] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            const float* lrow = S + (bi * SB + i) * LD;
-#pragma unroll 4
-            for (int k = 0; k < bi * SB; ++k) {
-                const float l = lrow[k];
-#pragma unroll
-                for (int bj = 0; bj < NB / SB - 1; ++bj) {
-                    if (bj < bi && k >= bj * SB) {
-                        const float4 y = *reinterpret_cast<const float4*>(Y + k * LDY + bj * SB + j4);
-                        acc[bj].x = fmaf(l, y.x, acc[bj].x); acc[bj].y = fmaf(l, y.y, acc[bj].y);
-                        acc[bj].z = fmaf(l, y.z, acc[bj].z); acc[bj].w = fmaf(l, y.w, acc[bj].w);
-                    }
-                }
-            }
-#pragma unroll
-            for (int bj = 0; bj < NB / SB - 1; ++bj) {
-                if (bj < bi) {
-                    float* trow = S + i * LD + (1 + bj) * SB + j4;
-                    trow[0] = acc[bj].x; trow[1] = acc[bj].y; trow[2] = acc[bj].z; trow[3] = acc[bj].w;
-                }
-            }
-            __syncthreads();
-            for (int bj = 0; bj < bi; ++bj) {
-                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                const float* yrow = Y + (bi * SB + i) * LDY + bi * SB;
-                for (int k = 0; k <= i; ++k) {
-                    const float y = yrow[k];
-                    const float* trow = S + k * LD + (1 + bj) * SB + j4;
-                    acc.x = fmaf(y, trow[0], acc.x); acc.y = fmaf(y, trow[1], acc.y);
-                    acc.z = fmaf(y, trow[2], acc.z); acc.w = fmaf(y, trow[3], acc.w);
-                }
-                *reinterpret_cast<float4*>(Y + (bi * SB + i) * LDY + bj * SB + j4) =
-                    make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-            }
-            __syncthreads();
-        }
-    }
-
-#pragma unroll 4
-    for (int idx = 4 * t; idx < NB * NB; idx += 4 * DIAG_THREADS) {
-        const int r = idx / NB, c = idx % NB;
-        float* arow = A + size_t(k0 + r) * d + k0 + c;
-        if (c + 3 <= r) {
-            *reinterpret_cast<float4*>(arow) =
-                make_float4(S[r * LD + c], S[r * LD + c + 1], S[r * LD + c + 2], S[r * LD + c + 3]);
-        } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (c + q <= r) arow[q] = S[r * LD + c + q];
-        }
-        const float4 yv = *reinterpret_cast<const float4*>(Y + r * LDY + c);
-        *reinterpret_cast<float4*>(Dinv + idx) =
-            make_float4((c <= r) ? yv.x : 0.0f, (c + 1 <= r) ? yv.y : 0.0f, (c + 2 <= r) ? yv.z : 0.0f,
-                        (c + 3 <= r) ? yv.w : 0.0f);
-    }
-}
-
-// Z[k*NB + c][k*NB + r] = Dinv_k[r][c]: diagonal block k of Z = L^-T,
-// transposed through shared memory (coalesced on both sides).
-__global__ void place_diag_inverse_t_kernel(const float* __restrict__ Dinv_k, int d, int k, float* __restrict__ Z) {
-    extern __shared__ float tile[];   // [NB][LD]
-    for (int idx = 4 * threadIdx.x; idx < NB * NB; idx += 4 * blockDim.x) {
-        const int r = idx / NB, c = idx % NB;
-        const float4 v = *reinterpret_cast<const float4*>(Dinv_k + idx);
-        tile[r * LD + c] = v.x; tile[r * LD + c + 1] = v.y; tile[r * LD + c + 2] = v.z; tile[r * LD + c + 3] = v.w;
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
-        const int c = idx / NB, r = idx % NB;
-        Z[size_t(k * NB + c) * d + k * NB + r] = tile[r * LD + c];
+    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
+        const int r = idx % NB, c = (idx / NB) * 4;
+        *reinterpret_cast<float4*>(Dinv + r * NB + c) =
+            make_float4(Yt[c * LDS + r], Yt[(c + 1) * LDS + r], Yt[(c + 2) * LDS + r], Yt[(c + 3) * LDS + r]);
     }
 }
 
@@ -353,7 +369,7 @@ struct AuxStream {
     cudaStream_t main = nullptr;    // the factorization's critical chain (highest priority)
     cudaStream_t s = nullptr;       // inverse steps
     cudaStream_t side = nullptr;    // trailing updates beyond the next block column
-    cudaEvent_t fork = nullptr, step = nullptr, rest = nullptr, join = nullptr, join_side = nullptr;
+    cudaEvent_t fork = nullptr, step = nullptr, rest = nullptr, join = nullptr, join_side = nullptr, filled = nullptr;
 };
 
 static int aux_stream(AuxStream** out) {
@@ -373,7 +389,8 @@ static int aux_stream(AuxStream** out) {
             cudaEventCreateWithFlags(&a.step, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.rest, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&a.join_side, cudaEventDisableTiming) != cudaSuccess)
+            cudaEventCreateWithFlags(&a.join_side, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&a.filled, cudaEventDisableTiming) != cudaSuccess)
             return GPTQ_ERR_CUDA;
     }
     *out = &a;
@@ -425,9 +442,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
         if (cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(DIAG_SMEM)) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(place_diag_inverse_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(NB * LD * sizeof(float))) != cudaSuccess)
+            cudaSuccess)
             return GPTQ_ERR_CUDA;
         attr_set[dev] = true;
     }
@@ -456,6 +471,9 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         const int rc = launch_fill(Z, int64_t(d) * d, 0.0f, as);
         if (rc) return rc;
     }
+    // the diagonal kernels write Z's diagonal blocks: after the fill
+    if (cudaEventRecord(aux->filled, as) != cudaSuccess || cudaStreamWaitEvent(stream, aux->filled, 0) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
 
     // Cholesky of A (lower), blocked right-looking, products on the tensor
     // cores.  Step k on `stream`: factor the diagonal block, solve the panel,
@@ -470,7 +488,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     for (int k = 0; k < nblk; ++k) {
         const int k0 = k * NB;
         float* dk = Dinv + size_t(k) * NB * NB;
-        potrf_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, stream>>>(A, d, k0, dk, info, st); count_launch();
+        potrf_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, stream>>>(A, d, k0, dk, Z, info, st); count_launch();
         const int rest = d - k0 - NB;
         float* panel = A + size_t(k0 + NB) * d + k0;
         int rc;
@@ -500,8 +518,8 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
                 if (cudaEventRecord(aux->rest, ss) != cudaSuccess) return GPTQ_ERR_CUDA;
             }
         }
-        // inverse block step k on the auxiliary stream
-        place_diag_inverse_t_kernel<<<1, 512, NB * LD * sizeof(float), as>>>(dk, d, k, Z); count_launch();
+        // inverse block step k on the auxiliary stream (Z's diagonal block k
+        // was written by the diagonal kernel)
         if (k > 0) {
             float* zi = Z + k0;   // in place is safe for the same reason as the panel
             rc = launch_tgemm(k0, NB, NB, 1.0f, zi, nullptr, d, dk, nullptr, NB, false, zi, d, false, as, st);
