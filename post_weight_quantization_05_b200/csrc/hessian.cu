@@ -5,26 +5,30 @@
 // (accumulated per layer over the calibration batches).
 //
 // Design (B200):
-//  - H is symmetric, so only output tiles that reach the upper triangle are
-//    computed.  Tile = 128 (a) x 256 (b) of H; the contraction runs over the
+//  - H is symmetric, so only the 256 x 256 output tiles (ta <= tb) that reach
+//    the upper triangle are computed; the contraction runs over the
 //    calibration rows r.  X is row-major [n, d], i.e. both operands of the
 //    product X[:, a-tile]^T X[:, b-tile] are MN-major (the a / b index is the
 //    contiguous one), which tcgen05 reads directly from 128-byte-swizzled
 //    shared memory -- no transpose pass over X.
-//  - Per stage a TMA load brings 64 calibration rows of the a-columns
-//    (16 KB) and of the b-columns (32 KB); 4 stages in flight.  One thread
-//    issues TMA, one thread issues tcgen05.mma (M=128, N=256, K=16, fp32
-//    accumulator in TMEM).
+//  - A cluster of two CTAs (two SMs) owns a tile and runs it as cta_group::2
+//    MMAs (M = 256, N = 256, K = 16, fp32 accumulators in TMEM): CTA r loads
+//    64 calibration rows of its 128 a-columns and of its 128 of the 256
+//    b-columns per stage (32 KB, six stages in flight), and the pair's MMA
+//    reads both CTAs' halves.  Per SM that is two thirds of the bytes a
+//    single-CTA 128 x 256 tile would stream for the same MMA work, which is
+//    what lets the loads stay ahead of the tensor cores.  One thread per CTA
+//    issues TMA, one thread of CTA 0 issues the MMAs.
 //  - Promotion: the tensor core's fp32 accumulation loses about half an ulp
 //    per accumulation step (measured: relative error ~4e-5 over a chain of
 //    16384 rows).  So the K loop is cut into chunks of 512 rows, each summed
 //    into one of two TMEM buffers (2 x 256 columns) while eight epilogue warps
-//    drain the other buffer and add it into fp32 registers (round to
+//    per CTA drain the other buffer and add it into fp32 registers (round to
 //    nearest); at the end they add 2 * sum into H.
 //  - fp32 inputs are split into three bf16 terms by `split3_kernel`; the
 //    contraction then runs over the six leading cross products
 //    (hh, hm, mh, mm, hl, lh), which the K loop walks one after another.
-//  - No TMA multicast anywhere.
+//  - No TMA load uses multicast (each CTA loads its own halves).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -33,61 +37,57 @@
 namespace gptq {
 namespace hess {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;
-constexpr int STAGES = 4;
+constexpr int BK = 64;            // calibration rows per stage
 constexpr int CHUNK = 8;          // k-steps (of BK rows) summed in TMEM before promotion
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int CHUNK_BYTES = 64 * BK * 2;  // one TMA box: 64 columns x 64 rows
-constexpr int TMEM_COLS = 2 * BN;         // two accumulator buffers
+constexpr int CHUNK_BYTES = 64 * BK * 2;  // one TMA box: 64 columns x 64 rows of bf16
 constexpr int EPI_WARPS = 8;              // 4 TMEM lane quadrants x 2 column halves
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
+constexpr int BMH = 128;                   // H rows per CTA (the pair covers 256)
+constexpr int BNP = 256;                   // H columns per pair (128 loaded by each CTA)
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BMH * BK * 2;      // 16 KB
+constexpr int B_BYTES = (BNP / 2) * BK * 2;  // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BNP;         // two accumulator buffers
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + size_t(STAGES) * STAGE_BYTES + 256 /*barriers*/;
 
+// Pair protocol: CTA r (r = 0, 1) loads a-columns a0 + 128 r .. + 127 and
+// b-columns b0 + 128 r .. + 127 of each slab; both CTAs' TMA loads complete on
+// CTA 0's `full` barrier; CTA 0's MMA commits arrive on both CTAs' `empty` and
+// `tfull`; the epilogue warps of both CTAs arrive on CTA 0's `tempty`.  Each
+// CTA's TMEM holds its 128 rows x 256 columns.
+
 struct Params {
-    int d;          // d_in
-    int n;          // calibration rows in this call
-    int npairs;     // number of (A part, B part) products
-    int pa[6];
-    int pb[6];
-    float alpha;    // 2.0
-    int tiles_b;    // ceil(d / BN)
-    int tiles_a;    // d / BM
+    int d, n, npairs;
+    int pa[6], pb[6];
+    float alpha;
+    int tiles;      // T (T + 1) / 2 tiles (ta <= tb) of 256 x 256, T = ceil(d / 256)
+    int T;
 };
 
-// Map a linear tile index to (ti, tj): tiles (ti, tj) with ti*BM <= tj*BN + BN - 1.
-__device__ __forceinline__ void tile_coords(int t, const Params& p, int& ti, int& tj) {
-    int acc = 0;
-    for (tj = 0; tj < p.tiles_b; ++tj) {
-        int cnt = min(p.tiles_a, (tj * BN + BN - 1) / BM + 1);
-        if (t < acc + cnt) {
-            ti = t - acc;
-            return;
-        }
-        acc += cnt;
-    }
-    ti = -1;
-}
-
-__global__ void __launch_bounds__(THREADS, 1)
-    syrk_kernel(const __grid_constant__ CUtensorMap tmX, const Params p, float* __restrict__ H,
-                DevStatus* st) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    syrk_pair_kernel(const __grid_constant__ CUtensorMap tmX, const Params p, float* __restrict__ H,
+                     DevStatus* st) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(STAGES) * STAGE_BYTES);
-    uint64_t* empty = full + STAGES;
-    uint64_t* tfull = empty + STAGES;   // [2] MMA -> epilogue: chunk summed in buffer b
-    uint64_t* tempty = tfull + 2;       // [2] epilogue -> MMA: buffer b drained
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(STAGES) * STAGE_BYTES);  // CTA 0: both halves landed
+    uint64_t* empty = full + STAGES;    // both CTAs: the pair's MMAs are done with the stage
+    uint64_t* tfull = empty + STAGES;   // [2] both CTAs: chunk summed in buffer b
+    uint64_t* tempty = tfull + 2;       // [2] CTA 0: buffer b drained by both CTAs
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
 
-    int ti, tj;
-    tile_coords(blockIdx.x, p, ti, tj);
-    if (ti < 0) return;
-    const int a0 = ti * BM;
-    const int b0 = tj * BN;
+    const uint32_t rank = cluster_ctarank();
+    // tile (ta, tb), ta <= tb, column-major over tb
+    int ta = 0, tb = 0;
+    {
+        int t = int(blockIdx.x >> 1), acc = 0;
+        for (tb = 0; tb < p.T; ++tb) {
+            if (t < acc + tb + 1) { ta = t - acc; break; }
+            acc += tb + 1;
+        }
+    }
+    const int a0 = ta * BNP + int(rank) * BMH;   // this CTA's H rows
+    const int b0 = tb * BNP;                     // the pair's H columns
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -99,16 +99,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], EPI_WARPS);
+            mbar_init(&tempty[b], 2 * EPI_WARPS);
         }
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();          // barriers of both CTAs initialized, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -118,72 +118,62 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- TMA producer
-            bool ok = true;
-            int last_round[STAGES];
-#pragma unroll
-            for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
+            // ---------------- TMA producer (both CTAs)
             for (int ks = 0; ks < ksteps; ++ks) {
                 const int s = ks % STAGES;
                 const uint32_t round = ks / STAGES;
-                if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, st, 101)) { ok = false; break; }
+                if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, st, 111)) break;
                 const int pair = ks / kper;
                 const int r0 = (ks - pair * kper) * BK;
                 uint8_t* sa = smem + size_t(s) * STAGE_BYTES;
                 uint8_t* sb = sa + A_BYTES;
-                mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
+                const uint32_t fb = mapa_shared(&full[s], 0);
 #pragma unroll
-                for (int h = 0; h < BM / 64; ++h)
-                    tma_load_3d(sa + h * CHUNK_BYTES, &tmX, a0 + 64 * h, r0, p.pa[pair], &full[s]);
+                for (int h = 0; h < BMH / 64; ++h)
+                    tma_load_3d_pair(sa + h * CHUNK_BYTES, &tmX, a0 + 64 * h, r0, p.pa[pair], fb);
 #pragma unroll
-                for (int h = 0; h < BN / 64; ++h)
-                    tma_load_3d(sb + h * CHUNK_BYTES, &tmX, b0 + 64 * h, r0, p.pb[pair], &full[s]);
-                last_round[s] = int(round);
-            }
-            if (!ok) {
-                // let the copies already in flight land before the CTA can exit
-#pragma unroll
-                for (int s = 0; s < STAGES; ++s)
-                    if (last_round[s] >= 0) (void)mbar_wait(&full[s], uint32_t(last_round[s]) & 1u, st, 104);
+                for (int h = 0; h < BNP / 128; ++h)
+                    tma_load_3d_pair(sb + h * CHUNK_BYTES, &tmX, b0 + int(rank) * 128 + 64 * h, r0, p.pb[pair], fb);
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- MMA issuer
-            constexpr uint32_t idesc = idesc_bf16_mn_mn(BM, BN);
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer (CTA 0 only)
+            constexpr uint32_t idesc = idesc_bf16_mn_mn(2 * BMH, BNP);
             bool ok = true;
             for (int c = 0; c < nchunks && ok; ++c) {
                 const int buf = c & 1;
                 const int use = c >> 1;
-                if (use > 0 && !mbar_wait(&tempty[buf], uint32_t(use - 1) & 1u, st, 105)) { ok = false; break; }
+                if (use > 0 && !mbar_wait_cluster(&tempty[buf], uint32_t(use - 1) & 1u, st, 115)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t dt = tmem_base + uint32_t(buf * BN);
+                const uint32_t dt = tmem_base + uint32_t(buf * BNP);
                 const int k_end = min(ksteps, (c + 1) * CHUNK);
                 for (int ks = c * CHUNK; ks < k_end; ++ks) {
                     const int s = ks % STAGES;
                     const uint32_t round = ks / STAGES;
-                    if (!mbar_wait(&full[s], round & 1u, st, 102)) { ok = false; break; }
+                    if (!mbar_wait(&full[s], round & 1u, st, 112)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + size_t(s) * STAGE_BYTES);
                     const uint32_t sb = sa + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        // 16 K rows = two 8-row groups of 128 bytes each
                         const uint64_t da = sdesc_sw128(sa + kk * 2048, CHUNK_BYTES, 1024);
                         const uint64_t db = sdesc_sw128(sb + kk * 2048, CHUNK_BYTES, 1024);
-                        umma_f16(dt, da, db, idesc, (ks > c * CHUNK || kk > 0) ? 1u : 0u);
+                        umma_f16_pair(dt, da, db, idesc, (ks > c * CHUNK || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(&empty[s]);  // frees the stage once these MMAs are done
+                    umma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
                 }
-                umma_commit(&tfull[buf]);    // this chunk's sum is complete (also on the error path)
+                umma_commit_pair_both(&tfull[buf]);     // chunk complete (also on the error path)
             }
         }
     } else {
-        // ---------------- epilogue warps: promote each chunk into fp32 registers
+        // ---------------- epilogue warps (both CTAs)
         const int e = warp - 2;
-        const int quad = warp & 3;           // TMEM lanes this warp may access
-        const int half = e >> 2;             // which 128 of the 256 columns
+        const int quad = warp & 3;
+        const int half = e >> 2;
         const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+        const uint32_t te = mapa_shared(&tempty[0], 0);   // CTA 0's tempty[0]; [1] is 8 bytes on
         float acc[128];
 #pragma unroll
         for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
@@ -191,21 +181,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
             const int use = c >> 1;
-            if (!mbar_wait(&tfull[buf], uint32_t(use) & 1u, st, 103)) { ok = false; break; }
+            if (!mbar_wait(&tfull[buf], uint32_t(use) & 1u, st, 113)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 float v[32];
-                tmem_ld_32x32b_x32(tmem_base + lane_addr + uint32_t(buf * BN + half * 128 + cc * 32), v);
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + uint32_t(buf * BNP + half * 128 + cc * 32), v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) acc[cc * 32 + i] += v[i];
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (lane == 0) mbar_arrive_cluster(te + uint32_t(buf) * 8u);
         }
-        if (ok && nchunks > 0) {
-            const int a = a0 + quad * 32 + lane;   // TMEM lane == row of the tile
+        const int a = a0 + quad * 32 + lane;   // TMEM lane == row of this CTA's half
+        if (ok && nchunks > 0 && a < p.d) {
             float* hrow = H + size_t(a) * p.d;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
@@ -230,8 +220,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
     tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem_base, TMEM_COLS);
+    cluster_sync();          // no remote arrival or pair MMA is still pending
+    if (warp == 0) tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
 // x = h + m + l with h, m, l bf16 (each the bf16 rounding of what remains).
@@ -288,20 +278,18 @@ int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, voi
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
-    p.tiles_a = int(d / BM);
-    p.tiles_b = int((d + BN - 1) / BN);
-    int tiles = 0;
-    for (int tj = 0; tj < p.tiles_b; ++tj) tiles += std::min(p.tiles_a, (tj * BN + BN - 1) / BM + 1);
+    p.T = int((d + BNP - 1) / BNP);
+    p.tiles = p.T * (p.T + 1) / 2;
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(syrk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES)) !=
+        if (cudaFuncSetAttribute(syrk_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES)) !=
             cudaSuccess)
             return GPTQ_ERR_CUDA;
         attr_set[dev] = true;
     }
-    syrk_kernel<<<tiles, THREADS, SMEM_BYTES, stream>>>(tm, p, H, st); count_launch();
+    syrk_pair_kernel<<<2 * p.tiles, THREADS, SMEM_BYTES, stream>>>(tm, p, H, st); count_launch();
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
