@@ -75,6 +75,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DevSta
     }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels launched with launch_pdl may start while the previous kernel in the
+// stream is still running.  Each such kernel sets up its shared memory / TMEM
+// first, then calls pdl_wait() -- which returns once the previous kernel has
+// finished and its writes are visible -- before it touches global memory, and
+// then pdl_trigger() to let the next kernel in the stream start its own setup.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---------------------------------------------------------------- clusters of two CTAs
 // (used by kernels launched with __cluster_dims__(2, 1, 1))
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -81,12 +81,13 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const fl
 // ---------------------------------------------------------------------------
 // One 128 x 128 diagonal block: L L^T = A_kk and L^-1, in one CTA of 12 warps.
 // The block is cut into 4 x 4 sub-blocks of 32.  Step kb (o = 32 kb):
-//   A: warp 0 factors the diagonal sub-block (kb, kb) in registers; the other
-//      warps meanwhile apply step kb-1 of the inverse's trailing update;
+//   A: warp 0 factors the diagonal sub-block (kb, kb) in registers; the warps
+//      on the other three schedulers meanwhile finish step kb-1: its trailing
+//      update beyond block column kb and its step of the inverse's update;
 //   B: warp 0 inverts the diagonal sub-block; warps 1-3 solve the sub-blocks
 //      below against it (one row per thread);
-//   C: the trailing update of the factorization (sub-blocks (bi, bj),
-//      kb < bj <= bi) and step kb of the inverse's block solve.
+//   C: the trailing update of block column kb+1 (what step kb+1 needs first)
+//      and step kb of the inverse's block solve.
 // The inverse Y = L^-1 is built right-looking on the identity (Y = X after
 //   X_k <- L_kk^-1 X_k;  X_i -= L_ik X_k  (i > k)  for k = 0..3)
 // and kept transposed (Yt = Y^T = L^-T) so that every product reads both of
@@ -96,7 +97,8 @@ __global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const fl
 constexpr int SB = 32;
 constexpr int LDS = NB + 4;              // S and Yt row stride (floats)
 constexpr int LDI = SB + 4;              // Lr row stride
-constexpr int DIAG_THREADS = 384;           // 12 warps: the most any phase below uses
+constexpr int DIAG_THREADS = 384;           // 12 warps
+constexpr int LDD = NB + 1;              // stride of the transposed inverse before it is written out
 constexpr size_t DIAG_SMEM = (size_t(2) * NB * LDS + size_t(SB) * LDI + 2 * SB + NB) * sizeof(float);
 
 // The 32 x 32 pieces are template recursions so that every register index is
@@ -135,6 +137,30 @@ struct RowChol32 {
         }
     }
 };
+
+// Warp-level Cholesky of one 32 x 32 diagonal sub-block in place: `row` is
+// this lane's row (row stride LDS in shared memory).  Kept out of line so that
+// its registers are allocated on their own, away from the rest of the kernel.
+__device__ __noinline__ void chol_sub_block(float* __restrict__ row, int lane, float* __restrict__ cb,
+                                            float* __restrict__ invd, uint32_t* badmask, uint32_t* nonfinite) {
+    float a[SB];
+#pragma unroll
+    for (int j = 0; j < SB; j += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(row + j);
+        a[j] = v.x; a[j + 1] = v.y; a[j + 2] = v.z; a[j + 3] = v.w;
+    }
+    cb[lane] = a[0];
+    __syncwarp();
+    uint32_t bad = 0, nf = 0;
+    RowChol32<0>::run(a, lane, cb, invd, bad, nf);
+#pragma unroll
+    for (int j = 0; j < SB; j += 4)
+        *reinterpret_cast<float4*>(row + j) =
+            make_float4(j <= lane ? a[j] : 0.0f, j + 1 <= lane ? a[j + 1] : 0.0f, j + 2 <= lane ? a[j + 2] : 0.0f,
+                        j + 3 <= lane ? a[j + 3] : 0.0f);
+    *badmask = bad;
+    *nonfinite = nf;
+}
 
 // One row x[] (32 values) solved against L (32 x 32 lower, shared memory,
 // row stride LDS):  x <- x L^-T  (right-looking, invd[c] = 1/L[c][c]).
@@ -215,21 +241,35 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
     float* cb = Lr + SB * LDI;         // [2][SB] published column (Cholesky steps)
     float* invd = cb + 2 * SB;         // [NB] 1 / L[c][c]
     __shared__ int failed;
+    pdl_wait();
+    pdl_trigger();
     if (*info != 0) return;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
 
-    // lower triangle of the block (zeros above), Yt = 0
-    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
-        const int r = idx / (NB / 4), c = (idx % (NB / 4)) * 4;
-        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        if (c <= r) {
-            v = *reinterpret_cast<const float4*>(A + size_t(k0 + r) * d + k0 + c);
-            if (c + 1 > r) v.y = 0.0f;
-            if (c + 2 > r) v.z = 0.0f;
-            if (c + 3 > r) v.w = 0.0f;
+    // lower triangle of the block (zeros above), Yt = 0; every load is issued
+    // before the first shared-memory store
+    {
+        constexpr int PER = (NB * NB / 4 + DIAG_THREADS - 1) / DIAG_THREADS;
+        float4 v[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int idx = t + i * DIAG_THREADS;
+            const int r = idx / (NB / 4), c = (idx % (NB / 4)) * 4;
+            v[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (idx < NB * NB / 4 && c <= r) v[i] = *reinterpret_cast<const float4*>(A + size_t(k0 + r) * d + k0 + c);
         }
-        *reinterpret_cast<float4*>(S + r * LDS + c) = v;
-        *reinterpret_cast<float4*>(Yt + r * LDS + c) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int idx = t + i * DIAG_THREADS;
+            if (idx >= NB * NB / 4) break;
+            const int r = idx / (NB / 4), c = (idx % (NB / 4)) * 4;
+            float4 w = v[i];
+            if (c + 1 > r) w.y = 0.0f;
+            if (c + 2 > r) w.z = 0.0f;
+            if (c + 3 > r) w.w = 0.0f;
+            *reinterpret_cast<float4*>(S + r * LDS + c) = w;
+            *reinterpret_cast<float4*>(Yt + r * LDS + c) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
     }
     if (t == 0) failed = 0;
     __syncthreads();
@@ -238,36 +278,38 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
         const int o = kb * SB;
         // ---- A: factor the diagonal sub-block (warp 0) || inverse update of step kb-1
         if (warp == 0) {
-            float a[SB];
-#pragma unroll
-            for (int j = 0; j < SB; j += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(S + (o + lane) * LDS + o + j);
-                a[j] = v.x; a[j + 1] = v.y; a[j + 2] = v.z; a[j + 3] = v.w;
-            }
-            cb[lane] = a[0];
-            __syncwarp();
             uint32_t badmask = 0, nonfinite = 0;   // the same in every lane
-            RowChol32<0>::run(a, lane, cb, invd + o, badmask, nonfinite);
-#pragma unroll
-            for (int j = 0; j < SB; j += 4)
-                *reinterpret_cast<float4*>(S + (o + lane) * LDS + o + j) =
-                    make_float4(j <= lane ? a[j] : 0.0f, j + 1 <= lane ? a[j + 1] : 0.0f,
-                                j + 2 <= lane ? a[j + 2] : 0.0f, j + 3 <= lane ? a[j + 3] : 0.0f);
+            chol_sub_block(S + (o + lane) * LDS + o, lane, cb, invd + o, &badmask, &nonfinite);
             if (badmask != 0 && lane == 0) {   // the first failing pivot of this sub-block
                 const int bad = __ffs(int(badmask)) - 1;
                 failed = 1;
                 if (atomicCAS(info, 0, k0 + o + bad + 1) == 0)
                     record_error(st, (nonfinite >> bad) & 1u ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_PD, k0 + o + bad + 1);
             }
-        } else if (kb > 0) {
-            // X_ij -= L_{i,kb-1} Y_{kb-1,j} for i >= kb, j < kb, transposed:
-            // Yt[j-block][i-block] -= Yt[j-block][(kb-1)-block] S[i-block][(kb-1)-block]^T
-            const int w = warp - 1;                  // 0..14
-            const int nj = kb, ni = NB / SB - kb;    // sub-blocks j < kb, i >= kb
-            if (w < 2 * ni * nj) {
-                const int blk = w >> 1, s = w & 1;
-                const int j = blk % nj, i = kb + blk / nj;
-                sub_block_update(Yt + (kb - 1) * SB, S + (kb - 1) * SB, Yt, j * SB, i * SB, s, lane);
+        } else if ((warp & 3) != 0 && kb > 0) {
+            // Work of step kb-1 that step kb's Cholesky does not wait for, on the
+            // warps that do not share warp 0's scheduler:
+            //  - the trailing update of step kb-1 beyond block column kb:
+            //    pairs (bi, bj), kb < bj <= bi;
+            //  - X_ij -= L_{i,kb-1} Y_{kb-1,j} for i >= kb, j < kb, transposed:
+            //    Yt[j-block][i-block] -= Yt[j-block][(kb-1)-block] S[i-block][(kb-1)-block]^T.
+            const int w = warp - 1 - (warp >> 2);              // 0 .. 3 * DIAG_THREADS / 128 - 1
+            const int nf = NB / SB - kb - 1;                   // sub-block columns after kb
+            const int far_tasks = nf * (nf + 1);               // two per pair
+            const int nj = kb, ni = NB / SB - kb;
+            const int tasks = far_tasks + 2 * ni * nj;
+            const int po = (kb - 1) * SB;
+            for (int task = w; task < tasks; task += 3 * DIAG_THREADS / 128) {
+                if (task < far_tasks) {
+                    int p = task >> 1, bi = kb + 1;
+                    while (p > bi - (kb + 1)) { p -= bi - kb; ++bi; }
+                    const int bj = kb + 1 + p;
+                    sub_block_update(S + po, S + po, S, bi * SB, bj * SB, task & 1, lane);
+                } else {
+                    const int blk = (task - far_tasks) >> 1, sh = (task - far_tasks) & 1;
+                    const int j = blk % nj, i = kb + blk / nj;
+                    sub_block_update(Yt + po, S + po, Yt, j * SB, i * SB, sh, lane);
+                }
             }
         }
         __syncthreads();
@@ -303,14 +345,13 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
 
         // ---- C: trailing update of the factorization || inverse solve of step kb
         {
-            const int nrest = NB / SB - kb - 1;            // sub-block rows / columns after kb
-            const int pair_warps = nrest * (nrest + 1);    // two warps per lower sub-block pair
+            // only block column kb+1 here (what step kb+1 needs first); the rest of
+            // this step's update runs beside step kb+1's Cholesky
+            const int nrest = NB / SB - kb - 1;            // sub-block rows after kb
+            const int pair_warps = 2 * nrest;              // two warps per pair (bi, kb+1)
             if (warp < pair_warps) {
-                // pair p = warp / 2 over (bi, bj), kb < bj <= bi, row-major
-                int p = warp >> 1, bi = kb + 1, bj = kb + 1;
-                while (p > bi - (kb + 1)) { p -= bi - kb; ++bi; }
-                bj = kb + 1 + p;
-                sub_block_update(S + o, S + o, S, bi * SB, bj * SB, warp & 1, lane);
+                const int bi = kb + 1 + (warp >> 1);
+                sub_block_update(S + o, S + o, S, bi * SB, (kb + 1) * SB, warp & 1, lane);
             } else if (warp < pair_warps + kb) {
                 // Y_{kb,j} = L_kk^-1 X_{kb,j} for j < kb: thread = column c of block j,
                 // reading X_{kb,j}[., c] as row (j*SB + c) of Yt
@@ -347,15 +388,20 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
         __syncthreads();
     }
 
-    // Z's diagonal block = Yt (rows), and Dinv = Yt^T
-    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
-        const int c = idx / (NB / 4), r = (idx % (NB / 4)) * 4;
-        *reinterpret_cast<float4*>(Z + size_t(k0 + c) * d + k0 + r) = *reinterpret_cast<const float4*>(Yt + c * LDS + r);
+    // Z's diagonal block = Yt (rows); Dinv = Yt^T, transposed into the factor's
+    // (now free) buffer with an odd row stride -- conflict-free on both sides --
+    // and written out row by row
+    float* D = S;   // [NB][LDD]
+    for (int idx = t; idx < NB * NB; idx += DIAG_THREADS) {
+        const int c = idx / NB, r = idx % NB;
+        const float v = Yt[c * LDS + r];
+        Z[size_t(k0 + c) * d + k0 + r] = v;
+        D[r * LDD + c] = v;
     }
-    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
-        const int r = idx % NB, c = (idx / NB) * 4;
-        *reinterpret_cast<float4*>(Dinv + r * NB + c) =
-            make_float4(Yt[c * LDS + r], Yt[(c + 1) * LDS + r], Yt[(c + 2) * LDS + r], Yt[(c + 3) * LDS + r]);
+    __syncthreads();
+    for (int idx = t; idx < NB * NB; idx += DIAG_THREADS) {
+        const int r = idx / NB, c = idx % NB;
+        Dinv[idx] = D[r * LDD + c];
     }
 }
 
@@ -488,7 +534,10 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     for (int k = 0; k < nblk; ++k) {
         const int k0 = k * NB;
         float* dk = Dinv + size_t(k) * NB * NB;
-        potrf_diag_kernel<<<1, DIAG_THREADS, DIAG_SMEM, stream>>>(A, d, k0, dk, Z, info, st); count_launch();
+        if (launch_pdl(potrf_diag_kernel, dim3(1), dim3(DIAG_THREADS), DIAG_SMEM, stream, static_cast<const float*>(A), d,
+                       k0, dk, Z, info, st) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        count_launch();
         const int rest = d - k0 - NB;
         float* panel = A + size_t(k0 + NB) * d + k0;
         int rc;

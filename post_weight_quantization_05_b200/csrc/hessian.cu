@@ -111,6 +111,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     cluster_sync();          // barriers of both CTAs initialized, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();              // H (and X) as the previous kernel left them
+    pdl_trigger();
 
     const int kper = (p.n + BK - 1) / BK;
     const int ksteps = kper * p.npairs;
@@ -289,7 +291,10 @@ int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, voi
             return GPTQ_ERR_CUDA;
         attr_set[dev] = true;
     }
-    syrk_pair_kernel<<<2 * p.tiles, THREADS, SMEM_BYTES, stream>>>(tm, p, H, st); count_launch();
+    if (launch_pdl(syrk_pair_kernel, dim3(2 * p.tiles), dim3(THREADS), SMEM_BYTES, stream, tm, p, H, st) !=
+        cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 

@@ -156,6 +156,8 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait();       // W as the previous trailing product left it
+    pdl_trigger();
     if (threadIdx.x == 0) {
         mbar_arrive_expect_tx(&bars[0], B * B * sizeof(float));
         tma_load_2d(Us, &tmU, i0, i0, &bars[0]);   // one 128 x 128 fp32 box, no swizzle
@@ -346,7 +348,10 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
         return GPTQ_ERR_CUDA;
     const int blocks = (a.d_out + SUB - 1) / SUB;
     for (int i0 = 0; i0 < a.d_in; i0 += B) {
-        sweep_block_kernel<BITS><<<blocks, SUB * NWIN, SMEM, stream>>>(tmU, a, i0); count_launch();
+        if (launch_pdl(sweep_block_kernel<BITS>, dim3(blocks), dim3(SUB * NWIN), SMEM, stream, tmU, a, i0) !=
+            cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        count_launch();
         const int tail = a.d_in - i0 - B;
         if (tail > 0) {
             // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]   (U[i0+k][i0+B+n] = Ut[i0+B+n][i0+k])

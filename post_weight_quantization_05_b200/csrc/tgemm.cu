@@ -166,6 +166,8 @@ __global__ void __launch_bounds__(Cfg<PRESPLIT>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();       // the previous kernel's output (our operands, C) is complete
+    pdl_trigger();
 
     if (warp == C::PRODUCER_WARP) {
         if (lane == 0) {
@@ -327,9 +329,11 @@ int launch_variant(const tg::Maps& maps, const tg::Args& g, cudaStream_t stream)
         attr_set[dev] = true;
     }
     const int grid = std::max(1, std::min(g.tiles, dev < 64 && sms[dev] > 0 ? sms[dev] : 148));
-    tg::tgemm_kernel<PRESPLIT><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(maps, g);
+    if (launch_pdl(tg::tgemm_kernel<PRESPLIT>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, maps, g) !=
+        cudaSuccess)
+        return GPTQ_ERR_CUDA;
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+    return GPTQ_OK;
 }
 }  // namespace
 
