@@ -356,9 +356,26 @@ __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
     lo = isfinite(x) ? x - hi : 0.0f;
 }
 
-// c = clamp(rint(w / s) + z, 0, maxq) (fp32, IEEE division).
-__device__ __forceinline__ float quant_code(float w, float s, float z, float maxq) {
-    return fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w, s)), z), 0.0f), maxq);
+// w / s rounded to nearest, given y = RN(1 / s) (__frcp_rn): q = RN(w y);
+// r = w - q s, exact with one fused multiply-add; RN(q + r y).  This is
+// P. Markstein's correction step for division with a fused multiply-add
+// ("Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Develop. 34(1), 1990): with y within half an ulp of
+// 1/s and q within one ulp of w/s, the result is the correctly rounded
+// quotient -- the same value as the IEEE division -- for normal operands; a
+// quotient too small to matter here (|w / s| < 2^-126) rounds to the same
+// integer either way.  Three dependent operations instead of a division on the
+// sweep's serial chain; the codes are checked against the fp32 oracle at
+// exact half-way points.
+__device__ __forceinline__ float div_by_recip(float w, float s, float y) {
+    const float q = __fmul_rn(w, y);
+    const float r = __fmaf_rn(-q, s, w);
+    return __fmaf_rn(r, y, q);
+}
+
+// c = clamp(rint(w / s) + z, 0, maxq) (fp32; inv_s = __frcp_rn(s)).
+__device__ __forceinline__ float quant_code(float w, float s, float inv_s, float z, float maxq) {
+    return fminf(fmaxf(__fadd_rn(rintf(div_by_recip(w, s, inv_s)), z), 0.0f), maxq);
 }
 
 // Non-tensor bulk copy global -> shared (16-byte aligned, size multiple of

@@ -10,9 +10,10 @@
 // Sweep kernel design: rows are independent given U (the same U serves every
 // row).  A CTA takes 32 rows (lane = row) and four warps, one per 32-column
 // window of the 128-column block.  Warp q holds its window of every row in
-// registers; it first applies the E of windows p < q (handed over through
-// shared memory, signalled by an mbarrier per window) to its columns, then
-// quantizes its window column by column.  The 128 x 128 diagonal block of U
+// registers; it applies the E of every column of the windows p < q as soon
+// as that column is done (each E goes through shared memory, followed by a
+// per-window progress count), so that the windows' sequential chains
+// overlap, then quantizes its own window column by column.  The 128 x 128 diagonal block of U
 // arrives by one TMA copy; every lane of a warp reads the same U element at
 // the same time (broadcast).  The block's E is written for the lazy trailing
 // product on the tensor cores.  The codes are packed in registers
@@ -89,28 +90,46 @@ struct Packer {
 };
 
 struct Grid {
-    float s, z, maxq;
+    float s, z, maxq, inv_s;   // inv_s = RN(1 / s)
 };
 
-// Column J of the window: quantize, pack, E = (w - q) / U_jj, and the rank-1
-// correction of the window's later columns (U row from shared memory).
+// Column J of the window: quantize, pack, E = (w - q) / U_jj, the rank-1
+// correction of the window's later columns (U row from shared memory, float4
+// broadcasts), and -- every PUB columns -- publishing the E so far to the
+// later windows (eh, then the window's progress count).
+constexpr int PUB = 8;
 template <int BITS, int J>
 struct WindowCol {
     __device__ __forceinline__ static void run(float (&w)[SUB], const float* __restrict__ Us, int wc,
                                                const float* __restrict__ invd, const Grid& gr, Packer<BITS>& pk,
-                                               float* Qw, bool& finite) {
+                                               float* Qw, bool& finite, float* eh, volatile int* prog, int lane) {
         const float wj = w[J];
-        const float c = quant_code(wj, gr.s, gr.z, gr.maxq);
+        const float c = quant_code(wj, gr.s, gr.inv_s, gr.z, gr.maxq);
         const float q = gr.s * (c - gr.z);
         const float e = (wj - q) * invd[J];
+        const float* urow = Us + (wc + J) * B + wc;
+#pragma unroll
+        for (int k4 = ((J + 1) / 4) * 4; k4 < SUB; k4 += 4) {
+            const float4 u = *reinterpret_cast<const float4*>(urow + k4);
+            if (k4 + 0 > J) w[k4 + 0] = fmaf(-e, u.x, w[k4 + 0]);
+            if (k4 + 1 > J) w[k4 + 1] = fmaf(-e, u.y, w[k4 + 1]);
+            if (k4 + 2 > J) w[k4 + 2] = fmaf(-e, u.z, w[k4 + 2]);
+            if (k4 + 3 > J) w[k4 + 3] = fmaf(-e, u.w, w[k4 + 3]);
+        }
+        w[J] = e;
+        if (eh != nullptr && (J % PUB == PUB - 1)) {   // (the same in every lane of the warp)
+#pragma unroll
+            for (int j = J + 1 - PUB; j <= J; ++j) eh[j] = w[j];
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                *prog = J + 1;
+            }
+        }
         finite &= isfinite(e);
         if (Qw) Qw[J] = q;
         pk.template put<J>(static_cast<uint32_t>(c));
-        const float* urow = Us + (wc + J) * B + wc;
-#pragma unroll
-        for (int k = J + 1; k < SUB; ++k) w[k] = fmaf(-e, urow[k], w[k]);
-        w[J] = e;
-        if constexpr (J + 1 < SUB) WindowCol<BITS, J + 1>::run(w, Us, wc, invd, gr, pk, Qw, finite);
+        if constexpr (J + 1 < SUB) WindowCol<BITS, J + 1>::run(w, Us, wc, invd, gr, pk, Qw, finite, eh, prog, lane);
     }
 };
 
@@ -131,7 +150,7 @@ struct SweepArgs {
 };
 
 // shared memory: U block, E hand-over (one [32][ELD] per window), 1/U_jj per
-// window, reduction and grid scratch, mbarriers
+// window, reduction and grid scratch, the U mbarrier and the progress counts
 constexpr size_t SMEM = 1024 /*align slack*/ +
                         (size_t(B) * B + size_t(NWIN) * SUB * ELD + B + 4 * NWIN * SUB) * sizeof(float) + 64;
 
@@ -144,7 +163,8 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
     float* Eh = Us + B * B;                    // Eh[p][row][j]: E of window p
     float* invd = Eh + NWIN * SUB * ELD;       // 1 / U[i0+j][i0+j]
     float* red = invd + B;                     // [2][NWIN][SUB] min / max, then [2][SUB] grid
-    uint64_t* bars = reinterpret_cast<uint64_t*>(red + 4 * NWIN * SUB);   // [0] U landed, [1+p] window p's E
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + 4 * NWIN * SUB);   // [0] U landed
+    int* prog = reinterpret_cast<int*>(bars + 1 + NWIN);   // [p]: columns of window p whose E is in Eh
     const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wc = q * SUB;
     const int r = blockIdx.x * SUB + lane;
@@ -152,16 +172,16 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[0], 1);
-        for (int p = 0; p < NWIN; ++p) mbar_init(&bars[1 + p], SUB);
+        for (int p = 0; p < NWIN; ++p) prog[p] = 0;
         fence_mbar_init();
     }
     __syncthreads();
-    pdl_wait();       // W as the previous trailing product left it
-    pdl_trigger();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0) {   // U is not written by the kernel before this one: copy it before waiting
         mbar_arrive_expect_tx(&bars[0], B * B * sizeof(float));
         tma_load_2d(Us, &tmU, i0, i0, &bars[0]);   // one 128 x 128 fp32 box, no swizzle
     }
+    pdl_wait();       // W as the previous trailing product left it
+    pdl_trigger();
 
     // this warp's window of this lane's row, and its min / max
     float w[SUB];
@@ -218,40 +238,53 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
     const bool loaded = mbar_wait(&bars[0], 0, a.st, 201);
     invd[wc + lane] = loaded ? 1.0f / Us[(wc + lane) * B + wc + lane] : 0.0f;
     __syncthreads();
-    Grid gr{gsh[lane], gsh[SUB + lane], a.maxq};
+    Grid gr{gsh[lane], gsh[SUB + lane], a.maxq, __frcp_rn(gsh[lane])};
 
-    // E of the earlier windows, applied to this window (in window order)
-    for (int p = 0; p < q; ++p) {
-        const bool ready = mbar_wait(&bars[1 + p], 0, a.st, 202);
-        if (!ready) break;
-        const float* eh = Eh + (p * SUB + lane) * ELD;
-#pragma unroll 4
-        for (int j = 0; j < SUB; ++j) {
-            const float e = eh[j];
-            const float4* u4 = reinterpret_cast<const float4*>(Us + (p * SUB + j) * B + wc);
+    // E of the earlier windows' columns, applied to this window as each column
+    // is published (in column order; the updates commute)
+    {
+        const int total = q * SUB;
+        int c = 0;
+        uint32_t spins = 0;
+        unsigned long long t0 = 0;
+        while (c < total) {
+            const int p = c / SUB;
+            const int avail = p * SUB + __shfl_sync(0xffffffffu, static_cast<volatile int*>(prog)[p], 0);
+            if (avail <= c) {
+                if ((++spins & 255u) == 0u) {   // bounded wait for the earlier window
+                    const unsigned long long now = globaltimer_ns();
+                    if (t0 == 0) t0 = now;
+                    else if (now - t0 > kWaitLimitNs) { record_error(a.st, GPTQ_ERR_TIMEOUT, 202); break; }
+                }
+                continue;
+            }
+            __threadfence_block();
+            for (; c < avail; c += PUB) {   // windows publish PUB columns at a time
+                float e[PUB];
 #pragma unroll
-            for (int k4 = 0; k4 < SUB / 4; ++k4) {
-                const float4 u = u4[k4];
-                w[4 * k4 + 0] = fmaf(-e, u.x, w[4 * k4 + 0]);
-                w[4 * k4 + 1] = fmaf(-e, u.y, w[4 * k4 + 1]);
-                w[4 * k4 + 2] = fmaf(-e, u.z, w[4 * k4 + 2]);
-                w[4 * k4 + 3] = fmaf(-e, u.w, w[4 * k4 + 3]);
+                for (int t = 0; t < PUB; ++t) e[t] = Eh[(p * SUB + lane) * ELD + (c - p * SUB) + t];
+#pragma unroll
+                for (int t = 0; t < PUB; ++t) {
+                    const float4* u4 = reinterpret_cast<const float4*>(Us + (c + t) * B + wc);
+#pragma unroll
+                    for (int k4 = 0; k4 < SUB / 4; ++k4) {
+                        const float4 u = u4[k4];
+                        w[4 * k4 + 0] = fmaf(-e[t], u.x, w[4 * k4 + 0]);
+                        w[4 * k4 + 1] = fmaf(-e[t], u.y, w[4 * k4 + 1]);
+                        w[4 * k4 + 2] = fmaf(-e[t], u.z, w[4 * k4 + 2]);
+                        w[4 * k4 + 3] = fmaf(-e[t], u.w, w[4 * k4 + 3]);
+                    }
+                }
             }
         }
     }
 
-    // this window, column by column
+    // this window, column by column (each E published to the later windows)
     Packer<BITS> pk;
     float* qrow = (a.Q && active) ? a.Q + size_t(r) * a.d_in + i0 + wc : nullptr;
-    WindowCol<BITS, 0>::run(w, Us, wc, invd + wc, gr, pk, qrow, finite);
+    float* eh = q + 1 < NWIN ? Eh + (q * SUB + lane) * ELD : nullptr;
+    WindowCol<BITS, 0>::run(w, Us, wc, invd + wc, gr, pk, qrow, finite, eh, prog + q, lane);
 
-    // hand E to the later windows, then write E and the codes
-    if (q + 1 < NWIN) {
-        float* eh = Eh + (q * SUB + lane) * ELD;
-#pragma unroll
-        for (int j = 0; j < SUB; ++j) eh[j] = w[j];
-        mbar_arrive(&bars[1 + q]);
-    }
     if (active) {
         // E leaves pre-split for the trailing product's tensor cores
         float* erow = a.E + size_t(r) * B + wc;
@@ -282,6 +315,7 @@ __global__ void rtn_kernel(const float* __restrict__ W, int d_out, int d_in, int
     const int c0 = u * 32;
     const size_t gi = size_t(r) * n_groups + c0 / group;
     const float s = __half2float(__ushort_as_half(scales[gi]));
+    const float inv_s = __frcp_rn(s);
     const float z = __half2float(__ushort_as_half(zeros[gi]));
     const float* src = W + size_t(r) * d_in + c0;
     uint32_t words[BITS] = {};
@@ -291,7 +325,7 @@ __global__ void rtn_kernel(const float* __restrict__ W, int d_out, int d_in, int
         const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t c = static_cast<uint32_t>(quant_code(vv[i], s, z, maxq));
+            const uint32_t c = static_cast<uint32_t>(quant_code(vv[i], s, inv_s, z, maxq));
             const int pos = (k + i) * BITS, word = pos / 32, off = pos % 32;
             words[word] |= c << off;
             if (off + BITS > 32) words[word + 1] |= c >> (32 - off);

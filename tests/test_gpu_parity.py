@@ -79,6 +79,48 @@ def test_rtn_degenerate_rows():
     assert np.array_equal(Q.cpu().numpy().astype(np.float64), ref["Q"])
 
 
+def _halfway_rows(n_rows, seed):
+    """Rows whose grid is known exactly (min and max are whole multiples of an
+    fp16 scale s) and whose other entries sit exactly on the half-way points
+    (k + 1/2) s and 1-2 ulps either side of them: the codes there depend on
+    the last bit of the fp32 quotient w / s and on round-half-even."""
+    rng = np.random.default_rng(seed)
+    W = np.zeros((n_rows, 128), dtype=np.float32)
+    for r in range(n_rows):
+        e = int(rng.integers(-14, 3))
+        s = np.float32(np.float16(2.0 ** e * (1 + int(rng.integers(0, 1024)) / 1024)))
+        lo = -int(rng.integers(1, 16)) if r % 2 else 0          # z = -lo (0 on even rows, > 0 on odd)
+        row = [np.float32(lo) * s, np.float32(lo + 15) * s]
+        for k in range(lo, lo + 15):
+            mid = np.float32((k + 0.5) * float(s))
+            assert float(mid) == (k + 0.5) * float(s)         # exact in fp32
+            for j in (-2, -1, 0, 1, 2):
+                v = mid
+                for _ in range(abs(j)):
+                    v = np.nextafter(v, np.float32(np.inf) if j > 0 else np.float32(-np.inf), dtype=np.float32)
+                row.append(v)
+        row = np.array(row, dtype=np.float32)
+        fill = (lo + rng.random(128 - len(row)) * 15).astype(np.float32) * s
+        W[r] = np.concatenate([row, fill])
+    return W
+
+
+def test_rtn_halfway_points_bit_exact():
+    """The GPU's fp32 quotient (reciprocal + one fused correction) must decide
+    every half-way code exactly as the oracle's IEEE division does."""
+    W = _halfway_rows(96, 7)
+    ref = oracle.rtn_quantize(W, 4, -1)
+    assert np.all(ref["zeros"][1::2] > 0) and np.all(ref["zeros"][0::2] == 0)
+    Wt = torch.from_numpy(W).cuda()
+    codes = torch.zeros((W.shape[0], 16), dtype=torch.int32, device="cuda")
+    scales = torch.zeros((W.shape[0], 1), dtype=torch.float16, device="cuda")
+    zeros = torch.zeros((W.shape[0], 1), dtype=torch.float16, device="cuda")
+    api.rtn_layer(Wt, 4, -1, codes, scales, zeros, None)
+    api.get_status()
+    assert np.array_equal(fp16_values(scales), ref["scales"])
+    assert np.array_equal(codes.cpu().numpy().view(np.uint32), oracle.pack_codes(ref["codes"], 4))
+
+
 # ---------------------------------------------------------------- H
 @pytest.mark.parametrize("n,d", [(1000, 384), (4096, 512), (333, 768), (64, 128), (20480, 1024)])
 def test_hessian_bf16(n, d):
