@@ -94,23 +94,34 @@ struct Grid {
 };
 
 // Column J of the window: quantize, pack, E = (w - q) / U_jj, the rank-1
-// correction of the window's later columns (U row from shared memory, float4
-// broadcasts), and -- every PUB columns -- publishing the E so far to the
-// later windows (eh, then the window's progress count).
+// correction of the window's later columns and -- every PUB columns --
+// publishing the E so far to the later windows (eh, then the window's
+// progress count).  Row J of the U block (float4 broadcasts from shared
+// memory) and 1 / U_jj arrive in ucur / icur: each column loads the next
+// column's while it computes, so no load latency sits on the serial chain.
 constexpr int PUB = 8;
+constexpr int SUB4 = SUB / 4;
 template <int BITS, int J>
 struct WindowCol {
     __device__ __forceinline__ static void run(float (&w)[SUB], const float* __restrict__ Us, int wc,
                                                const float* __restrict__ invd, const Grid& gr, Packer<BITS>& pk,
-                                               float* Qw, bool& finite, float* eh, volatile int* prog, int lane) {
+                                               float* Qw, bool& finite, float* eh, volatile int* prog, int lane,
+                                               const float4 (&ucur)[SUB4], float icur) {
+        float4 unext[SUB4];
+        float inext = 0.0f;
+        if constexpr (J + 1 < SUB) {
+            const float* nrow = Us + (wc + J + 1) * B + wc;
+#pragma unroll
+            for (int k4 = ((J + 2) / 4) * 4; k4 < SUB; k4 += 4) unext[k4 / 4] = *reinterpret_cast<const float4*>(nrow + k4);
+            inext = invd[J + 1];
+        }
         const float wj = w[J];
         const float c = quant_code(wj, gr.s, gr.inv_s, gr.z, gr.maxq);
         const float q = gr.s * (c - gr.z);
-        const float e = (wj - q) * invd[J];
-        const float* urow = Us + (wc + J) * B + wc;
+        const float e = (wj - q) * icur;
 #pragma unroll
         for (int k4 = ((J + 1) / 4) * 4; k4 < SUB; k4 += 4) {
-            const float4 u = *reinterpret_cast<const float4*>(urow + k4);
+            const float4 u = ucur[k4 / 4];
             if (k4 + 0 > J) w[k4 + 0] = fmaf(-e, u.x, w[k4 + 0]);
             if (k4 + 1 > J) w[k4 + 1] = fmaf(-e, u.y, w[k4 + 1]);
             if (k4 + 2 > J) w[k4 + 2] = fmaf(-e, u.z, w[k4 + 2]);
@@ -129,7 +140,8 @@ struct WindowCol {
         finite &= isfinite(e);
         if (Qw) Qw[J] = q;
         pk.template put<J>(static_cast<uint32_t>(c));
-        if constexpr (J + 1 < SUB) WindowCol<BITS, J + 1>::run(w, Us, wc, invd, gr, pk, Qw, finite, eh, prog, lane);
+        if constexpr (J + 1 < SUB)
+            WindowCol<BITS, J + 1>::run(w, Us, wc, invd, gr, pk, Qw, finite, eh, prog, lane, unext, inext);
     }
 };
 
@@ -149,24 +161,40 @@ struct SweepArgs {
     DevStatus* st;
 };
 
-// shared memory: U block, E hand-over (one [32][ELD] per window), 1/U_jj per
-// window, reduction and grid scratch, the U mbarrier and the progress counts
+// Four warps per window.  Before a window's serial chain starts, its columns
+// must receive the E of every earlier column (a rank-1 update per column); the
+// four warps of the window share that work (8 columns each), then three of
+// them hand their columns to the window's owner warp (h = 0), which runs the
+// chain.
+constexpr int HELP = 4;                       // warps per window
+constexpr int HC = SUB / HELP;                // columns per warp while updating
+constexpr int SWEEP_THREADS = 32 * NWIN * HELP;
+constexpr int HLD = SUB + 1;                  // hand-over rows (conflict-free)
+
+// shared memory: U block, E hand-over (one [32][ELD] per window), column
+// hand-over to the owners ([NWIN][32][HLD]), 1/U_jj, min / max per warp and
+// the grid, the U mbarrier and the progress counts
 constexpr size_t SMEM = 1024 /*align slack*/ +
-                        (size_t(B) * B + size_t(NWIN) * SUB * ELD + B + 4 * NWIN * SUB) * sizeof(float) + 64;
+                        (size_t(B) * B + size_t(NWIN) * SUB * ELD + size_t(NWIN) * SUB * HLD + B +
+                         2 * size_t(NWIN) * HELP * SUB + 2 * SUB) * sizeof(float) + 64;
 
 template <int BITS>
-__global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_constant__ CUtensorMap tmU,
-                                                                 const SweepArgs a, int i0) {
+__global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(const __grid_constant__ CUtensorMap tmU,
+                                                                    const SweepArgs a, int i0) {
     extern __shared__ uint8_t smem_raw[];
     float* sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* Us = sm;                            // Us[j][k] = U[i0+j][i0+k]  (TMA destination: 1024-aligned)
     float* Eh = Us + B * B;                    // Eh[p][row][j]: E of window p
-    float* invd = Eh + NWIN * SUB * ELD;       // 1 / U[i0+j][i0+j]
-    float* red = invd + B;                     // [2][NWIN][SUB] min / max, then [2][SUB] grid
-    uint64_t* bars = reinterpret_cast<uint64_t*>(red + 4 * NWIN * SUB);   // [0] U landed
+    float* Hv = Eh + NWIN * SUB * ELD;         // Hv[q][row][k]: window q's columns after the update
+    float* invd = Hv + NWIN * SUB * HLD;       // 1 / U[i0+j][i0+j]
+    float* red = invd + B;                     // [2][NWIN * HELP][SUB] min / max per warp
+    float* gsh = red + 2 * NWIN * HELP * SUB;  // [2][SUB] grid of each row
+    uint64_t* bars = reinterpret_cast<uint64_t*>(gsh + 2 * SUB);   // [0] U landed
     int* prog = reinterpret_cast<int*>(bars + 1 + NWIN);   // [p]: columns of window p whose E is in Eh
-    const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wc = q * SUB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp / HELP, h = warp % HELP;   // window, and this warp's share of it
+    const int wc = q * SUB;                       // window's first column in the block
+    const int hc = wc + h * HC;                   // this warp's columns while updating
     const int r = blockIdx.x * SUB + lane;
     const bool active = r < a.d_out;
 
@@ -183,25 +211,26 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
     pdl_wait();       // W as the previous trailing product left it
     pdl_trigger();
 
-    // this warp's window of this lane's row, and its min / max
-    float w[SUB];
-    const float* wsrc = a.W + size_t(active ? r : 0) * a.d_in + i0 + wc;
-    float mn = INFINITY, mx = -INFINITY;
+    // this warp's 8 columns of this lane's row, and their min / max
+    float v[HC];
+    {
+        const float* wsrc = a.W + size_t(active ? r : 0) * a.d_in + i0 + hc;
+        float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < SUB; k += 4) {
-        const float4 v = active ? *reinterpret_cast<const float4*>(wsrc + k) : make_float4(0.f, 0.f, 0.f, 0.f);
-        w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
-        mn = fminf(fminf(mn, v.x), fminf(v.y, fminf(v.z, v.w)));
-        mx = fmaxf(fmaxf(mx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
+        for (int k = 0; k < HC; k += 4) {
+            const float4 x = active ? *reinterpret_cast<const float4*>(wsrc + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[k] = x.x; v[k + 1] = x.y; v[k + 2] = x.z; v[k + 3] = x.w;
+            mn = fminf(fminf(mn, x.x), fminf(x.y, fminf(x.z, x.w)));
+            mx = fmaxf(fmaxf(mx, x.x), fmaxf(x.y, fmaxf(x.z, x.w)));
+        }
+        red[warp * SUB + lane] = mn;
+        red[(NWIN * HELP + warp) * SUB + lane] = mx;
     }
-    red[q * SUB + lane] = mn;
-    red[(NWIN + q) * SUB + lane] = mx;
     __syncthreads();
 
-    // grid of each row (warp 0), handed to the other warps through shared memory
-    float* gsh = red + 2 * NWIN * SUB;
+    // grid of each row (warp 0), handed to the others through shared memory
     bool finite = true;
-    if (q == 0 && active) {
+    if (warp == 0 && active) {
         float s, z;
         if (a.groupsize < 0) {
             s = __half2float(__ushort_as_half(a.scales[r]));
@@ -211,17 +240,17 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
             if (i0 % a.groupsize == 0) {
                 // grid from the current weights of the group: this block as loaded,
                 // later columns of the group from W (already lazily updated)
-                float gmn = red[lane], gmx = red[NWIN * SUB + lane];
+                float gmn = red[lane], gmx = red[NWIN * HELP * SUB + lane];
 #pragma unroll
-                for (int p = 1; p < NWIN; ++p) {
+                for (int p = 1; p < NWIN * HELP; ++p) {
                     gmn = fminf(gmn, red[p * SUB + lane]);
-                    gmx = fmaxf(gmx, red[(NWIN + p) * SUB + lane]);
+                    gmx = fmaxf(gmx, red[(NWIN * HELP + p) * SUB + lane]);
                 }
                 const float* rowp = a.W + size_t(r) * a.d_in + i0;
                 for (int c = B; c < a.groupsize; c += 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(rowp + c);
-                    gmn = fminf(fminf(gmn, v.x), fminf(v.y, fminf(v.z, v.w)));
-                    gmx = fmaxf(fmaxf(gmx, v.x), fmaxf(v.y, fmaxf(v.z, v.w)));
+                    const float4 x = *reinterpret_cast<const float4*>(rowp + c);
+                    gmn = fminf(fminf(gmn, x.x), fminf(x.y, fminf(x.z, x.w)));
+                    gmx = fmaxf(fmaxf(gmx, x.x), fmaxf(x.y, fmaxf(x.z, x.w)));
                 }
                 __half s16, z16;
                 finite &= grid_params(gmn, gmx, a.maxq, s, z, s16, z16);
@@ -236,14 +265,13 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
         gsh[SUB + lane] = z;
     }
     const bool loaded = mbar_wait(&bars[0], 0, a.st, 201);
-    invd[wc + lane] = loaded ? 1.0f / Us[(wc + lane) * B + wc + lane] : 0.0f;
+    if (threadIdx.x < B) invd[threadIdx.x] = loaded ? 1.0f / Us[threadIdx.x * B + threadIdx.x] : 0.0f;
     __syncthreads();
-    Grid gr{gsh[lane], gsh[SUB + lane], a.maxq, __frcp_rn(gsh[lane])};
 
-    // E of the earlier windows' columns, applied to this window as each column
-    // is published (in column order; the updates commute)
+    // E of the earlier windows' columns, applied to this warp's 8 columns as
+    // each batch is published (in column order; the updates commute)
     {
-        const int total = q * SUB;
+        const int total = wc;
         int c = 0;
         uint32_t spins = 0;
         unsigned long long t0 = 0;
@@ -265,25 +293,42 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
                 for (int t = 0; t < PUB; ++t) e[t] = Eh[(p * SUB + lane) * ELD + (c - p * SUB) + t];
 #pragma unroll
                 for (int t = 0; t < PUB; ++t) {
-                    const float4* u4 = reinterpret_cast<const float4*>(Us + (c + t) * B + wc);
+                    const float4* u4 = reinterpret_cast<const float4*>(Us + (c + t) * B + hc);
 #pragma unroll
-                    for (int k4 = 0; k4 < SUB / 4; ++k4) {
+                    for (int k4 = 0; k4 < HC / 4; ++k4) {
                         const float4 u = u4[k4];
-                        w[4 * k4 + 0] = fmaf(-e[t], u.x, w[4 * k4 + 0]);
-                        w[4 * k4 + 1] = fmaf(-e[t], u.y, w[4 * k4 + 1]);
-                        w[4 * k4 + 2] = fmaf(-e[t], u.z, w[4 * k4 + 2]);
-                        w[4 * k4 + 3] = fmaf(-e[t], u.w, w[4 * k4 + 3]);
+                        v[4 * k4 + 0] = fmaf(-e[t], u.x, v[4 * k4 + 0]);
+                        v[4 * k4 + 1] = fmaf(-e[t], u.y, v[4 * k4 + 1]);
+                        v[4 * k4 + 2] = fmaf(-e[t], u.z, v[4 * k4 + 2]);
+                        v[4 * k4 + 3] = fmaf(-e[t], u.w, v[4 * k4 + 3]);
                     }
                 }
             }
         }
     }
 
-    // this window, column by column (each E published to the later windows)
+    // hand the updated columns to the window's owner
+    if (h != 0) {
+#pragma unroll
+        for (int k = 0; k < HC; ++k) Hv[(q * SUB + lane) * HLD + h * HC + k] = v[k];
+    }
+    named_barrier_sync(1 + q, 32 * HELP);
+    if (h != 0) return;
+
+    // the owner: this window, column by column (each E published to the later windows)
+    float w[SUB];
+#pragma unroll
+    for (int k = 0; k < HC; ++k) w[k] = v[k];
+#pragma unroll
+    for (int k = HC; k < SUB; ++k) w[k] = Hv[(q * SUB + lane) * HLD + k];
+    const Grid gr{gsh[lane], gsh[SUB + lane], a.maxq, __frcp_rn(gsh[lane])};
     Packer<BITS> pk;
     float* qrow = (a.Q && active) ? a.Q + size_t(r) * a.d_in + i0 + wc : nullptr;
     float* eh = q + 1 < NWIN ? Eh + (q * SUB + lane) * ELD : nullptr;
-    WindowCol<BITS, 0>::run(w, Us, wc, invd + wc, gr, pk, qrow, finite, eh, prog + q, lane);
+    float4 u0[SUB4];
+#pragma unroll
+    for (int k4 = 0; k4 < SUB4; ++k4) u0[k4] = *reinterpret_cast<const float4*>(Us + wc * B + wc + 4 * k4);
+    WindowCol<BITS, 0>::run(w, Us, wc, invd + wc, gr, pk, qrow, finite, eh, prog + q, lane, u0, invd[wc]);
 
     if (active) {
         // E leaves pre-split for the trailing product's tensor cores
@@ -291,11 +336,11 @@ __global__ void __launch_bounds__(SUB * NWIN) sweep_block_kernel(const __grid_co
         float* elo = a.E_lo + size_t(r) * B + wc;
 #pragma unroll
         for (int j = 0; j < SUB; j += 4) {
-            float4 h, l;
-            split_tf32(w[j], h.x, l.x); split_tf32(w[j + 1], h.y, l.y);
-            split_tf32(w[j + 2], h.z, l.z); split_tf32(w[j + 3], h.w, l.w);
-            *reinterpret_cast<float4*>(erow + j) = h;
-            *reinterpret_cast<float4*>(elo + j) = l;
+            float4 hi, lo;
+            split_tf32(w[j], hi.x, lo.x); split_tf32(w[j + 1], hi.y, lo.y);
+            split_tf32(w[j + 2], hi.z, lo.z); split_tf32(w[j + 3], hi.w, lo.w);
+            *reinterpret_cast<float4*>(erow + j) = hi;
+            *reinterpret_cast<float4*>(elo + j) = lo;
         }
         pk.store(a.codes + size_t(r) * (size_t(a.d_in) * BITS / 32) + size_t(i0 + wc) * BITS / 32);
         if (!finite) record_error(a.st, GPTQ_ERR_NONFINITE, r);
@@ -382,7 +427,7 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
         return GPTQ_ERR_CUDA;
     const int blocks = (a.d_out + SUB - 1) / SUB;
     for (int i0 = 0; i0 < a.d_in; i0 += B) {
-        if (launch_pdl(sweep_block_kernel<BITS>, dim3(blocks), dim3(SUB * NWIN), SMEM, stream, tmU, a, i0) !=
+        if (launch_pdl(sweep_block_kernel<BITS>, dim3(blocks), dim3(SWEEP_THREADS), SMEM, stream, tmU, a, i0) !=
             cudaSuccess)
             return GPTQ_ERR_CUDA;
         count_launch();
