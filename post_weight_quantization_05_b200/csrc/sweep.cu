@@ -192,7 +192,10 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(const __grid
     uint64_t* bars = reinterpret_cast<uint64_t*>(gsh + 2 * SUB);   // [0] U landed
     int* prog = reinterpret_cast<int*>(bars + 1 + NWIN);   // [p]: columns of window p whose E is in Eh
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = warp / HELP, h = warp % HELP;   // window, and this warp's share of it
+    // window q's four warps are q, q + 4, q + 8, q + 12: one scheduler per
+    // window, so a window's serial chain never shares issue slots with the
+    // updates the later windows run meanwhile
+    const int q = warp % NWIN, h = warp / NWIN;   // window, and this warp's share of it
     const int wc = q * SUB;                       // window's first column in the block
     const int hc = wc + h * HC;                   // this warp's columns while updating
     const int r = blockIdx.x * SUB + lane;
