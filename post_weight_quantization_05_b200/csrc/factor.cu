@@ -27,6 +27,9 @@ namespace gptq {
 namespace factor {
 
 constexpr int NB = 128;
+// Block columns the critical stream updates after each panel (the rest of the
+// trailing update goes to the side stream).
+constexpr int NEAR = 3;
 
 struct Layout {
     size_t a_off, y_off, dinv_off, scal_off, total;
@@ -409,13 +412,15 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
 // The factorization's critical chain runs on a high-priority stream; the
 // inverse's block steps run on another, each as soon as the factorization has
 // finished the block column it needs; the trailing update beyond the next
-// block column runs on a low-priority stream, so that the next diagonal block
-// is factored while it proceeds (look-ahead) and gets the SMs first.
+// NEAR block columns runs on a low-priority stream, so that the next diagonal
+// blocks are factored while it proceeds (look-ahead) and get the SMs first.
 struct AuxStream {
     cudaStream_t main = nullptr;    // the factorization's critical chain (highest priority)
     cudaStream_t s = nullptr;       // inverse steps
-    cudaStream_t side = nullptr;    // trailing updates beyond the next block column
-    cudaEvent_t fork = nullptr, step = nullptr, rest = nullptr, join = nullptr, join_side = nullptr, filled = nullptr;
+    cudaStream_t side = nullptr;    // trailing updates beyond the next NEAR block columns
+    static constexpr int RING = 4;
+    cudaEvent_t fork = nullptr, step = nullptr, join = nullptr, join_side = nullptr, filled = nullptr;
+    cudaEvent_t far_done[RING] = {};   // the far update of step k, slot k % RING
 };
 
 static int aux_stream(AuxStream** out) {
@@ -433,11 +438,13 @@ static int aux_stream(AuxStream** out) {
             cudaStreamCreateWithPriority(&a.side, cudaStreamNonBlocking, least) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.step, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&a.rest, cudaEventDisableTiming) != cudaSuccess ||
+
             cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.join_side, cudaEventDisableTiming) != cudaSuccess ||
             cudaEventCreateWithFlags(&a.filled, cudaEventDisableTiming) != cudaSuccess)
             return GPTQ_ERR_CUDA;
+        for (int i = 0; i < AuxStream::RING; ++i)
+            if (cudaEventCreateWithFlags(&a.far_done[i], cudaEventDisableTiming) != cudaSuccess) return GPTQ_ERR_CUDA;
     }
     *out = &a;
     return GPTQ_OK;
@@ -508,10 +515,10 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     damp_lambda_kernel<<<1, 1024, 0, stream>>>(H, d, percdamp, lam, info, st); count_launch();
     reverse_damp_kernel<<<ew_blocks, 256, 0, stream>>>(H, d, lam, A); count_launch();
     // fork: the inverse (stream `as`) starts from a zeroed Z; `ss` takes the
-    // trailing updates beyond the next block column
+    // trailing updates beyond the next NEAR block columns
     const cudaStream_t ss = aux->side;
     if (cudaEventRecord(aux->fork, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->fork, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(ss, aux->fork, 0) != cudaSuccess || cudaEventRecord(aux->rest, ss) != cudaSuccess)
+        cudaStreamWaitEvent(ss, aux->fork, 0) != cudaSuccess)
         return GPTQ_ERR_CUDA;
     {
         const int rc = launch_fill(Z, int64_t(d) * d, 0.0f, as);
@@ -523,8 +530,8 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
 
     // Cholesky of A (lower), blocked right-looking, products on the tensor
     // cores.  Step k on `stream`: factor the diagonal block, solve the panel,
-    // update the next block column (after the previous step's far update on
-    // `ss` is done); the rest of the trailing update goes to `ss`.
+    // update the next NEAR block columns; the rest of the trailing update goes
+    // to `ss`.
     // Z = L^-T (upper) on `as`: block step i needs only L's block column i and
     // Dinv_i, so it runs as soon as the factorization has them:
     //   Z[i][i] = Dinv_i^T;  Z[0:i0, i] <- Z[0:i0, i] Dinv_i^T;
@@ -534,6 +541,13 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     for (int k = 0; k < nblk; ++k) {
         const int k0 = k * NB;
         float* dk = Dinv + size_t(k) * NB * NB;
+        // Block k needs every far update j <= k - NEAR - 1 (side stream, see
+        // below).  One wait every NEAR steps, for the far update of two steps
+        // back, covers all of them (the side stream runs in order) and keeps
+        // the other steps' kernels back to back for programmatic launch.
+        if (k % NEAR == 0 && k >= 2 &&
+            cudaStreamWaitEvent(stream, aux->far_done[(k - 2) % AuxStream::RING], 0) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
         if (launch_pdl(potrf_diag_kernel, dim3(1), dim3(DIAG_THREADS), DIAG_SMEM, stream, static_cast<const float*>(A), d,
                        k0, dk, Z, info, st) != cudaSuccess)
             return GPTQ_ERR_CUDA;
@@ -551,21 +565,25 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->step, 0) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         if (rest > 0) {
-            // next block column (it holds the next diagonal block) on `stream` ...
-            if (cudaStreamWaitEvent(stream, aux->rest, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
+            // the next NEAR block columns (they hold the next diagonal blocks) on
+            // `stream` ...
+            const int near_cols = std::min(rest, NEAR * NB);
             float* next = A + size_t(k0 + NB) * d + k0 + NB;
-            rc = launch_tgemm(rest, NB, NB, -1.0f, panel, nullptr, d, panel, nullptr, d, true, next, d, true, stream, st);
+            rc = launch_tgemm(rest, near_cols, NB, -1.0f, panel, nullptr, d, panel, nullptr, d, true, next, d, true,
+                              stream, st);
             if (rc) return rc;
-            // ... the columns after it on `ss`
-            if (rest > NB) {
+            // ... the columns after them on `ss` (reduce-adds into regions the
+            // next update may also be adding to: each element's add is atomic)
+            if (rest > NEAR * NB) {
                 if (cudaStreamWaitEvent(ss, aux->step, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
-                float* far = A + size_t(k0 + 2 * NB) * d + k0 + 2 * NB;
-                const float* prow = panel + size_t(NB) * d;
-                rc = launch_tgemm(rest - NB, rest - NB, NB, -1.0f, prow, nullptr, d, prow, nullptr, d, true, far, d, true,
-                                  ss, st);
+                const int f0 = k0 + (NEAR + 1) * NB;
+                float* far = A + size_t(f0) * d + f0;
+                const float* prow = panel + size_t(NEAR) * NB * d;
+                rc = launch_tgemm(rest - NEAR * NB, rest - NEAR * NB, NB, -1.0f, prow, nullptr, d, prow, nullptr, d,
+                                  true, far, d, true, ss, st);
                 if (rc) return rc;
-                if (cudaEventRecord(aux->rest, ss) != cudaSuccess) return GPTQ_ERR_CUDA;
             }
+            if (cudaEventRecord(aux->far_done[k % AuxStream::RING], ss) != cudaSuccess) return GPTQ_ERR_CUDA;
         }
         // inverse block step k on the auxiliary stream (Z's diagonal block k
         // was written by the diagonal kernel)
