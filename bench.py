@@ -48,7 +48,7 @@ def syrk_traffic_per_launch():
     """DRAM bytes (read + write) of one X^T X launch from the committed ncu
     summary, or None if the kernel's sources changed since that capture."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "syrk_kernel_attn4096.md")
+    path = os.path.join(ROOT, "profiles", "syrk_pair_kernel_attn4096.md")
     try:
         text = open(path).read()
     except OSError:
@@ -319,7 +319,7 @@ def main():
     flops_per_launch = n_b * p.d_in * (p.d_in + 1)       # upper triangle incl. diagonal, 2 flops per MAC
     h_launch_avg = statistics.mean(h_launch_ms)
     achieved = flops_per_launch / (h_launch_avg / 1e3) / 1e12
-    roof = {"kernel": "hessian syrk_kernel (tcgen05)", "bound": "tensor", "achieved": achieved,
+    roof = {"kernel": "hess::syrk_pair_kernel (tcgen05 cta_group::2)", "bound": "tensor", "achieved": achieved,
             "peak": sustained, "unit": "TFLOP/s", "frac": achieved / sustained,
             "peak_kind": f"bf16 dense sustained ({src})", "traffic": syrk_traffic_per_launch(),
             "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
