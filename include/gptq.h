@@ -94,6 +94,26 @@ int gptq_hessian_accumulate(const void* X, int dtype, int64_t n, int64_t d_in,
                             float* H, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Stage 1 over several calibration batches in one call: the same result as
+ * calling gptq_hessian_accumulate on X[0], X[1], ... in order, with the same
+ * H, dtype, d_in, workspace and stream (source as above: H accumulated over
+ * the calibration data).
+ *
+ *   X      HOST array of `count` device pointers; X[i] is [n[i], d_in]
+ *          row-major, 16-byte aligned (may be NULL where n[i] = 0).
+ *   n      HOST array of `count` row counts, each 0 <= n[i] < 2^31.
+ *   ws     as above, sized for the largest batch (fp32 only).
+ * Returns GPTQ_ERR_INVALID_ARG (launching nothing) if any argument is
+ * invalid.  Faster than separate calls for bf16 X: each batch's kernel
+ * waits for the previous batch's only before it updates H, so their
+ * contractions overlap on the GPU.  The batches must not be written by the
+ * GPU while the call's kernels run (they are read as the stream reaches
+ * them).
+ * ---------------------------------------------------------------------- */
+int gptq_hessian_accumulate_batches(const void* const* X, const int64_t* n, int count, int dtype,
+                                    int64_t d_in, float* H, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Stage 2 -- dampening and the upper Cholesky factor of the inverse.
  * Source: itwiki "GPTQ", "GPTQ의 세 가지 변경" row 3 (add 1% of the mean
  * diagonal; only the Cholesky form of H^-1 is needed, computed once up

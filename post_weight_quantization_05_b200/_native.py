@@ -24,6 +24,7 @@ SIGNATURES = {
     "gptq_status_string": (ctypes.c_char_p, [c_int]),
     "gptq_hessian_workspace_size": (c_size, [c_int, c_i64, c_i64]),
     "gptq_hessian_accumulate": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_size, c_vp]),
+    "gptq_hessian_accumulate_batches": (c_int, [c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_vp, c_size, c_vp]),
     "gptq_prepare_hinv_workspace_size": (c_size, [c_i64]),
     "gptq_prepare_hinv": (c_int, [c_vp, c_i64, c_float, c_vp, c_vp, c_vp, c_size, c_vp]),
     "gptq_quantize_workspace_size": (c_size, [c_i64, c_i64, c_int]),

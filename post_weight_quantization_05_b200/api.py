@@ -96,6 +96,30 @@ def hessian_accumulate(X: torch.Tensor, H: torch.Tensor, ws: torch.Tensor | None
     _check(code, "gptq_hessian_accumulate")
 
 
+def hessian_accumulate_batches(Xs, H: torch.Tensor, ws: torch.Tensor | None = None, stream=None):
+    """H += 2 X_i^T X_i for every batch X_i in order (one call; the batches'
+    contractions overlap on the GPU).  All X_i share one dtype and d_in."""
+    Xs = list(Xs)
+    if not Xs:
+        return
+    d = H.shape[0]
+    if Xs[0].dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("X must be bf16 or fp32")
+    dtype = GPTQ_BF16 if Xs[0].dtype == torch.bfloat16 else GPTQ_F32
+    for X in Xs:
+        _need(X, Xs[0].dtype, (X.shape[0], d), "X")
+    _need(H, torch.float32, (d, d), "H")
+    need = hessian_workspace_size(dtype, max(X.shape[0] for X in Xs), d)
+    if need and ws is None:
+        raise ValueError(f"fp32 X needs a workspace of {need} bytes")
+    ptrs = (ctypes.c_void_p * len(Xs))(*[X.data_ptr() for X in Xs])
+    rows = (ctypes.c_int64 * len(Xs))(*[X.shape[0] for X in Xs])
+    code = _lib().gptq_hessian_accumulate_batches(ptrs, rows, len(Xs), dtype, d, _ptr(H), _ptr(ws),
+                                                  0 if ws is None else ws.numel() * ws.element_size(),
+                                                  _stream(stream))
+    _check(code, "gptq_hessian_accumulate_batches")
+
+
 def prepare_hinv(H: torch.Tensor, U: torch.Tensor, ws: torch.Tensor, percdamp: float = 0.01,
                  info: torch.Tensor | None = None, stream=None):
     """U = upper Cholesky factor of (H + percdamp * mean(diag H) I)^-1."""
@@ -206,6 +230,10 @@ class LayerQuantizer:
 
     def add_batch(self, X: torch.Tensor, stream=None):
         hessian_accumulate(X, self.H, self.ws_h, stream)
+
+    def add_batches(self, Xs, stream=None):
+        """Several resident batches in one call (faster than add_batch each)."""
+        hessian_accumulate_batches(Xs, self.H, self.ws_h, stream)
 
     def finish(self, stream=None):
         prepare_hinv(self.H, self.U, self.ws_hinv, self.percdamp, self.info, stream)

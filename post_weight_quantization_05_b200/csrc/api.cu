@@ -1,5 +1,6 @@
 // C ABI of libgptq (declared in include/gptq.h): host-side validation, the
 // per-device status word, and the stream-ordered launches of each stage.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -118,6 +119,34 @@ int gptq_hessian_accumulate(const void* X, int dtype, int64_t n, int64_t d_in, f
     PFN_encodeTiled enc = nullptr;
     if (status_ptr(&st) || encode_fn(&enc)) return GPTQ_ERR_CUDA;
     return launch_hessian(X, dtype, n, d_in, H, ws, static_cast<cudaStream_t>(stream), st, enc);
+}
+
+int gptq_hessian_accumulate_batches(const void* const* X, const int64_t* n, int count, int dtype, int64_t d_in,
+                                    float* H, void* ws, size_t ws_bytes, void* stream) {
+    if (dtype != GPTQ_F32 && dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+    if (!valid_d_in(d_in) || count < 0 || (count > 0 && (!X || !n))) return GPTQ_ERR_INVALID_ARG;
+    if (!H || !aligned16(H)) return GPTQ_ERR_INVALID_ARG;
+    int64_t n_max = 0;
+    for (int i = 0; i < count; ++i) {
+        if (n[i] < 0 || n[i] > (int64_t(1) << 31) - 1) return GPTQ_ERR_INVALID_ARG;
+        if (n[i] > 0 && (!X[i] || !aligned16(X[i]))) return GPTQ_ERR_INVALID_ARG;
+        n_max = std::max(n_max, n[i]);
+    }
+    if (n_max == 0) return GPTQ_OK;
+    if (dtype == GPTQ_F32 && (!ws || !aligned16(ws) || ws_bytes < gptq_hessian_workspace_size(dtype, n_max, d_in)))
+        return GPTQ_ERR_INVALID_ARG;
+    DevStatus* st = nullptr;
+    PFN_encodeTiled enc = nullptr;
+    if (status_ptr(&st) || encode_fn(&enc)) return GPTQ_ERR_CUDA;
+    bool launched = false;
+    for (int i = 0; i < count; ++i) {
+        if (n[i] == 0) continue;
+        const int rc = launch_hessian(X[i], dtype, n[i], d_in, H, ws, static_cast<cudaStream_t>(stream), st, enc,
+                                      launched);
+        if (rc) return rc;
+        launched = true;
+    }
+    return GPTQ_OK;
 }
 
 size_t gptq_prepare_hinv_workspace_size(int64_t d_in) {

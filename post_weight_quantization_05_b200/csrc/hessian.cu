@@ -63,6 +63,7 @@ struct Params {
     float alpha;
     int tiles;      // T (T + 1) / 2 tiles (ta <= tb) of 256 x 256, T = ceil(d / 256)
     int T;
+    int late_wait;  // the previous kernel in the stream is this kernel on another batch
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
@@ -111,7 +112,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     cluster_sync();          // barriers of both CTAs initialized, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    pdl_wait();              // H (and X) as the previous kernel left them
+    // Wait for the previous kernel in the stream before any global access --
+    // unless it is this kernel on another batch (late_wait): that one never
+    // writes X, so only the final update of H has to wait for it, and the whole
+    // main loop overlaps its last wave.
+    if (!p.late_wait) pdl_wait();
     pdl_trigger();
 
     const int kper = (p.n + BK - 1) / BK;
@@ -197,6 +202,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive_cluster(te + uint32_t(buf) * 8u);
         }
         const int a = a0 + quad * 32 + lane;   // TMEM lane == row of this CTA's half
+        if (p.late_wait) pdl_wait();           // the previous batch's H is complete
         if (ok && nchunks > 0 && a < p.d) {
             float* hrow = H + size_t(a) * p.d;
 #pragma unroll
@@ -247,7 +253,7 @@ __global__ void split3_kernel(const float* __restrict__ X, __nv_bfloat16* __rest
 namespace gptq {
 
 int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, void* ws, cudaStream_t stream,
-                   DevStatus* st, PFN_encodeTiled encode) {
+                   DevStatus* st, PFN_encodeTiled encode, bool after_own_launch) {
     using namespace hess;
     if (n == 0) return GPTQ_OK;
     const void* base = X;
@@ -280,6 +286,7 @@ int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, voi
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
+    p.late_wait = (after_own_launch && dtype != GPTQ_F32) ? 1 : 0;
     p.T = int((d + BNP - 1) / BNP);
     p.tiles = p.T * (p.T + 1) / 2;
     static bool attr_set[64] = {false};

@@ -27,9 +27,11 @@ int validate_quantize_args(const float* W, int64_t d_out, int64_t d_in, const fl
                            int groupsize, const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
                            const float* Q);
 
-// hessian.cu
+// hessian.cu.  after_own_launch: the previous kernel in `stream` is this
+// library's H accumulation of another batch (bf16 only: the kernel then waits
+// for it only before updating H).
 int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, void* ws, cudaStream_t stream,
-                   DevStatus* st, PFN_encodeTiled encode);
+                   DevStatus* st, PFN_encodeTiled encode, bool after_own_launch = false);
 
 // tgemm.cu: C[M,N] = alpha * A[M,K] * B (accumulate = false) or
 // C[M,N] += alpha * A[M,K] * B (accumulate = true), B(k, n) = Bt[n * ldb + k],

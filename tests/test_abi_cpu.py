@@ -72,6 +72,26 @@ def test_hessian_rejects_bad_arguments(lib):
     assert f(None, 1, 0, 512, None, None, 0, None) == 0             # n == 0: no-op
 
 
+def test_hessian_batches_rejects_bad_arguments(lib):
+    f = lib.gptq_hessian_accumulate_batches
+    P = ctypes.c_void_p
+    X2 = (P * 2)(FAKE.value, FAKE.value)
+    n2 = (ctypes.c_int64 * 2)(64, 32)
+    assert f(X2, n2, 2, 1, 512, None, None, 0, None) == 1                       # NULL H
+    assert f(None, n2, 2, 1, 512, FAKE, None, 0, None) == 1                     # NULL X array
+    assert f(X2, None, 2, 1, 512, FAKE, None, 0, None) == 1                     # NULL n array
+    assert f(X2, n2, -1, 1, 512, FAKE, None, 0, None) == 1                      # negative count
+    assert f(X2, n2, 2, 7, 512, FAKE, None, 0, None) == 1                       # dtype
+    assert f(X2, n2, 2, 1, 500, FAKE, None, 0, None) == 1                       # d_in % 128
+    assert f((P * 2)(FAKE.value, MIS.value), n2, 2, 1, 512, FAKE, None, 0, None) == 1   # misaligned batch
+    assert f((P * 2)(FAKE.value, None), n2, 2, 1, 512, FAKE, None, 0, None) == 1        # NULL batch with rows
+    assert f(X2, (ctypes.c_int64 * 2)(64, -1), 2, 1, 512, FAKE, None, 0, None) == 1     # negative rows
+    assert f(X2, n2, 2, 0, 512, FAKE, None, 0, None) == 1                       # fp32 needs workspace
+    assert f(X2, n2, 2, 0, 512, FAKE, FAKE, 3 * 32 * 512 * 2, None) == 1        # sized for the smaller batch
+    assert f((P * 2)(None, None), (ctypes.c_int64 * 2)(0, 0), 2, 1, 512, FAKE, None, 0, None) == 0   # all empty
+    assert f(None, None, 0, 1, 512, FAKE, None, 0, None) == 0                   # no batches
+
+
 def test_prepare_hinv_rejects_bad_arguments(lib):
     f = lib.gptq_prepare_hinv
     ws = lib.gptq_prepare_hinv_workspace_size(512)

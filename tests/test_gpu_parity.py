@@ -122,6 +122,30 @@ def test_rtn_halfway_points_bit_exact():
 
 
 # ---------------------------------------------------------------- H
+@pytest.mark.parametrize("x_dtype,d", [("bf16", 640), ("bf16", 1024), ("f32", 512)])
+def test_hessian_batches_equal_separate_calls(x_dtype, d):
+    """One call over several batches (the contractions overlap on the GPU)
+    gives exactly the H of one call per batch, in the same order."""
+    p = synth.custom("hb", 8, d, 3 * 4096, x_dtype=x_dtype, n_batches=3, layer=d + 7)
+    xs = [to_dev_x(p, p.x_batch(b)) for b in range(p.n_batches)]
+    xs.insert(1, xs[0][:0])                                   # an empty batch in between
+    ws = None
+    if x_dtype == "f32":
+        ws = api.workspace(api.hessian_workspace_size(api.GPTQ_F32, max(x.shape[0] for x in xs), d), "cuda")
+    H1 = torch.zeros((d, d), dtype=torch.float32, device="cuda")
+    for x in xs:
+        if x.shape[0]:
+            api.hessian_accumulate(x, H1, ws)
+    H2 = torch.zeros((d, d), dtype=torch.float32, device="cuda")
+    api.hessian_accumulate_batches(xs, H2, ws)
+    api.get_status()
+    iu = np.triu_indices(d)
+    assert np.array_equal(H1.cpu().numpy()[iu], H2.cpu().numpy()[iu])
+    ref = oracle.hessian([synth.x_as_f32(p, p.x_batch(b)) for b in range(p.n_batches)])
+    got = H2.cpu().numpy().astype(np.float64)[iu]
+    assert np.linalg.norm(got - ref[iu]) / np.linalg.norm(ref[iu]) < H_TOL
+
+
 @pytest.mark.parametrize("n,d", [(1000, 384), (4096, 512), (333, 768), (64, 128), (20480, 1024)])
 def test_hessian_bf16(n, d):
     p = synth.custom("h", 8, d, n, x_dtype="bf16", n_batches=2, layer=d + n)
