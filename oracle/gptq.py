@@ -32,7 +32,11 @@ notes):
       j with j % g == 0, from the current (partially updated) W[:, j:j+g].
   R7  packing: little-endian bit stream of the codes along d_in, 32 codes per
       `bits` 32-bit words (int4: nibble k of word w holds code 8w+k).
-  R8  natural column order 0..d_in-1.
+  R8  natural column order 0..d_in-1 (act-order is a separate entry point).
+  R14 act-order: columns by descending diag(H), ties by index; the damping
+      is the same; groups are formed in processing order; codes / scales /
+      zeros stay in processing order together with the permutation, and Q is
+      returned in the original column order.
 
 Parity status: every function here is pinned by a test in
 tests/test_oracle_pins.py (closed forms, brute force, invariants, the page's
@@ -47,7 +51,7 @@ __all__ = [
     "hessian", "hessian_accumulate", "damp", "hinv_upper_factor", "hinv_upper_factor_ul",
     "grid_params", "quant_codes", "dequant", "gptq_quantize", "rtn_quantize",
     "pack_codes", "unpack_codes", "layer_loss_direct", "layer_loss_hessian",
-    "obq_fixed_order_row", "least_squares_refit",
+    "obq_fixed_order_row", "least_squares_refit", "act_order_perm", "gptq_quantize_act_order",
 ]
 
 FP16_MIN_NORMAL = 2.0 ** -14
@@ -211,6 +215,36 @@ def gptq_quantize(W, U, bits: int = 4, blocksize: int = 128, groupsize: int = -1
     if return_trace:
         out["W_at"] = W_at
         out["E"] = E_all
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Act-order ([wiki] "실무 변형": quantize the columns with the largest Hessian
+# diagonal -- the largest input activations -- first, so that the large errors
+# come early and the remaining columns can compensate for them)
+# ---------------------------------------------------------------------------
+def act_order_perm(H) -> np.ndarray:
+    """The processing order: column indices by descending diag(H), ties by
+    index (reading R14).  perm[k] is the original index of the k-th column
+    processed."""
+    return np.argsort(-np.diag(np.asarray(H, dtype=np.float64)), kind="stable")
+
+
+def gptq_quantize_act_order(W, H, bits: int = 4, blocksize: int = 128, groupsize: int = -1,
+                            percdamp: float = 0.01):
+    """GPTQ with the columns taken in act-order: the same Algorithm 1 on the
+    permuted problem (W[:, perm], H[perm][:, perm], damped as usual -- lambda
+    does not depend on the order).  Codes, scales and zeros stay in processing
+    order (groups are formed in that order, reading R14); Q is returned in the
+    original column order; `perm` is returned with them."""
+    H = np.asarray(H, dtype=np.float64)
+    perm = act_order_perm(H)
+    Hp = H[np.ix_(perm, perm)]
+    Hd, _ = damp(Hp, percdamp)
+    U = hinv_upper_factor(Hd)
+    out = gptq_quantize(np.asarray(W)[:, perm], U, bits, blocksize, groupsize)
+    out["Q"] = out["Q"][:, np.argsort(perm)]
+    out["perm"] = perm
     return out
 
 
