@@ -215,6 +215,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-act-order", action="store_true")
     ap.add_argument("--profile-case", action="store_true",
                     help="small case for ncu captures: one 16384-row batch of the same layer, 3 passes, no timing")
     args = ap.parse_args()
@@ -331,6 +332,11 @@ def main():
     stages = {"widen_W+zero_H": statistics.mean(begin_ms), "hessian_16_batches": statistics.mean(h_ms),
               "prepare_hinv": statistics.mean(prep_ms), "quantize_layer": statistics.mean(quant_ms)}
 
+    # ---- the same layer with act-order (columns by descending diag(H))
+    act = None
+    if not args.no_act_order:
+        act = act_order_timing(p, X_dev, W_dev, dev, stream, flush, args, api)
+
     # ---- end to end through the public API with host buffers (rank 0 .. all ranks)
     e2e = None
     if not args.no_e2e:
@@ -351,13 +357,52 @@ def main():
                            "blocksize": p.blocksize, "parallelism": f"replicas x{world}",
                            "l2": "flushed before every step (256 MiB write, outside the step events)"},
                 "ms_per_layer": ms_per_step, "stages_ms": stages, "roofline": roof, "cpu_baseline": cpu,
-                "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+                "e2e": e2e, "gpu_launches": launches, "clocks": clk, "act_order": act,
                 "input_generation_s": gen_s}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def act_order_timing(p, X_dev, W_dev, dev, stream, flush, args, api):
+    """The timed step again with act-order: the order, the permuted Hessian
+    and the permuted working copy of W between accumulation and
+    factorization.  Reports the step and the added stage (device events)."""
+    import torch
+    lq = api.LayerQuantizer(p.d_out, p.d_in, p.bits, p.groupsize, p.blocksize, p.percdamp, device=dev,
+                            act_order=True)
+
+    def step(evs):
+        evs[0].record(stream)
+        lq.begin(W_dev)
+        lq.add_batches(X_dev)
+        evs[1].record(stream)
+        api.act_order_perm(lq.H, lq.perm)
+        api.permute_hessian(lq.H, lq.perm, lq.Hp)
+        api.permute_columns(lq.W, lq.perm)
+        evs[2].record(stream)
+        api.prepare_hinv(lq.Hp, lq.U, lq.ws_hinv, p.percdamp, lq.info)
+        api.quantize_layer(lq.W, lq.U, p.bits, p.blocksize, p.groupsize, lq.codes, lq.scales, lq.zeros, lq.ws_q)
+        evs[3].record(stream)
+
+    runs = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        step(evs)
+        if i >= args.warmup:
+            runs.append(evs)
+    torch.cuda.synchronize(dev)
+    api.get_status(stream)
+    step_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in runs)
+    perm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in runs)
+    weights = p.d_out * p.d_in
+    return {"ms_per_step": step_ms, "value": weights / (step_ms / 1e3), "unit": "weights/s",
+            "order_and_permute_ms": perm_ms,
+            "stage": "act_order_perm + permute_hessian + permute_columns(W), device events",
+            "steps": args.steps, "warmup": args.warmup}
 
 
 def end_to_end(p, xs_host, w_bits, lq, dev, args, world, dist):

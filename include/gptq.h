@@ -218,6 +218,56 @@ int gptq_rtn_layer(const float* W, int64_t d_out, int64_t d_in, int bits, int gr
                    void* stream);
 
 /* ------------------------------------------------------------------------
+ * Act-order -- the columns in order of decreasing Hessian diagonal.
+ * Source: itwiki "GPTQ", "실무 변형" (act-order: the columns whose inputs
+ * carry the largest diag(H) are quantized first; it helps models with
+ * outlier channels).  The sweep itself is unchanged: it runs on the permuted
+ * problem.  A layer quantized with act-order is
+ *
+ *   gptq_act_order_perm(H, d_in, perm)                     processing order
+ *   gptq_permute_hessian(H, d_in, perm, Hp)                Hp = H[perm][:, perm]
+ *   gptq_prepare_hinv(Hp, ...)                             U of the permuted H
+ *   gptq_permute_columns(W, d_out, d_in, perm, 0, W)       W = W[:, perm]
+ *   gptq_quantize_layer(W, ..., U, ..., Q)                 codes in processing order
+ *   gptq_permute_columns(Q, d_out, d_in, perm, 1, Q)       Q back to W's order
+ *
+ * codes, scales and zeros stay in processing order (a group is `groupsize`
+ * consecutive columns of that order); column k of the codes belongs to
+ * column perm[k] of W.  Dampening does not depend on the order.
+ *
+ * gptq_act_order_perm: perm[k] = index of the column processed k-th: the
+ * indices sorted by diag(H) descending, equal values (-0 equal to +0) in
+ * increasing index order, NaN after every number.  Always a permutation.
+ *   H     device [d_in, d_in] fp32 (only the diagonal is read), 16-byte aligned.
+ *   perm  device int32 [d_in] output, 4-byte aligned, not inside H.
+ *
+ * gptq_permute_hessian: Hp[a][b] = Hs[perm[a]][perm[b]] for all a, b, where Hs
+ * is the symmetric matrix whose upper triangle is H's (the lower triangle of
+ * H is not read).  Hp is written whole (both triangles).
+ *   H, Hp device [d_in, d_in] fp32, 16-byte aligned, not overlapping.
+ *   perm  device int32 [d_in], a permutation of 0 .. d_in-1.  An entry
+ *         outside that range is recorded as GPTQ_ERR_INVALID_ARG in the status
+ *         word and the outputs it selects are NaN (nothing is read out of
+ *         bounds).
+ *
+ * gptq_permute_columns: for every row r of a [rows, cols] fp32 matrix,
+ *   inverse = 0:  dst[r][k] = src[r][perm[k]]     (into processing order)
+ *   inverse = 1:  dst[r][perm[k]] = src[r][k]     (back to the original order)
+ *   src, dst device, 16-byte aligned; either the same array (in place) or
+ *         not overlapping.  rows in [0, 2^24]; cols like d_in (a multiple of
+ *         128, at most 32768).
+ *   perm  device int32 [cols] as above; entries outside [0, cols) are
+ *         recorded as GPTQ_ERR_INVALID_ARG and select NaN; with inverse = 1,
+ *         slots of dst that no entry reaches are NaN.
+ * All three return GPTQ_ERR_INVALID_ARG (launching nothing) for a bad size,
+ * pointer, alignment or overlap.
+ * ---------------------------------------------------------------------- */
+int gptq_act_order_perm(const float* H, int64_t d_in, int32_t* perm, void* stream);
+int gptq_permute_hessian(const float* H, int64_t d_in, const int32_t* perm, float* Hp, void* stream);
+int gptq_permute_columns(const float* src, int64_t rows, int64_t cols, const int32_t* perm, int inverse,
+                         float* dst, void* stream);
+
+/* ------------------------------------------------------------------------
  * Helpers on the same stream (not steps of the method).
  * ---------------------------------------------------------------------- */
 /* dst[i] = (float) src[i] for bf16 bit patterns src (a bf16 layer's fp32

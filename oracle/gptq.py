@@ -231,18 +231,21 @@ def act_order_perm(H) -> np.ndarray:
 
 
 def gptq_quantize_act_order(W, H, bits: int = 4, blocksize: int = 128, groupsize: int = -1,
-                            percdamp: float = 0.01):
+                            percdamp: float = 0.01, perm=None, return_trace: bool = False):
     """GPTQ with the columns taken in act-order: the same Algorithm 1 on the
     permuted problem (W[:, perm], H[perm][:, perm], damped as usual -- lambda
     does not depend on the order).  Codes, scales and zeros stay in processing
     order (groups are formed in that order, reading R14); Q is returned in the
-    original column order; `perm` is returned with them."""
+    original column order; `perm` is returned with them.  `perm` may be given
+    (an order decided on another copy of the diagonal, e.g. an fp32 one whose
+    near-ties round differently); by default it is act_order_perm(H)."""
     H = np.asarray(H, dtype=np.float64)
-    perm = act_order_perm(H)
+    perm = act_order_perm(H) if perm is None else np.asarray(perm, dtype=np.int64)
+    assert np.array_equal(np.sort(perm), np.arange(H.shape[0])), "perm must be a permutation"
     Hp = H[np.ix_(perm, perm)]
     Hd, _ = damp(Hp, percdamp)
     U = hinv_upper_factor(Hd)
-    out = gptq_quantize(np.asarray(W)[:, perm], U, bits, blocksize, groupsize)
+    out = gptq_quantize(np.asarray(W)[:, perm], U, bits, blocksize, groupsize, return_trace=return_trace)
     out["Q"] = out["Q"][:, np.argsort(perm)]
     out["perm"] = perm
     return out

@@ -33,6 +33,9 @@ SIGNATURES = {
     "gptq_quantize_layer_noalloc": (c_int, [c_vp, c_i64, c_i64, c_vp, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp,
                                             c_vp]),
     "gptq_rtn_layer": (c_int, [c_vp, c_i64, c_i64, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "gptq_act_order_perm": (c_int, [c_vp, c_i64, c_vp, c_vp]),
+    "gptq_permute_hessian": (c_int, [c_vp, c_i64, c_vp, c_vp, c_vp]),
+    "gptq_permute_columns": (c_int, [c_vp, c_i64, c_i64, c_vp, c_int, c_vp, c_vp]),
     "gptq_widen_bf16": (c_int, [c_vp, c_vp, c_i64, c_vp]),
     "gptq_fill_f32": (c_int, [c_vp, c_i64, c_float, c_vp]),
     "gptq_get_status": (c_int, [c_vp, ctypes.POINTER(c_int)]),

@@ -172,6 +172,36 @@ def rtn_layer(W: torch.Tensor, bits: int, groupsize: int, codes: torch.Tensor, s
     _check(code, "gptq_rtn_layer")
 
 
+def act_order_perm(H: torch.Tensor, perm: torch.Tensor, stream=None):
+    """perm = column indices by descending diag(H) (ties by index, NaN last)."""
+    d = H.shape[0]
+    _need(H, torch.float32, (d, d), "H")
+    _need(perm, torch.int32, (d,), "perm")
+    _check(_lib().gptq_act_order_perm(_ptr(H), d, _ptr(perm), _stream(stream)), "gptq_act_order_perm")
+
+
+def permute_hessian(H: torch.Tensor, perm: torch.Tensor, Hp: torch.Tensor, stream=None):
+    """Hp = Hs[perm][:, perm], Hs the symmetric matrix of H's upper triangle."""
+    d = H.shape[0]
+    _need(H, torch.float32, (d, d), "H")
+    _need(perm, torch.int32, (d,), "perm")
+    _need(Hp, torch.float32, (d, d), "Hp")
+    _check(_lib().gptq_permute_hessian(_ptr(H), d, _ptr(perm), _ptr(Hp), _stream(stream)), "gptq_permute_hessian")
+
+
+def permute_columns(src: torch.Tensor, perm: torch.Tensor, dst: torch.Tensor | None = None, inverse: bool = False,
+                    stream=None):
+    """dst[:, k] = src[:, perm[k]] (inverse: dst[:, perm[k]] = src[:, k]); in
+    place when dst is src or None."""
+    rows, cols = src.shape
+    dst = src if dst is None else dst
+    _need(src, torch.float32, (rows, cols), "src")
+    _need(dst, torch.float32, (rows, cols), "dst")
+    _need(perm, torch.int32, (cols,), "perm")
+    _check(_lib().gptq_permute_columns(_ptr(src), rows, cols, _ptr(perm), 1 if inverse else 0, _ptr(dst),
+                                       _stream(stream)), "gptq_permute_columns")
+
+
 def widen_bf16(src: torch.Tensor, dst: torch.Tensor, stream=None):
     if src.dtype != torch.bfloat16 or dst.dtype != torch.float32 or src.numel() != dst.numel():
         raise ValueError("widen_bf16: bf16 -> fp32 of equal size")
@@ -198,12 +228,16 @@ class LayerQuantizer:
     """Device buffers for one layer shape plus the four calls in order.
 
     Allocation happens here, once (torch caching allocator); the calls
-    themselves only enqueue kernels."""
+    themselves only enqueue kernels.  With act_order the columns are taken by
+    descending diag(H): codes, scales and zeros come out in that processing
+    order (self.perm[k] is the column of W that code column k belongs to) and
+    Q in W's own order."""
 
     def __init__(self, d_out: int, d_in: int, bits: int = 4, groupsize: int = -1, blocksize: int = 128,
-                 percdamp: float = 0.01, device="cuda", want_q: bool = False, max_f32_rows: int = 0):
+                 percdamp: float = 0.01, device="cuda", want_q: bool = False, max_f32_rows: int = 0,
+                 act_order: bool = False):
         self.d_out, self.d_in, self.bits, self.groupsize = d_out, d_in, bits, groupsize
-        self.blocksize, self.percdamp = blocksize, percdamp
+        self.blocksize, self.percdamp, self.act_order = blocksize, percdamp, act_order
         dev = torch.device(device)
         self.H = torch.empty((d_in, d_in), dtype=torch.float32, device=dev)
         self.U = torch.empty((d_in, d_in), dtype=torch.float32, device=dev)
@@ -217,6 +251,8 @@ class LayerQuantizer:
         self.ws_hinv = workspace(prepare_hinv_workspace_size(d_in), dev)
         self.ws_q = workspace(quantize_workspace_size(d_out, d_in, blocksize), dev)
         self.ws_h = workspace(hessian_workspace_size(GPTQ_F32, max_f32_rows, d_in), dev) if max_f32_rows else None
+        self.perm = torch.empty((d_in,), dtype=torch.int32, device=dev) if act_order else None
+        self.Hp = torch.empty((d_in, d_in), dtype=torch.float32, device=dev) if act_order else None
 
     def begin(self, W_src: torch.Tensor, stream=None):
         """Load the working copy of W (fp32 copy or bf16 widening) and zero H."""
@@ -236,6 +272,14 @@ class LayerQuantizer:
         hessian_accumulate_batches(Xs, self.H, self.ws_h, stream)
 
     def finish(self, stream=None):
-        prepare_hinv(self.H, self.U, self.ws_hinv, self.percdamp, self.info, stream)
+        H = self.H
+        if self.act_order:
+            act_order_perm(self.H, self.perm, stream)
+            permute_hessian(self.H, self.perm, self.Hp, stream)
+            permute_columns(self.W, self.perm, stream=stream)
+            H = self.Hp
+        prepare_hinv(H, self.U, self.ws_hinv, self.percdamp, self.info, stream)
         quantize_layer(self.W, self.U, self.bits, self.blocksize, self.groupsize, self.codes, self.scales,
                        self.zeros, self.ws_q, self.Q, stream)
+        if self.act_order and self.Q is not None:
+            permute_columns(self.Q, self.perm, inverse=True, stream=stream)

@@ -199,6 +199,45 @@ int gptq_rtn_layer(const float* W, int64_t d_out, int64_t d_in, int bits, int gr
                       st);
 }
 
+int gptq_act_order_perm(const float* H, int64_t d_in, int32_t* perm, void* stream) {
+    if (!valid_d_in(d_in) || !H || !perm || !aligned16(H) || (reinterpret_cast<uintptr_t>(perm) & 3u))
+        return GPTQ_ERR_INVALID_ARG;
+    const uintptr_t h0 = reinterpret_cast<uintptr_t>(H), h1 = h0 + size_t(d_in) * size_t(d_in) * sizeof(float);
+    const uintptr_t p0 = reinterpret_cast<uintptr_t>(perm), p1 = p0 + size_t(d_in) * sizeof(int32_t);
+    if (p0 < h1 && h0 < p1) return GPTQ_ERR_INVALID_ARG;
+    return launch_act_order_perm(H, d_in, perm, static_cast<cudaStream_t>(stream));
+}
+
+int gptq_permute_hessian(const float* H, int64_t d_in, const int32_t* perm, float* Hp, void* stream) {
+    if (!valid_d_in(d_in) || !H || !perm || !Hp || !aligned16(H) || !aligned16(Hp) ||
+        (reinterpret_cast<uintptr_t>(perm) & 3u))
+        return GPTQ_ERR_INVALID_ARG;
+    const size_t bytes = size_t(d_in) * size_t(d_in) * sizeof(float);
+    const uintptr_t h0 = reinterpret_cast<uintptr_t>(H), o0 = reinterpret_cast<uintptr_t>(Hp);
+    const uintptr_t p0 = reinterpret_cast<uintptr_t>(perm), p1 = p0 + size_t(d_in) * sizeof(int32_t);
+    if ((o0 < h0 + bytes && h0 < o0 + bytes) || (p0 < o0 + bytes && o0 < p1)) return GPTQ_ERR_INVALID_ARG;
+    DevStatus* st = nullptr;
+    if (status_ptr(&st)) return GPTQ_ERR_CUDA;
+    return launch_permute_hessian(H, d_in, perm, Hp, static_cast<cudaStream_t>(stream), st);
+}
+
+int gptq_permute_columns(const float* src, int64_t rows, int64_t cols, const int32_t* perm, int inverse,
+                         float* dst, void* stream) {
+    if (rows < 0 || rows > (int64_t(1) << 24) || !valid_d_in(cols) || (inverse != 0 && inverse != 1))
+        return GPTQ_ERR_INVALID_ARG;
+    if (rows == 0) return GPTQ_OK;
+    if (!src || !dst || !perm || !aligned16(src) || !aligned16(dst) || (reinterpret_cast<uintptr_t>(perm) & 3u))
+        return GPTQ_ERR_INVALID_ARG;
+    const size_t bytes = size_t(rows) * size_t(cols) * sizeof(float);
+    const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+    const uintptr_t p0 = reinterpret_cast<uintptr_t>(perm), p1 = p0 + size_t(cols) * sizeof(int32_t);
+    if (s0 != d0 && s0 < d0 + bytes && d0 < s0 + bytes) return GPTQ_ERR_INVALID_ARG;   // partial overlap
+    if (p0 < d0 + bytes && d0 < p1) return GPTQ_ERR_INVALID_ARG;
+    DevStatus* st = nullptr;
+    if (status_ptr(&st)) return GPTQ_ERR_CUDA;
+    return launch_permute_columns(src, rows, cols, perm, inverse != 0, dst, static_cast<cudaStream_t>(stream), st);
+}
+
 int gptq_widen_bf16(const uint16_t* src, float* dst, int64_t count, void* stream) {
     if (count < 0) return GPTQ_ERR_INVALID_ARG;
     if (count == 0) return GPTQ_OK;

@@ -63,6 +63,14 @@ int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int b
 int launch_rtn(const float* W, int64_t d_out, int64_t d_in, int bits, int groupsize, uint32_t* codes,
                uint16_t* scales, uint16_t* zeros, float* Q, cudaStream_t stream, DevStatus* st);
 int launch_widen_bf16(const uint16_t* src, float* dst, int64_t count, cudaStream_t stream);
+
+// permute.cu (act-order): the processing order from diag(H), the permuted
+// Hessian, and the column permutation of a row-major matrix (in place allowed).
+int launch_act_order_perm(const float* H, int64_t d, int32_t* perm, cudaStream_t stream);
+int launch_permute_hessian(const float* H, int64_t d, const int32_t* perm, float* Hp, cudaStream_t stream,
+                           DevStatus* st);
+int launch_permute_columns(const float* src, int64_t rows, int64_t cols, const int32_t* perm, bool inverse,
+                           float* dst, cudaStream_t stream, DevStatus* st);
 int launch_fill(float* p, int64_t count, float value, cudaStream_t stream);
 
 }  // namespace gptq

@@ -147,6 +147,36 @@ def test_rtn_and_helpers_reject_bad_arguments(lib):
     assert lib.gptq_fill_f32(ctypes.c_void_p(0x10001), 10, 0.0, None) == 1
 
 
+def test_act_order_entries_reject_bad_arguments(lib):
+    d = 512
+    big = 0x10000 + d * d * 4 + 4096                  # an address past H / Hp / src
+    P = ctypes.c_void_p(big)
+    f = lib.gptq_act_order_perm
+    assert f(None, d, P, None) == 1
+    assert f(FAKE, d, None, None) == 1
+    assert f(MIS, d, P, None) == 1
+    assert f(FAKE, 500, P, None) == 1                 # d_in % 128 != 0
+    assert f(FAKE, d, ctypes.c_void_p(big + 2), None) == 1
+    assert f(FAKE, d, ctypes.c_void_p(0x10000 + 64), None) == 1     # perm inside H
+    g = lib.gptq_permute_hessian
+    HP = ctypes.c_void_p(big + 65536)
+    assert g(None, d, P, HP, None) == 1
+    assert g(FAKE, d, None, HP, None) == 1
+    assert g(FAKE, d, P, None, None) == 1
+    assert g(FAKE, d, P, ctypes.c_void_p(0x10000 + 4096), None) == 1  # Hp overlaps H
+    assert g(FAKE, d, P, ctypes.c_void_p(big + 65536 + 4), None) == 1
+    assert g(FAKE, 0, P, HP, None) == 1
+    c = lib.gptq_permute_columns
+    assert c(FAKE, 64, d, P, 2, FAKE, None) == 1        # inverse not 0 / 1
+    assert c(FAKE, -1, d, P, 0, FAKE, None) == 1
+    assert c(FAKE, 64, 300, P, 0, FAKE, None) == 1
+    assert c(FAKE, 64, d, None, 0, FAKE, None) == 1
+    assert c(MIS, 64, d, P, 0, FAKE, None) == 1
+    assert c(FAKE, 64, d, P, 0, ctypes.c_void_p(0x10000 + 1024), None) == 1   # partial overlap
+    assert c(FAKE, 64, d, ctypes.c_void_p(0x10000 + 256), 0, FAKE, None) == 1  # perm inside dst
+    assert c(None, 0, d, None, 0, None, None) == 0      # no rows: nothing to do
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError):
         _native._lib = None

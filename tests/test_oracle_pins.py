@@ -451,6 +451,26 @@ def test_act_order_q_in_original_order():
     assert abs(l_orig - l_perm) <= 1e-10 * l_perm
 
 
+def test_act_order_given_order():
+    """An explicit order equal to the default gives the same result; the
+    identity order is plain GPTQ on the unpermuted problem; a non-permutation
+    is refused."""
+    rng = np.random.default_rng(24)
+    d, n = 256, 1024
+    X = rng.standard_normal((n, d)) * np.exp(rng.normal(0, 1.0, d))[None, :]
+    H = oracle.hessian([X])
+    W = rng.normal(0, 0.02, (16, d))
+    a = oracle.gptq_quantize_act_order(W, H, 4, 128, -1)
+    b = oracle.gptq_quantize_act_order(W, H, 4, 128, -1, perm=oracle.act_order_perm(H))
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["Q"], b["Q"])
+    ident = oracle.gptq_quantize_act_order(W, H, 4, 128, -1, perm=np.arange(d))
+    Hd, _ = oracle.damp(H, 0.01)
+    plain = oracle.gptq_quantize(W, oracle.hinv_upper_factor(Hd), 4, 128, -1)
+    assert np.array_equal(ident["codes"], plain["codes"]) and np.array_equal(ident["Q"], plain["Q"])
+    with pytest.raises(AssertionError):
+        oracle.gptq_quantize_act_order(W, H, 4, 128, -1, perm=np.zeros(d, dtype=np.int64))
+
+
 def test_act_order_with_diagonal_h_is_rtn():
     """Uncorrelated inputs (diagonal H): no compensation crosses columns, so
     act-order GPTQ is RTN on the per-row grid in any order."""
