@@ -37,6 +37,9 @@ notes):
       is the same; groups are formed in processing order; codes / scales /
       zeros stay in processing order together with the permutation, and Q is
       returned in the original column order.
+  R15 the inference product y = x W^T is computed from the stored form
+      (packed codes, fp16 scales / zeros, the permutation) with W^ rebuilt
+      exactly as s (c - z).
 
 Parity status: every function here is pinned by a test in
 tests/test_oracle_pins.py (closed forms, brute force, invariants, the page's
@@ -52,6 +55,7 @@ __all__ = [
     "grid_params", "quant_codes", "dequant", "gptq_quantize", "rtn_quantize",
     "pack_codes", "unpack_codes", "layer_loss_direct", "layer_loss_hessian",
     "obq_fixed_order_row", "least_squares_refit", "act_order_perm", "gptq_quantize_act_order",
+    "dequant_gemv",
 ]
 
 FP16_MIN_NORMAL = 2.0 ** -14
@@ -304,6 +308,31 @@ def unpack_codes(words, bits: int, d_in: int) -> np.ndarray:
             bit = (words[:, pos // 32] >> np.uint64(pos % 32)) & np.uint64(1)
             codes[:, k] |= (bit.astype(np.int64) << b)
     return codes
+
+
+# ---------------------------------------------------------------------------
+# Inference consumer (reading R15): the layer's output computed from the
+# stored form.  [wiki] "결과": a dedicated kernel unpacks the weights as it
+# needs them and cuts the per-token latency; [blog] section 5: production
+# implementations store INT4/INT8 codes and dequantize them during inference.
+# ---------------------------------------------------------------------------
+def dequant_gemv(words, scales, zeros, bits: int, groupsize: int, x, perm=None) -> np.ndarray:
+    """y[m][r] = sum_k s[r][g(k)] (c[r][k] - z[r][g(k)]) x[m][perm[k]] in fp64.
+
+    words [d_out, d_in*bits/32] packed codes (R7), scales / zeros [d_out,
+    n_groups] fp16 values, x [m, d_in] (the layer input, one row per token).
+    Code column k belongs to input column perm[k] (act-order, R14); perm=None
+    is the natural order.  g(k) = k // groupsize (0 for a per-row grid)."""
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    d_in = x.shape[1]
+    c = unpack_codes(words, bits, d_in)
+    g = d_in if groupsize <= 0 else groupsize
+    gi = np.arange(d_in) // g
+    s = np.asarray(scales, dtype=np.float64)[:, gi]
+    z = np.asarray(zeros, dtype=np.float64)[:, gi]
+    Q = dequant(c, s, z)                    # [d_out, d_in], processing order
+    xp = x if perm is None else x[:, np.asarray(perm, dtype=np.int64)]
+    return xp @ Q.T
 
 
 # ---------------------------------------------------------------------------

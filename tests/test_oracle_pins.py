@@ -471,6 +471,49 @@ def test_act_order_given_order():
         oracle.gptq_quantize_act_order(W, H, 4, 128, -1, perm=np.zeros(d, dtype=np.int64))
 
 
+def _golden_gemv(golden_dir):
+    g = {}
+    for line in open(os.path.join(golden_dir, "dequant_gemv_hand.txt")):
+        if line.strip() and not line.startswith("#"):
+            k, *v = line.split()
+            g[k] = v
+    words = np.array([[int(g["word0"][0], 16)], [int(g["word1"][0], 16)]], dtype=np.uint32)
+    s = np.array([[float(v) for v in g["s0"]], [float(v) for v in g["s1"]]])
+    z = np.array([[float(v) for v in g["z0"]], [float(v) for v in g["z1"]]])
+    x = np.array([[float(v) for v in g["x"]]])
+    perm = np.array([int(v) for v in g["perm"]])
+    return words, s, z, x, perm, [float(v) for v in g["y"]], [float(v) for v in g["y_perm"]]
+
+
+def test_dequant_gemv_hand_example(golden_dir):
+    words, s, z, x, perm, y, y_perm = _golden_gemv(golden_dir)
+    assert oracle.dequant_gemv(words, s, z, 4, 4, x)[0].tolist() == y
+    assert oracle.dequant_gemv(words, s, z, 4, 4, x, perm)[0].tolist() == y_perm
+
+
+@pytest.mark.parametrize("act", [False, True])
+def test_dequant_gemv_equals_layer_output_of_q(act):
+    """The stored form (packed codes, fp16 grid, permutation) reproduces the
+    layer output of the quantizer's own Q, for several tokens at once."""
+    rng = np.random.default_rng(31)
+    d, n = 256, 1024
+    X = rng.standard_normal((n, d)) * np.exp(rng.normal(0, 1.0, d))[None, :]
+    H = oracle.hessian([X])
+    W = rng.normal(0, 0.02, (40, d))
+    if act:
+        out = oracle.gptq_quantize_act_order(W, H, 4, 128, 128)
+        perm = out["perm"]
+    else:
+        Hd, _ = oracle.damp(H, 0.01)
+        out = oracle.gptq_quantize(W, oracle.hinv_upper_factor(Hd), 4, 128, 128)
+        perm = None
+    words = oracle.pack_codes(out["codes"], 4)
+    xt = rng.standard_normal((5, d))
+    y = oracle.dequant_gemv(words, out["scales"], out["zeros"], 4, 128, xt, perm)
+    ref = xt @ out["Q"].T
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
 def test_act_order_with_diagonal_h_is_rtn():
     """Uncorrelated inputs (diagonal H): no compensation crosses columns, so
     act-order GPTQ is RTN on the per-row grid in any order."""
@@ -531,3 +574,35 @@ def test_planted_act_order_mistakes_are_caught(mistake, monkeypatch, golden_dir)
 def _check_golden_with(perm_fn, golden_dir):
     diag, perm = _golden_act_order(golden_dir)
     assert np.array_equal(perm_fn(np.diag(diag)), perm)
+
+
+def _mutant_gemv(mistake):
+    def f(words, scales, zeros, bits, groupsize, x, perm=None):
+        x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+        d_in = x.shape[1]
+        c = oracle.unpack_codes(words, bits, d_in)
+        g = d_in if groupsize <= 0 else groupsize
+        ng = np.asarray(scales).shape[1]
+        gi = np.arange(d_in) % ng if mistake == "group_index" else np.arange(d_in) // g
+        s = np.asarray(scales, dtype=np.float64)[:, gi]
+        z = np.asarray(zeros, dtype=np.float64)[:, gi]
+        Q = s * (c + z) if mistake == "zero_sign" else s * (c - z)
+        if perm is not None:
+            p = np.argsort(perm) if mistake == "inverse_perm" else np.asarray(perm)
+            x = x[:, p]
+        return x @ Q.T
+    return f
+
+
+@pytest.mark.parametrize("mistake", ["inverse_perm", "zero_sign", "group_index"])
+def test_planted_gemv_mistakes_are_caught(mistake, monkeypatch, golden_dir):
+    """Each plausible slip in the stored-form product fails a pin above."""
+    monkeypatch.setattr(oracle, "dequant_gemv", _mutant_gemv(mistake))
+    caught = 0
+    for pin in (lambda: test_dequant_gemv_hand_example(golden_dir),
+                lambda: test_dequant_gemv_equals_layer_output_of_q(True)):
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught >= 1
