@@ -186,8 +186,9 @@ def run_reference(args):
 # --------------------------------------------------------------------------- profiling case
 def run_profile_case():
     """The per-launch shape of the benchmark (one 16384 x 4096 bf16 batch, the
-    same 4096 x 4096 layer) run three times end to end, for ncu captures of
-    single kernels (a few hundred MB on the device)."""
+    same 4096 x 4096 layer) run three times end to end, once more with
+    act-order, then the stored-form product on the largest layer shape, for
+    ncu captures of single kernels (a few hundred MB on the device)."""
     import torch
 
     from post_weight_quantization_05_b200 import api, build_lib, synth
@@ -201,6 +202,26 @@ def run_profile_case():
         lq.begin(w)
         lq.add_batch(x)
         lq.finish()
+    api.get_status()
+    # then the same layer once with act-order (the permutation kernels) ...
+    la = api.LayerQuantizer(p.d_out, p.d_in, p.bits, p.groupsize, p.blocksize, p.percdamp, act_order=True)
+    la.begin(w)
+    la.add_batch(x)
+    la.finish()
+    api.get_status()
+    # ... and the inference product on the 8192 x 28672 g128 stored form
+    # (synthetic codes, 125 MB), m = 1 then m = 8, two launches each
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1234)
+    d_out, d_in = 8192, 28672
+    codes = torch.randint(-2 ** 31, 2 ** 31 - 1, (d_out, d_in // 8), dtype=torch.int32, device="cuda", generator=gen)
+    scales = (torch.rand((d_out, d_in // 128), device="cuda", generator=gen) * 3e-3 + 1e-4).half()
+    zeros = torch.randint(0, 16, (d_out, d_in // 128), device="cuda", generator=gen).half()
+    for m in (1, 8):
+        xt = torch.randn((m, d_in), device="cuda", generator=gen).bfloat16()
+        y = torch.empty((m, d_out), dtype=torch.float32, device="cuda")
+        for _ in range(2):
+            api.dequant_gemv(codes, scales, zeros, 4, 128, xt, y)
     api.get_status()
     print("profile case done")
     return 0
@@ -216,6 +237,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-act-order", action="store_true")
+    ap.add_argument("--no-gemv", action="store_true")
     ap.add_argument("--profile-case", action="store_true",
                     help="small case for ncu captures: one 16384-row batch of the same layer, 3 passes, no timing")
     args = ap.parse_args()
@@ -337,6 +359,11 @@ def main():
     if not args.no_act_order:
         act = act_order_timing(p, X_dev, W_dev, dev, stream, flush, args, api)
 
+    # ---- the inference product from the stored form
+    gemv = None
+    if not args.no_gemv:
+        gemv = gemv_timing(dev, stream, flush, args, api, peaks()[2])
+
     # ---- end to end through the public API with host buffers (rank 0 .. all ranks)
     e2e = None
     if not args.no_e2e:
@@ -357,7 +384,7 @@ def main():
                            "blocksize": p.blocksize, "parallelism": f"replicas x{world}",
                            "l2": "flushed before every step (256 MiB write, outside the step events)"},
                 "ms_per_layer": ms_per_step, "stages_ms": stages, "roofline": roof, "cpu_baseline": cpu,
-                "e2e": e2e, "gpu_launches": launches, "clocks": clk, "act_order": act,
+                "e2e": e2e, "gpu_launches": launches, "clocks": clk, "act_order": act, "dequant_gemv": gemv,
                 "input_generation_s": gen_s}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -403,6 +430,52 @@ def act_order_timing(p, X_dev, W_dev, dev, stream, flush, args, api):
             "order_and_permute_ms": perm_ms,
             "stage": "act_order_perm + permute_hessian + permute_columns(W), device events",
             "steps": args.steps, "warmup": args.warmup}
+
+
+def gemv_timing(dev, stream, flush, args, api, hbm_gbs):
+    """The inference product from the stored form (W4A16) on the largest layer
+    shape, 8192 x 28672 with groups of 128: synthetic uniform codes, fp16
+    scales and zeros, m = 1 and 8 bf16 tokens.  Device events per launch, L2
+    flushed before each; the bf16 product of the same shape through
+    torch.matmul (cuBLAS) is timed the same way for context."""
+    import torch
+    d_out, d_in, g = 8192, 28672, 128
+    ng = d_in // g
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    codes = torch.randint(-2 ** 31, 2 ** 31 - 1, (d_out, d_in // 8), dtype=torch.int32, device=dev, generator=gen)
+    scales = (torch.rand((d_out, ng), device=dev, generator=gen) * 3e-3 + 1e-4).half()
+    zeros = torch.randint(0, 16, (d_out, ng), device=dev, generator=gen).half()
+    w16 = torch.randn((d_out, d_in), device=dev, generator=gen).bfloat16()
+    out = {"workload": f"{d_out}x{d_in} 4-bit g{g}, synthetic codes", "peak_gbs": hbm_gbs}
+    n_iter = max(args.steps, 10)
+
+    def timed(fn):
+        ts = []
+        for i in range(args.warmup + n_iter):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            if i >= args.warmup:
+                ts.append((a, b))
+        torch.cuda.synchronize(dev)
+        return statistics.mean(x.elapsed_time(y) for x, y in ts) * 1e3      # us
+
+    for m in (1, 8):
+        x = torch.randn((m, d_in), device=dev, generator=gen).bfloat16()
+        y = torch.empty((m, d_out), dtype=torch.float32, device=dev)
+        l0 = api.launch_count()
+        us = timed(lambda: api.dequant_gemv(codes, scales, zeros, 4, g, x, y))
+        launches = (api.launch_count() - l0) // (args.warmup + n_iter)
+        api.get_status(stream)
+        ref_us = timed(lambda: torch.matmul(x, w16.t()))
+        nbytes = d_out * d_in // 2 + 2 * d_out * ng * 2 + m * d_in * 2 + m * d_out * 4
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[f"m{m}"] = {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs,
+                        "launches": launches, "bf16_matmul_us": ref_us, "speedup_vs_bf16": ref_us / us}
+    return out
 
 
 def end_to_end(p, xs_host, w_bits, lq, dev, args, world, dist):

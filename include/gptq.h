@@ -268,6 +268,39 @@ int gptq_permute_columns(const float* src, int64_t rows, int64_t cols, const int
                          float* dst, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Inference -- the layer output computed from the stored form (W4A16).
+ * Source: itwiki "GPTQ", "결과" (a dedicated kernel unpacks the weights as
+ * it needs them at inference and cuts the per-token latency against FP16);
+ * blog "GPTQ를 밑바닥부터 구현하며 배운 것들", section 5 (production
+ * implementations store INT4 codes and dequantize them during inference).
+ *
+ *   y[t][r] = sum_k s[r][g(k)] * (c[r][k] - z[r][g(k)]) * x[t][perm[k]]
+ *
+ * for tokens t < m and rows r < d_out; g(k) = k / groupsize (0 for a per-row
+ * grid); c, s, z as gptq_quantize_layer writes them (processing order).
+ *   codes   device uint32 [d_out, d_in * bits / 32], 16-byte aligned.
+ *   scales, zeros  device fp16 bit patterns [d_out, n_groups].
+ *   bits    4 (2, 3 and 8 return GPTQ_ERR_UNSUPPORTED in this build).
+ *   groupsize  -1 or a multiple of 128 dividing d_in.
+ *   perm    device int32 [d_in] (act-order: code column k multiplies input
+ *           column perm[k]) or NULL (natural order).  An entry outside
+ *           [0, d_in) is recorded as GPTQ_ERR_INVALID_ARG in the status word
+ *           and its input is taken as NaN.
+ *   x       device bf16 bit patterns [m, d_in] row-major, 16-byte aligned;
+ *           0 <= m <= 8 (m = 0: nothing to do).
+ *   y       device fp32 [m, d_out] row-major output.
+ *   ws      device workspace of gptq_dequant_gemv_workspace_size(m, d_in,
+ *           perm != NULL) bytes (x gathered into processing order); 0 bytes
+ *           and may be NULL without perm.
+ * Every product c * x is exact (both are bf16 values, accumulated in fp32);
+ * each 128-column block is scaled and offset in fp32: s (sum c x - z sum x).
+ * ---------------------------------------------------------------------- */
+size_t gptq_dequant_gemv_workspace_size(int64_t m, int64_t d_in, int with_perm);
+int gptq_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
+                      int64_t d_in, int bits, int groupsize, const int32_t* perm, const uint16_t* x, int64_t m,
+                      float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Helpers on the same stream (not steps of the method).
  * ---------------------------------------------------------------------- */
 /* dst[i] = (float) src[i] for bf16 bit patterns src (a bf16 layer's fp32

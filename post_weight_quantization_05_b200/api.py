@@ -202,6 +202,33 @@ def permute_columns(src: torch.Tensor, perm: torch.Tensor, dst: torch.Tensor | N
                                        _stream(stream)), "gptq_permute_columns")
 
 
+def dequant_gemv_workspace_size(m: int, d_in: int, with_perm: bool) -> int:
+    return _lib().gptq_dequant_gemv_workspace_size(m, d_in, 1 if with_perm else 0)
+
+
+def dequant_gemv(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, bits: int, groupsize: int,
+                 x: torch.Tensor, y: torch.Tensor, perm: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                 stream=None):
+    """y[t] = x[t] W^T with W^ rebuilt from the stored form (codes in
+    processing order; perm maps code column k to input column perm[k])."""
+    d_out = codes.shape[0]
+    m, d_in = x.shape
+    ng = n_groups(d_in, groupsize)
+    _need(codes, torch.int32, (d_out, d_in * bits // 32), "codes")
+    _need(scales, torch.float16, (d_out, ng), "scales")
+    _need(zeros, torch.float16, (d_out, ng), "zeros")
+    _need(x, torch.bfloat16, (m, d_in), "x")
+    _need(y, torch.float32, (m, d_out), "y")
+    if perm is not None:
+        _need(perm, torch.int32, (d_in,), "perm")
+        if ws is None:
+            ws = workspace(dequant_gemv_workspace_size(m, d_in, True), x.device)
+    code = _lib().gptq_dequant_gemv(_ptr(codes), _ptr(scales), _ptr(zeros), d_out, d_in, bits, groupsize,
+                                    _ptr(perm), _ptr(x), m, _ptr(y), _ptr(ws),
+                                    0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check(code, "gptq_dequant_gemv")
+
+
 def widen_bf16(src: torch.Tensor, dst: torch.Tensor, stream=None):
     if src.dtype != torch.bfloat16 or dst.dtype != torch.float32 or src.numel() != dst.numel():
         raise ValueError("widen_bf16: bf16 -> fp32 of equal size")

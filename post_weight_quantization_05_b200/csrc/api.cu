@@ -238,6 +238,30 @@ int gptq_permute_columns(const float* src, int64_t rows, int64_t cols, const int
     return launch_permute_columns(src, rows, cols, perm, inverse != 0, dst, static_cast<cudaStream_t>(stream), st);
 }
 
+size_t gptq_dequant_gemv_workspace_size(int64_t m, int64_t d_in, int with_perm) {
+    if (m <= 0 || m > 8 || !valid_d_in(d_in)) return 0;
+    return gemv_workspace_bytes(m, d_in, with_perm != 0);
+}
+
+int gptq_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
+                      int64_t d_in, int bits, int groupsize, const int32_t* perm, const uint16_t* x, int64_t m,
+                      float* y, void* ws, size_t ws_bytes, void* stream) {
+    if (d_out <= 0 || d_out > (int64_t(1) << 24) || !valid_d_in(d_in)) return GPTQ_ERR_INVALID_ARG;
+    if (!valid_bits(bits) || !valid_group(groupsize, d_in) || m < 0 || m > 8) return GPTQ_ERR_INVALID_ARG;
+    if (bits != 4) return GPTQ_ERR_UNSUPPORTED;
+    if (m == 0) return GPTQ_OK;
+    if (!codes || !scales || !zeros || !x || !y) return GPTQ_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(x) || (reinterpret_cast<uintptr_t>(y) & 3u) ||
+        (reinterpret_cast<uintptr_t>(scales) & 1u) || (reinterpret_cast<uintptr_t>(zeros) & 1u) ||
+        (perm && (reinterpret_cast<uintptr_t>(perm) & 3u)))
+        return GPTQ_ERR_INVALID_ARG;
+    if (perm && (!ws || !aligned16(ws) || ws_bytes < gemv_workspace_bytes(m, d_in, true))) return GPTQ_ERR_INVALID_ARG;
+    DevStatus* st = nullptr;
+    if (status_ptr(&st)) return GPTQ_ERR_CUDA;
+    return launch_dequant_gemv(codes, scales, zeros, d_out, d_in, groupsize, perm, x, m, y, ws,
+                               static_cast<cudaStream_t>(stream), st);
+}
+
 int gptq_widen_bf16(const uint16_t* src, float* dst, int64_t count, void* stream) {
     if (count < 0) return GPTQ_ERR_INVALID_ARG;
     if (count == 0) return GPTQ_OK;

@@ -64,6 +64,13 @@ int launch_rtn(const float* W, int64_t d_out, int64_t d_in, int bits, int groups
                uint16_t* scales, uint16_t* zeros, float* Q, cudaStream_t stream, DevStatus* st);
 int launch_widen_bf16(const uint16_t* src, float* dst, int64_t count, cudaStream_t stream);
 
+// gemv.cu: y = x W^T from the stored form (4-bit codes), m <= 8 tokens; with
+// perm, x is first gathered into ws (gemv_workspace_bytes).
+size_t gemv_workspace_bytes(int64_t m, int64_t d_in, bool with_perm);
+int launch_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
+                        int64_t d_in, int groupsize, const int32_t* perm, const uint16_t* x, int64_t m, float* y,
+                        void* ws, cudaStream_t stream, DevStatus* st);
+
 // permute.cu (act-order): the processing order from diag(H), the permuted
 // Hessian, and the column permutation of a row-major matrix (in place allowed).
 int launch_act_order_perm(const float* H, int64_t d, int32_t* perm, cudaStream_t stream);

@@ -177,6 +177,31 @@ def test_act_order_entries_reject_bad_arguments(lib):
     assert c(None, 0, d, None, 0, None, None) == 0      # no rows: nothing to do
 
 
+def test_dequant_gemv_rejects_bad_arguments(lib):
+    assert lib.gptq_dequant_gemv_workspace_size(1, 4096, 1) == 8192
+    assert lib.gptq_dequant_gemv_workspace_size(3, 640, 1) == (3 * 640 * 2 + 255) // 256 * 256
+    assert lib.gptq_dequant_gemv_workspace_size(1, 4096, 0) == 0
+    assert lib.gptq_dequant_gemv_workspace_size(9, 4096, 1) == 0
+    f = lib.gptq_dequant_gemv
+    ok = dict(codes=FAKE, scales=FAKE, zeros=FAKE, d_out=64, d_in=512, bits=4, g=128, perm=None, x=FAKE, m=2,
+              y=FAKE, ws=None, ws_bytes=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["codes"], a["scales"], a["zeros"], a["d_out"], a["d_in"], a["bits"], a["g"], a["perm"], a["x"],
+                 a["m"], a["y"], a["ws"], a["ws_bytes"], None)
+    assert call(bits=3) == 2 and call(bits=8) == 2 and call(bits=2) == 2      # valid, not in this build
+    assert call(bits=5) == 1
+    assert call(m=9) == 1 and call(m=-1) == 1
+    assert call(m=0, codes=None, x=None, y=None) == 0                       # nothing to do
+    assert call(d_in=300) == 1 and call(g=100) == 1 and call(d_out=0) == 1
+    assert call(codes=MIS) == 1 and call(x=MIS) == 1 and call(y=ctypes.c_void_p(0x10002)) == 1
+    assert call(scales=ctypes.c_void_p(0x10001)) == 1 and call(codes=None) == 1
+    assert call(perm=FAKE) == 1                                              # perm needs a workspace
+    assert call(perm=FAKE, ws=FAKE, ws_bytes=100) == 1
+    assert call(perm=ctypes.c_void_p(0x10002), ws=FAKE, ws_bytes=4096) == 1
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError):
         _native._lib = None
