@@ -435,9 +435,11 @@ def act_order_timing(p, X_dev, W_dev, dev, stream, flush, args, api):
 def gemv_timing(dev, stream, flush, args, api, hbm_gbs):
     """The inference product from the stored form (W4A16) on the largest layer
     shape, 8192 x 28672 with groups of 128: synthetic uniform codes, fp16
-    scales and zeros, m = 1 and 8 bf16 tokens.  Device events per launch, L2
-    flushed before each; the bf16 product of the same shape through
-    torch.matmul (cuBLAS) is timed the same way for context."""
+    scales and zeros, m = 1 and 8 bf16 tokens.  The call (its two kernels) is
+    captured once in a CUDA graph and replayed, so that host-side argument
+    handling stays out of the device events; L2 is flushed before each replay.
+    The bf16 product of the same shape through torch.matmul (cuBLAS) is timed
+    the same way for context."""
     import torch
     d_out, d_in, g = 8192, 28672, 128
     ng = d_in // g
@@ -451,24 +453,35 @@ def gemv_timing(dev, stream, flush, args, api, hbm_gbs):
     n_iter = max(args.steps, 10)
 
     def timed(fn):
+        fn()                                     # first call: one-time setup outside the capture
+        torch.cuda.synchronize(dev)
+        side = torch.cuda.Stream(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                fn()
+        torch.cuda.synchronize(dev)
         ts = []
         for i in range(args.warmup + n_iter):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            fn()
+            graph.replay()
             b.record(stream)
             if i >= args.warmup:
                 ts.append((a, b))
         torch.cuda.synchronize(dev)
+        del graph
         return statistics.mean(x.elapsed_time(y) for x, y in ts) * 1e3      # us
 
     for m in (1, 8):
         x = torch.randn((m, d_in), device=dev, generator=gen).bfloat16()
         y = torch.empty((m, d_out), dtype=torch.float32, device=dev)
+        ws = api.workspace(api.dequant_gemv_workspace_size(m, d_in, False), dev)
         l0 = api.launch_count()
-        us = timed(lambda: api.dequant_gemv(codes, scales, zeros, 4, g, x, y))
-        launches = (api.launch_count() - l0) // (args.warmup + n_iter)
+        api.dequant_gemv(codes, scales, zeros, 4, g, x, y, ws=ws)
+        launches = api.launch_count() - l0
+        us = timed(lambda: api.dequant_gemv(codes, scales, zeros, 4, g, x, y, ws=ws))
         api.get_status(stream)
         ref_us = timed(lambda: torch.matmul(x, w16.t()))
         nbytes = d_out * d_in // 2 + 2 * d_out * ng * 2 + m * d_in * 2 + m * d_out * 4

@@ -290,10 +290,15 @@ int gptq_permute_columns(const float* src, int64_t rows, int64_t cols, const int
  *           0 <= m <= 8 (m = 0: nothing to do).
  *   y       device fp32 [m, d_out] row-major output.
  *   ws      device workspace of gptq_dequant_gemv_workspace_size(m, d_in,
- *           perm != NULL) bytes (x gathered into processing order); 0 bytes
- *           and may be NULL without perm.
- * Every product c * x is exact (both are bf16 values, accumulated in fp32);
- * each 128-column block is scaled and offset in fp32: s (sum c x - z sum x).
+ *           perm != NULL) bytes, 16-byte aligned: x in processing order as
+ *           fp16, scaled by a power of two per 128-column block, with each
+ *           block's sum and scale.
+ * Every product c * x is exact: each 128-column block of x is scaled by 2^-e
+ * so that its largest magnitude lies in [2^14, 2^15), which keeps every bf16
+ * value down to 2^-28 of that maximum exact in fp16 (smaller ones round to
+ * fp16's subnormals); codes and scaled x meet on the tensor cores with fp32
+ * accumulation; each block is scaled and offset in fp32,
+ * 2^e s (sum c x - z sum x).
  * ---------------------------------------------------------------------- */
 size_t gptq_dequant_gemv_workspace_size(int64_t m, int64_t d_in, int with_perm);
 int gptq_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,

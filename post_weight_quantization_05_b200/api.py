@@ -221,8 +221,8 @@ def dequant_gemv(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
     _need(y, torch.float32, (m, d_out), "y")
     if perm is not None:
         _need(perm, torch.int32, (d_in,), "perm")
-        if ws is None:
-            ws = workspace(dequant_gemv_workspace_size(m, d_in, True), x.device)
+    if ws is None and m > 0:
+        ws = workspace(dequant_gemv_workspace_size(m, d_in, perm is not None), x.device)
     code = _lib().gptq_dequant_gemv(_ptr(codes), _ptr(scales), _ptr(zeros), d_out, d_in, bits, groupsize,
                                     _ptr(perm), _ptr(x), m, _ptr(y), _ptr(ws),
                                     0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))

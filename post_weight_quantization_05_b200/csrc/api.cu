@@ -255,11 +255,12 @@ int gptq_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint1
         (reinterpret_cast<uintptr_t>(scales) & 1u) || (reinterpret_cast<uintptr_t>(zeros) & 1u) ||
         (perm && (reinterpret_cast<uintptr_t>(perm) & 3u)))
         return GPTQ_ERR_INVALID_ARG;
-    if (perm && (!ws || !aligned16(ws) || ws_bytes < gemv_workspace_bytes(m, d_in, true))) return GPTQ_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws) || ws_bytes < gemv_workspace_bytes(m, d_in, perm != nullptr)) return GPTQ_ERR_INVALID_ARG;
     DevStatus* st = nullptr;
-    if (status_ptr(&st)) return GPTQ_ERR_CUDA;
+    PFN_encodeTiled enc = nullptr;
+    if (status_ptr(&st) || encode_fn(&enc)) return GPTQ_ERR_CUDA;
     return launch_dequant_gemv(codes, scales, zeros, d_out, d_in, groupsize, perm, x, m, y, ws,
-                               static_cast<cudaStream_t>(stream), st);
+                               static_cast<cudaStream_t>(stream), st, enc);
 }
 
 int gptq_widen_bf16(const uint16_t* src, float* dst, int64_t count, void* stream) {

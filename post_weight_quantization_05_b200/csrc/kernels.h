@@ -69,7 +69,7 @@ int launch_widen_bf16(const uint16_t* src, float* dst, int64_t count, cudaStream
 size_t gemv_workspace_bytes(int64_t m, int64_t d_in, bool with_perm);
 int launch_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
                         int64_t d_in, int groupsize, const int32_t* perm, const uint16_t* x, int64_t m, float* y,
-                        void* ws, cudaStream_t stream, DevStatus* st);
+                        void* ws, cudaStream_t stream, DevStatus* st, PFN_encodeTiled encode);
 
 // permute.cu (act-order): the processing order from diag(H), the permuted
 // Hessian, and the column permutation of a row-major matrix (in place allowed).

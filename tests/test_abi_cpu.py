@@ -178,13 +178,13 @@ def test_act_order_entries_reject_bad_arguments(lib):
 
 
 def test_dequant_gemv_rejects_bad_arguments(lib):
-    assert lib.gptq_dequant_gemv_workspace_size(1, 4096, 1) == 8192
-    assert lib.gptq_dequant_gemv_workspace_size(3, 640, 1) == (3 * 640 * 2 + 255) // 256 * 256
-    assert lib.gptq_dequant_gemv_workspace_size(1, 4096, 0) == 0
+    r256 = lambda b: (b + 255) // 256 * 256  # noqa: E731
+    assert lib.gptq_dequant_gemv_workspace_size(1, 4096, 1) == r256(8192) + r256(32 * 8)
+    assert lib.gptq_dequant_gemv_workspace_size(3, 640, 0) == r256(3 * 640 * 2) + r256(3 * 5 * 8)
     assert lib.gptq_dequant_gemv_workspace_size(9, 4096, 1) == 0
     f = lib.gptq_dequant_gemv
     ok = dict(codes=FAKE, scales=FAKE, zeros=FAKE, d_out=64, d_in=512, bits=4, g=128, perm=None, x=FAKE, m=2,
-              y=FAKE, ws=None, ws_bytes=0)
+              y=FAKE, ws=FAKE, ws_bytes=1 << 20)
 
     def call(**kw):
         a = dict(ok, **kw)
@@ -197,8 +197,7 @@ def test_dequant_gemv_rejects_bad_arguments(lib):
     assert call(d_in=300) == 1 and call(g=100) == 1 and call(d_out=0) == 1
     assert call(codes=MIS) == 1 and call(x=MIS) == 1 and call(y=ctypes.c_void_p(0x10002)) == 1
     assert call(scales=ctypes.c_void_p(0x10001)) == 1 and call(codes=None) == 1
-    assert call(perm=FAKE) == 1                                              # perm needs a workspace
-    assert call(perm=FAKE, ws=FAKE, ws_bytes=100) == 1
+    assert call(ws=None) == 1 and call(ws_bytes=100) == 1 and call(ws=MIS) == 1   # the workspace is required
     assert call(perm=ctypes.c_void_p(0x10002), ws=FAKE, ws_bytes=4096) == 1
 
 
