@@ -57,6 +57,11 @@ struct Args {
     const float2* xaux;       // [m][d_in / 128]: {sum of the block's fp16 x, 2^e}
     float* y;                 // [m, d_out]
     int d_out, d_in, m, group, n_groups;
+    // fp16x2 constants of the code conversion (1024, -1024, 1/16, -64), passed
+    // as launch arguments: an instruction can take one of them straight from
+    // the constant bank next to an immediate mask, where two immediates would
+    // cost an extra move per use
+    uint32_t k_mag, k_sub, k_s16, k_sub64;
     uint32_t kpg_magic;       // ceil(2^32 / (group / 128)), 0 when group = 128: the group of column block kb
     int side_off;             // byte offset of the staged scales / zeros / block data in shared memory
 };
@@ -76,6 +81,12 @@ __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
 // ORed into the mantissa of 1024.0 and 1024 subtracted; the high nibble gives
 // 1024 + 16 c, times 1/16, minus 64.  Both exact; one LOP and one packed FMA
 // per two codes, the pairs (p, p + 4) of a word sharing a register.
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -98,7 +109,7 @@ struct Tile {
 // 4 j + 2 h + 1: k slots 2q, 2q+1 <-> nibbles (2h, 2h+4), slots 8+2q, 9+2q
 // <-> nibbles (2h+1, 2h+5) of word j.  Then y += 2^e s (acc - z sum x).
 __device__ __forceinline__ void compute_tile(const Tile& t, const float (&sv)[4], const float (&zv)[4], float2 xa0,
-                                             float2 xa1, float (&yacc)[2][4]) {
+                                             float2 xa1, float (&yacc)[2][4], const Args& A) {
     const uint32_t X[16] = {t.x[0].x, t.x[0].y, t.x[0].z, t.x[0].w, t.x[1].x, t.x[1].y, t.x[1].z, t.x[1].w,
                             t.x[2].x, t.x[2].y, t.x[2].z, t.x[2].w, t.x[3].x, t.x[3].y, t.x[3].z, t.x[3].w};
     const uint32_t C[4][4] = {{t.c[0].x, t.c[0].y, t.c[0].z, t.c[0].w}, {t.c[1].x, t.c[1].y, t.c[1].z, t.c[1].w},
@@ -114,10 +125,10 @@ __device__ __forceinline__ void compute_tile(const Tile& t, const float (&sv)[4]
                 // rows g + 16 r (A rows 0..7) and g + 16 r + 8 (A rows 8..15)
                 const uint32_t wl = h ? (C[2 * r][j] >> 8) : C[2 * r][j];
                 const uint32_t wh = h ? (C[2 * r + 1][j] >> 8) : C[2 * r + 1][j];
-                const uint32_t a0 = hfma2((wl & 0x000F000Fu) | 0x64006400u, 0x3C003C00u, 0xE400E400u);
-                const uint32_t a1 = hfma2((wh & 0x000F000Fu) | 0x64006400u, 0x3C003C00u, 0xE400E400u);
-                const uint32_t a2 = hfma2((wl & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD400D400u);
-                const uint32_t a3 = hfma2((wh & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD400D400u);
+                const uint32_t a0 = hadd2((wl & 0x000F000Fu) | A.k_mag, A.k_sub);
+                const uint32_t a1 = hadd2((wh & 0x000F000Fu) | A.k_mag, A.k_sub);
+                const uint32_t a2 = hfma2((wl & 0x00F000F0u) | A.k_mag, A.k_s16, A.k_sub64);
+                const uint32_t a3 = hfma2((wh & 0x00F000F0u) | A.k_mag, A.k_s16, A.k_sub64);
                 mma_f16(acc[r], a0, a1, a2, a3, b0, b1);
             }
         }
@@ -167,13 +178,9 @@ __global__ void __launch_bounds__(THREADS, 2) w4_kernel(const __grid_constant__ 
         // that runs just before this kernel: start them first
         for (int it = 0; it < first; ++it) issue_codes(it, it);
     }
-    pdl_wait();                 // x and its block data come from the x preparation
-    if (threadIdx.x == 0)
-        for (int it = 0; it < first; ++it) issue_x(it, it);
-    __syncthreads();
-
     // scales and zeros of the block's rows (all groups) and the tokens' block
-    // data, staged once: the loop then reads only shared memory
+    // data, staged once: the loop then reads only shared memory.  The scales
+    // and zeros do not depend on the x preparation: stage them before waiting.
     const int rows_here = min(ROWS, a.d_out - r0);
     uint16_t* sS = reinterpret_cast<uint16_t*>(ring + a.side_off);
     uint16_t* sZ = sS + ROWS * a.n_groups;
@@ -186,8 +193,11 @@ __global__ void __launch_bounds__(THREADS, 2) w4_kernel(const __grid_constant__ 
             sS[e] = row < rows_here ? a.scales[o] : uint16_t(0);
             sZ[e] = a.zeros[o];
         }
-        for (int e = threadIdx.x; e < a.m * nkb; e += THREADS) sXA[e] = a.xaux[e];
     }
+    pdl_wait();                 // x and its block data come from the x preparation
+    if (threadIdx.x == 0)
+        for (int it = 0; it < first; ++it) issue_x(it, it);
+    for (int e = threadIdx.x; e < a.m * nkb; e += THREADS) sXA[e] = a.xaux[e];
     __syncthreads();
 
     const int g = lane >> 2, q = lane & 3;
@@ -243,7 +253,7 @@ __global__ void __launch_bounds__(THREADS, 2) w4_kernel(const __grid_constant__ 
                 sv[i] = h2f(sS[(g + 8 * i) * a.n_groups + gi]);
                 zv[i] = h2f(sZ[(g + 8 * i) * a.n_groups + gi]);
             }
-            compute_tile(t, sv, zv, xa0p[kb], xa1p[kb], yacc);
+            compute_tile(t, sv, zv, xa0p[kb], xa1p[kb], yacc, a);
         }
         if (++sidx == stages) { sidx = 0; par ^= 1u; }
     }
@@ -375,6 +385,10 @@ int launch_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uin
     a.group = groupsize > 0 ? groupsize : int(d_in);
     a.n_groups = groupsize > 0 ? int(d_in / groupsize) : 1;
     // kb / kpg as umulhi(kb, ceil(2^32 / kpg)) -- exact for kb, kpg <= 256; 0 marks kpg = 1
+    a.k_mag = 0x64006400u;
+    a.k_sub = 0xE400E400u;
+    a.k_s16 = 0x2C002C00u;
+    a.k_sub64 = 0xD400D400u;
     const uint64_t kpg = uint64_t(a.group / KB);
     a.kpg_magic = kpg == 1 ? 0u : uint32_t(((uint64_t(1) << 32) + kpg - 1) / kpg);
     // shared memory: the ring, then the staged scales, zeros (u16, 32 rows x
