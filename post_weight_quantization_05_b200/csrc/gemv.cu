@@ -159,6 +159,8 @@ __global__ void __launch_bounds__(THREADS, 2) w4_kernel(const __grid_constant__ 
     const int nkb = a.d_in / KB;
     const int nst = (nkb + KPS - 1) / KPS;
     const uint32_t stage_bytes = CODE_BYTES + uint32_t(a.m) * XBLK_BYTES;
+    // a stage holds 512 contiguous bytes of each of the 32 rows (column blocks
+    // it*8 .. it*8+7), row-major: long row runs keep the HBM stream efficient
     auto issue_codes = [&](int it, int sidx) {
         mbar_arrive_expect_tx(&full[sidx], stage_bytes);
         tma_load_2d(ring + size_t(sidx) * stage_bytes, &maps.codes, it * (KPS * KB / 8), r0, &full[sidx]);
@@ -182,16 +184,43 @@ __global__ void __launch_bounds__(THREADS, 2) w4_kernel(const __grid_constant__ 
     // data, staged once: the loop then reads only shared memory.  The scales
     // and zeros do not depend on the x preparation: stage them before waiting.
     const int rows_here = min(ROWS, a.d_out - r0);
-    uint16_t* sS = reinterpret_cast<uint16_t*>(ring + a.side_off);
-    uint16_t* sZ = sS + ROWS * a.n_groups;
-    float2* sXA = reinterpret_cast<float2*>(sZ + ROWS * a.n_groups);   // 128 n_groups bytes in: 16-byte aligned
+    const int ng = a.n_groups, sstride = ng + 1;        // words per row: the 8 rows of a warp on distinct banks
+    uint32_t* sSZ = reinterpret_cast<uint32_t*>(ring + a.side_off);   // (s | z << 16) per row and group
+    float2* sXA = reinterpret_cast<float2*>(ring + a.side_off + ((size_t(ROWS) * sstride * 4 + 15) & ~size_t(15)));
     {
-        const int ng = a.n_groups;
-        for (int e = threadIdx.x; e < ROWS * ng; e += THREADS) {
-            const int row = e / ng, grp = e - row * ng;
-            const size_t o = size_t(r0 + min(row, rows_here - 1)) * ng + grp;
-            sS[e] = row < rows_here ? a.scales[o] : uint16_t(0);
-            sZ[e] = a.zeros[o];
+        uint16_t* h = reinterpret_cast<uint16_t*>(sSZ);
+        const int n_el = rows_here * ng;
+        const float inv_ng = 1.0f / float(ng);
+        auto put = [&](int idx, uint16_t v, int half) {
+            const int row = int((float(idx) + 0.5f) * inv_ng);
+            h[2 * (row * sstride + (idx - row * ng)) + half] = v;
+        };
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint16_t* src = (half ? a.zeros : a.scales) + size_t(r0) * ng;
+            int done = 0;
+            if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {   // 16-byte loads, all in flight
+                const int n16 = n_el / 8;
+                uint4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = threadIdx.x + u * THREADS;
+                    if (c < n16) v[u] = __ldg(reinterpret_cast<const uint4*>(src) + c);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = threadIdx.x + u * THREADS;
+                    if (c < n16) {
+                        const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) put(8 * c + e, uint16_t(wv[e >> 1] >> (16 * (e & 1))), half);
+                    }
+                }
+                done = 8 * min(n16, 4 * THREADS);
+            }
+            for (int idx = done + threadIdx.x; idx < n_el; idx += THREADS) put(idx, src[idx], half);
+            // rows past d_out: scale 0, zero 0
+            for (int idx = n_el + threadIdx.x; idx < ROWS * ng; idx += THREADS) put(idx, uint16_t(0), half);
         }
     }
     pdl_wait();                 // x and its block data come from the x preparation
@@ -223,9 +252,9 @@ __global__ void __launch_bounds__(THREADS, 2) w4_kernel(const __grid_constant__ 
             for (int i = 0; i < 4; ++i)
                 t.c[i] = *reinterpret_cast<const uint4*>(src + (g + 8 * i) * (KPS * KB / 2) + w * (KB / 2) + q * 16);
             if (xvalid) {
-                const uint8_t* xsrc = src + CODE_BYTES + g * XBLK_BYTES + w * (KB * 2) + q * 64;
+                const uint8_t* xsrc = src + CODE_BYTES + g * XBLK_BYTES + w * (KB * 2) + q * 16;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) t.x[i] = *reinterpret_cast<const uint4*>(xsrc + i * 16);
+                for (int i = 0; i < 4; ++i) t.x[i] = *reinterpret_cast<const uint4*>(xsrc + i * 64);
             }
         }
         // this warp's reads of the stage are ordered before the TMA that
@@ -250,8 +279,10 @@ __global__ void __launch_bounds__(THREADS, 2) w4_kernel(const __grid_constant__ 
             float sv[4], zv[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                sv[i] = h2f(sS[(g + 8 * i) * a.n_groups + gi]);
-                zv[i] = h2f(sZ[(g + 8 * i) * a.n_groups + gi]);
+                const uint32_t v = sSZ[(g + 8 * i) * sstride + gi];
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+                sv[i] = f.x;
+                zv[i] = f.y;
             }
             compute_tile(t, sv, zv, xa0p[kb], xa1p[kb], yacc, a);
         }
@@ -280,9 +311,10 @@ __global__ void __launch_bounds__(THREADS, 2) w4_kernel(const __grid_constant__ 
 
 // Warp (t, b) -- token t = blockIdx.y, column block b = blockIdx.x * 8 +
 // warp: amax = max |x[t][perm[k]]| over the block, e with amax 2^-e in
-// [2^14, 2^15) (e = 0 for amax 0 or not finite), xh[t][kk] =
-// fp16(x[t][perm[k]] 2^-e) with kk the fragment order of k (in each group of
-// 8: k = 8u + {0,4,1,5,2,6,3,7}), and xaux[t][b] = {sum of the block's fp16
+// [2^14, 2^15) (e = 0 for amax 0 or not finite), xh[t][slot] =
+// fp16(x[t][perm[k]] 2^-e) with the slot of k in the order the product's
+// lanes read (pairs (p, p + 4) of each group of 8 adjacent, the four lanes'
+// 16-byte chunks interleaved), and xaux[t][b] = {sum of the block's fp16
 // values in fp32 (fixed order), 2^e}.  An index outside [0, d_in) is reported
 // and read as NaN.
 __global__ void __launch_bounds__(PREP_THREADS)
@@ -298,9 +330,14 @@ __global__ void __launch_bounds__(PREP_THREADS)
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int kk = b * KB + 4 * lane + i;
-        const int p = kk & 7;
-        const int k = (kk & ~7) + (p >> 1) + ((p & 1) ? 4 : 0);
+        // physical slot 4 lane + i of the block holds 16-byte chunk c = slot / 8:
+        // lane q = c % 4 of the product reads chunk j = c / 4 as its j-th 16
+        // bytes, i.e. fragment position f = 32 q + 8 j + (slot % 8), which is
+        // k = 8u + {0,4,1,5,2,6,3,7}[f % 8] with u = f / 8
+        const int slot = 4 * lane + i, c = slot >> 3;
+        const int f = (c & 3) * 32 + (c >> 2) * 8 + (slot & 7);
+        const int p = f & 7;
+        const int k = b * KB + (f & ~7) + (p >> 1) + ((p & 1) ? 4 : 0);
         int src = k;
         bool ok = true;
         if (perm) {
@@ -391,11 +428,11 @@ int launch_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uin
     a.k_sub64 = 0xD400D400u;
     const uint64_t kpg = uint64_t(a.group / KB);
     a.kpg_magic = kpg == 1 ? 0u : uint32_t(((uint64_t(1) << 32) + kpg - 1) / kpg);
-    // shared memory: the ring, then the staged scales, zeros (u16, 32 rows x
-    // n_groups each) and block data (float2, m x d_in / 128); as many stages
+    // shared memory: the ring, then the staged scale / zero pairs (u32, 32 rows
+    // x (n_groups + 1)) and block data (float2, m x d_in / 128); as many stages
     // (4, 3, 2) as keep two blocks on an SM
     const size_t stage_bytes = CODE_BYTES + size_t(m) * XBLK_BYTES;
-    const size_t side = ((size_t(ROWS) * a.n_groups * 2 * 2 + 15) & ~size_t(15)) + size_t(m) * (d_in / KB) * 8;
+    const size_t side = ((size_t(ROWS) * (a.n_groups + 1) * 4 + 15) & ~size_t(15)) + size_t(m) * (d_in / KB) * 8;
     int stages = 4;
     while (stages > 2 && size_t(stages) * stage_bytes + side > size_t(110) * 1024) --stages;
     const size_t ring_bytes = std::max(size_t(stages) * stage_bytes, size_t(WARPS) * ROWS * (MAX_TOKENS + 1) * 4);
