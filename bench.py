@@ -353,6 +353,7 @@ def main():
 
     stages = {"widen_W+zero_H": statistics.mean(begin_ms), "hessian_16_batches": statistics.mean(h_ms),
               "prepare_hinv": statistics.mean(prep_ms), "quantize_layer": statistics.mean(quant_ms)}
+    stage_roof = stage_rooflines(p, stages, burst, sustained, hbm)
 
     # ---- the same layer with act-order (columns by descending diag(H))
     act = None
@@ -383,7 +384,8 @@ def main():
                            "batches": p.n_batches, "bits": p.bits, "groupsize": p.groupsize,
                            "blocksize": p.blocksize, "parallelism": f"replicas x{world}",
                            "l2": "flushed before every step (256 MiB write, outside the step events)"},
-                "ms_per_layer": ms_per_step, "stages_ms": stages, "roofline": roof, "cpu_baseline": cpu,
+                "ms_per_layer": ms_per_step, "stages_ms": stages, "stage_roofline": stage_roof, "roofline": roof,
+                "cpu_baseline": cpu,
                 "e2e": e2e, "gpu_launches": launches, "clocks": clk, "act_order": act, "dequant_gemv": gemv,
                 "input_generation_s": gen_s}
         print(json.dumps(line), flush=True)
@@ -391,6 +393,40 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def stage_rooflines(p, stages, burst, sustained, hbm):
+    """Each stage's algorithmic work over its own live event time, against
+    the measured peak of what bounds it.  The factorization and the sweep are
+    chains of dependent 128-column steps: their fractions say how far the
+    chain's latency keeps them from the hardware's rate, not how fast a
+    single kernel runs."""
+    d_out, d_in, B = p.d_out, p.d_in, p.blocksize
+    nb = d_in // B
+    h_flops = p.n * d_in * (d_in + 1)                        # upper triangle incl. diagonal, 2 per MAC
+    h_tf = h_flops / (stages["hessian_16_batches"] / 1e3) / 1e12
+    # factorization: Cholesky (d^3/3) + triangular inverse (d^3/3) + U from the inverse (d^3/3), 2 per MAC
+    f_flops = 2.0 * d_in ** 3
+    f_tf = f_flops / (stages["prepare_hinv"] / 1e3) / 1e12
+    # sweep: each block reads its W columns and U diagonal block, writes E (tf32 hi / lo) and the codes;
+    # trailing products: sum over blocks of 2 d_out (d_in - B (i + 1)) B
+    sweep_bytes = d_out * d_in * (4 + 8 + p.bits / 8) + nb * B * B * 4
+    t_flops = sum(2.0 * d_out * (d_in - B * (i + 1)) * B for i in range(nb))
+    q_s = stages["quantize_layer"] / 1e3
+    return {
+        "hessian": {"bound": "tensor", "achieved": h_tf, "unit": "TFLOP/s", "peak": sustained,
+                    "frac": h_tf / sustained, "peak_kind": "bf16 dense sustained (measured)"},
+        "prepare_hinv": {"bound": "latency: 32 dependent 128-column steps", "achieved": f_tf, "unit": "TFLOP/s",
+                         "peak": sustained, "frac": f_tf / sustained,
+                         "work": "2 d^3 flops (Cholesky, triangular inverse, U), 3 tf32 passes issued for each"},
+        "quantize_layer": {"bound": "latency: 32 dependent sweep blocks, each followed by its trailing product",
+                           "sweep_gbs_over_stage": sweep_bytes / q_s / 1e9, "hbm_peak_gbs": hbm,
+                           "sweep_frac_over_stage": sweep_bytes / q_s / 1e9 / hbm,
+                           "trailing_tflops_over_stage": t_flops / q_s / 1e12, "tensor_peak": sustained,
+                           "trailing_frac_over_stage": t_flops / q_s / 1e12 / sustained,
+                           "work": f"sweep {sweep_bytes / 1e6:.1f} MB, trailing products {t_flops:.3e} flops "
+                                   "(3 tf32 passes issued), both over the whole stage time"},
+    }
 
 
 def act_order_timing(p, X_dev, W_dev, dev, stream, flush, args, api):
