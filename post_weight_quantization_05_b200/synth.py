@@ -22,6 +22,13 @@ checkpoint is used):
                  channels (seed-chosen) scaled x20.
 * ``mlp28672``   W [8192, 28672] bf16 ~ N(0, 0.01^2); X 65536 x 28672 bf16,
                  AR(1) rho = 0.9, 8 batches of 8192 rows.
+* ``gptstack``   weights of a stack of pre-LN GPT blocks (qkv [3d, d],
+                 attn_out [d, d], fc [4d, d], mlp_proj [d, 4d], all ~ N(0, 0.02^2),
+                 no biases, LayerNorms with unit gain and zero shift) and the
+                 calibration activations fed to its first block: batches of
+                 [seqs, tokens, d] with the gpt768 channel statistics (AR(1)
+                 rho = 0.8, per-channel std LogNormal(0, 0.5)).  Whole-model
+                 calibration passes them through the blocks in order.
 
 The AR(1) rows are drawn by the exact recursion x_0 = z_0,
 x_a = rho * x_{a-1} + sqrt(1 - rho^2) * z_a over the channel index a, which
@@ -37,7 +44,7 @@ from __future__ import annotations
 import dataclasses
 import numpy as np
 
-WORKLOAD_IDS = {"smoke": 1, "gpt768": 2, "attn4096": 3, "mlp11008": 4, "mlp28672": 5}
+WORKLOAD_IDS = {"smoke": 1, "gpt768": 2, "attn4096": 3, "mlp11008": 4, "mlp28672": 5, "gptstack": 6}
 
 _STREAM_W = 0
 _STREAM_X = 1
@@ -259,3 +266,32 @@ def x_batches_threaded(problem: LayerProblem, workers: int = 8):
 def x_as_f32(problem: LayerProblem, xb: np.ndarray) -> np.ndarray:
     """A batch as fp32 values (exact widening of the bf16 bytes)."""
     return bf16_bits_to_f32(xb) if problem.x_dtype == "bf16" else np.asarray(xb, dtype=np.float32)
+
+
+# ---------------------------------------------------------------------------
+# A stack of GPT blocks for block-sequential calibration
+# ---------------------------------------------------------------------------
+GPT_LINEARS = ("qkv", "attn_out", "fc", "mlp_proj")
+
+
+def gpt_stack_weights(n_blocks: int, d_model: int, base_seed: int = 0, w_std: float = 0.02):
+    """Per block a dict name -> fp32 weight [d_out, d_in] (nn.Linear layout)."""
+    shapes = {"qkv": (3 * d_model, d_model), "attn_out": (d_model, d_model), "fc": (4 * d_model, d_model),
+              "mlp_proj": (d_model, 4 * d_model)}
+    blocks = []
+    for b in range(n_blocks):
+        blocks.append({name: normal_weights(rng_for("gptstack", b, i, _STREAM_W, base_seed), *shapes[name], w_std)
+                       for i, name in enumerate(GPT_LINEARS)})
+    return blocks
+
+
+def gpt_stack_inputs(n_batches: int, seqs: int, tokens: int, d_model: int, base_seed: int = 0):
+    """Calibration activations entering the first block: n_batches arrays
+    [seqs, tokens, d_model] fp32 (AR(1) rho = 0.8 over channels, per-channel
+    std LogNormal(0, 0.5))."""
+    ch_scale = np.exp(rng_for("gptstack", 0, 0, _STREAM_SCALE, base_seed).normal(0.0, 0.5, size=d_model))
+    out = []
+    for b in range(n_batches):
+        x = ar1_rows(rng_for("gptstack", 0, b, _STREAM_X, base_seed), seqs * tokens, d_model, 0.8)
+        out.append((x * ch_scale[None, :].astype(np.float32)).reshape(seqs, tokens, d_model))
+    return out
