@@ -238,6 +238,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-act-order", action="store_true")
     ap.add_argument("--no-gemv", action="store_true")
+    ap.add_argument("--no-whole-model", action="store_true")
     ap.add_argument("--profile-case", action="store_true",
                     help="small case for ncu captures: one 16384-row batch of the same layer, 3 passes, no timing")
     args = ap.parse_args()
@@ -360,6 +361,11 @@ def main():
     if not args.no_act_order:
         act = act_order_timing(p, X_dev, W_dev, dev, stream, flush, args, api)
 
+    # ---- block-sequential calibration of a whole model
+    whole = None
+    if not args.no_whole_model:
+        whole = whole_model_timing(dev, args, api)
+
     # ---- the inference product from the stored form
     gemv = None
     if not args.no_gemv:
@@ -386,7 +392,7 @@ def main():
                            "l2": "flushed before every step (256 MiB write, outside the step events)"},
                 "ms_per_layer": ms_per_step, "stages_ms": stages, "stage_roofline": stage_roof, "roofline": roof,
                 "cpu_baseline": cpu,
-                "e2e": e2e, "gpu_launches": launches, "clocks": clk, "act_order": act, "dequant_gemv": gemv,
+                "e2e": e2e, "gpu_launches": launches, "clocks": clk, "act_order": act, "dequant_gemv": gemv, "whole_model": whole,
                 "input_generation_s": gen_s}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -525,6 +531,40 @@ def gemv_timing(dev, stream, flush, args, api, hbm_gbs):
         out[f"m{m}"] = {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs,
                         "launches": launches, "bf16_matmul_us": ref_us, "speedup_vs_bf16": ref_us / us}
     return out
+
+
+def whole_model_timing(dev, args, api):
+    """Block-sequential calibration of the 12-block d_model = 768 GPT (12
+    heads, bf16, random-init weights) on 10 batches x 8 sequences x 256
+    tokens of synthetic activations, 4-bit per-row grids: H for every linear
+    layer from forward hooks, each layer quantized, the quantized block
+    feeding the next.  Device events around the whole call; the model is
+    rebuilt from the same weights before each run, outside the events."""
+    import torch
+    from post_weight_quantization_05_b200 import driver, gpt_block, synth
+    n_blocks, d, heads = 12, 768, 12
+    weights = synth.gpt_stack_weights(n_blocks, d)
+    xs = [torch.from_numpy(x).to(dev).bfloat16() for x in synth.gpt_stack_inputs(10, 8, 256, d)]
+    n_weights = sum(w.size for W in weights for w in W.values())
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    runs = max(1, min(args.steps, 3))
+    for i in range(1 + runs):
+        blocks = gpt_block.gpt_stack(weights, heads, device=dev, dtype=torch.bfloat16)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        driver.BlockSequential(bits=4).quantize(blocks, xs)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        api.get_status(stream)
+        if i >= 1:
+            times.append(a.elapsed_time(b))
+        del blocks
+    ms = statistics.mean(times)
+    return {"workload": "12 pre-LN GPT blocks, d_model 768, 12 heads, bf16, 10 x 8 x 256 calibration tokens, "
+                        "4-bit per-row, B=128", "ms": ms, "ms_per_block": ms / n_blocks, "weights": n_weights,
+            "weights_per_s": n_weights / (ms / 1e3), "runs": runs, "warmup": 1}
 
 
 def end_to_end(p, xs_host, w_bits, lq, dev, args, world, dist):
