@@ -73,6 +73,24 @@ def peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+# --------------------------------------------------------------------------- ranks
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The job's time: the slowest rank's.  Every rank calls this at the same
+    point (a collective); dist = None for a single process."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput of N replicas: all ranks' units over the slowest
+    rank's time."""
+    return units_per_rank_step * world * steps / (ms_max / 1e3)
+
+
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi clock / throttle samples while the timed region runs."""
@@ -330,14 +348,9 @@ def main():
     prep_ms = [e[2].elapsed_time(e[3]) for e in all_evs]
     quant_ms = [e[3].elapsed_time(e[n_ev]) for e in all_evs]
     begin_ms = [e[0].elapsed_time(e[1]) for e in all_evs]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist if world > 1 else None, dev)
     ms_per_step = total_ms / args.steps
-    weights = p.d_out * p.d_in * world * args.steps
-    value = weights / (total_ms / 1e3)
+    value = job_throughput(p.d_out * p.d_in, world, args.steps, total_ms)
 
     # roofline of the dominant kernel: the X^T X launch (one per batch)
     burst, sustained, hbm, src = peaks()
@@ -627,13 +640,9 @@ def end_to_end(p, xs_host, w_bits, lq, dev, args, world, dist):
         one_step()
     end.record(comp)
     torch.cuda.synchronize(dev)
-    ms = start.elapsed_time(end)
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dist, dev)
     api.get_status(comp)
-    return {"value": p.d_out * p.d_in * world * steps / (ms / 1e3), "unit": "weights/s",
+    return {"value": job_throughput(p.d_out * p.d_in, world, steps, ms), "unit": "weights/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps, "steps": steps}
 
 
