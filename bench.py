@@ -543,6 +543,14 @@ def gemv_timing(dev, stream, flush, args, api, hbm_gbs):
         gbs = nbytes / (us * 1e-6) / 1e9
         out[f"m{m}"] = {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs,
                         "launches": launches, "bf16_matmul_us": ref_us, "speedup_vs_bf16": ref_us / us}
+    # the weights rebuilt from the stored form (bf16), the way a prefill-sized
+    # product uses them: this call, then a plain library GEMM
+    wq = torch.empty((d_out, d_in), dtype=torch.bfloat16, device=dev)
+    us = timed(lambda: api.dequantize(codes, scales, zeros, 4, g, wq))
+    api.get_status(stream)
+    nbytes = d_out * d_in // 2 + 2 * d_out * ng * 2 + d_out * d_in * 2
+    gbs = nbytes / (us * 1e-6) / 1e9
+    out["dequantize_bf16"] = {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs}
     return out
 
 

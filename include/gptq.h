@@ -306,6 +306,31 @@ int gptq_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint1
                       float* y, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Inference -- the weights rebuilt from the stored form.
+ * Source: note "Model Quantization", section "주요 양자화 기법", the GPTQ
+ * entry (at inference the INT4 weights are restored to FP16 for the
+ * computation); blog "GPTQ를 밑바닥부터 구현하며 배운 것들", section 5 (codes
+ * stored, dequantized for use).  A product with more tokens than
+ * gptq_dequant_gemv takes (prefill) is this call plus a plain library GEMM.
+ *
+ *   out[r][perm[k]] = s[r][g(k)] * (c[r][k] - z[r][g(k)])
+ *
+ * for every row r < d_out and code column k < d_in (processing order);
+ * perm = NULL: out[r][k].  g(k) = k / groupsize (0 for a per-row grid).
+ *   codes   device uint32 [d_out, d_in * bits / 32], 4-byte aligned;
+ *           bits 2, 3, 4 or 8.
+ *   scales, zeros  device fp16 bit patterns [d_out, n_groups].
+ *   perm    device int32 [d_in], 16-byte aligned, or NULL.  An entry outside
+ *           [0, d_in) is recorded as GPTQ_ERR_INVALID_ARG and skipped; a
+ *           column that no entry reaches is NaN.
+ *   out_dtype  0 fp32 (exact), 1 bf16, 2 fp16 (both rounded to nearest even).
+ *   out     device [d_out, d_in] of that type, row-major, 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+int gptq_dequantize(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
+                    int64_t d_in, int bits, int groupsize, const int32_t* perm, int out_dtype, void* out,
+                    void* stream);
+
+/* ------------------------------------------------------------------------
  * Helpers on the same stream (not steps of the method).
  * ---------------------------------------------------------------------- */
 /* dst[i] = (float) src[i] for bf16 bit patterns src (a bf16 layer's fp32

@@ -39,6 +39,7 @@ SIGNATURES = {
     "gptq_dequant_gemv_workspace_size": (c_size, [c_i64, c_i64, c_int]),
     "gptq_dequant_gemv": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_int, c_int, c_vp, c_vp, c_i64, c_vp, c_vp,
                                   c_size, c_vp]),
+    "gptq_dequantize": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_int, c_int, c_vp, c_int, c_vp, c_vp]),
     "gptq_widen_bf16": (c_int, [c_vp, c_vp, c_i64, c_vp]),
     "gptq_fill_f32": (c_int, [c_vp, c_i64, c_float, c_vp]),
     "gptq_get_status": (c_int, [c_vp, ctypes.POINTER(c_int)]),

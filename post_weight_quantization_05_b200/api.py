@@ -229,6 +229,27 @@ def dequant_gemv(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
     _check(code, "gptq_dequant_gemv")
 
 
+_OUT_DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, bits: int, groupsize: int,
+               out: torch.Tensor, perm: torch.Tensor | None = None, stream=None):
+    """out = the weights rebuilt from the stored form, in W's column order
+    (fp32 exact; bf16 / fp16 rounded)."""
+    d_out, d_in = out.shape
+    ng = n_groups(d_in, groupsize)
+    _need(codes, torch.int32, (d_out, d_in * bits // 32), "codes")
+    _need(scales, torch.float16, (d_out, ng), "scales")
+    _need(zeros, torch.float16, (d_out, ng), "zeros")
+    if out.dtype not in _OUT_DTYPES:
+        raise ValueError("out must be fp32, bf16 or fp16")
+    _need(out, out.dtype, (d_out, d_in), "out")
+    if perm is not None:
+        _need(perm, torch.int32, (d_in,), "perm")
+    _check(_lib().gptq_dequantize(_ptr(codes), _ptr(scales), _ptr(zeros), d_out, d_in, bits, groupsize, _ptr(perm),
+                                  _OUT_DTYPES[out.dtype], _ptr(out), _stream(stream)), "gptq_dequantize")
+
+
 def widen_bf16(src: torch.Tensor, dst: torch.Tensor, stream=None):
     if src.dtype != torch.bfloat16 or dst.dtype != torch.float32 or src.numel() != dst.numel():
         raise ValueError("widen_bf16: bf16 -> fp32 of equal size")

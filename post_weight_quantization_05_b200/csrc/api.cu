@@ -263,6 +263,22 @@ int gptq_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint1
                                static_cast<cudaStream_t>(stream), st, enc);
 }
 
+int gptq_dequantize(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
+                    int64_t d_in, int bits, int groupsize, const int32_t* perm, int out_dtype, void* out,
+                    void* stream) {
+    if (d_out <= 0 || d_out > (int64_t(1) << 24) || !valid_d_in(d_in)) return GPTQ_ERR_INVALID_ARG;
+    if (!valid_bits(bits) || !valid_group(groupsize, d_in) || out_dtype < 0 || out_dtype > 2)
+        return GPTQ_ERR_INVALID_ARG;
+    if (!codes || !scales || !zeros || !out) return GPTQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(codes) & 3u) || !aligned16(out) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
+        (reinterpret_cast<uintptr_t>(zeros) & 1u) || (perm && !aligned16(perm)))
+        return GPTQ_ERR_INVALID_ARG;
+    DevStatus* st = nullptr;
+    if (status_ptr(&st)) return GPTQ_ERR_CUDA;
+    return launch_dequantize(codes, scales, zeros, d_out, d_in, bits, groupsize, perm, out_dtype, out,
+                             static_cast<cudaStream_t>(stream), st);
+}
+
 int gptq_widen_bf16(const uint16_t* src, float* dst, int64_t count, void* stream) {
     if (count < 0) return GPTQ_ERR_INVALID_ARG;
     if (count == 0) return GPTQ_OK;

@@ -71,6 +71,12 @@ int launch_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uin
                         int64_t d_in, int groupsize, const int32_t* perm, const uint16_t* x, int64_t m, float* y,
                         void* ws, cudaStream_t stream, DevStatus* st, PFN_encodeTiled encode);
 
+// dequant.cu: the weights rebuilt from the stored form (2/3/4/8-bit codes,
+// act-order undone), out_dtype 0 fp32, 1 bf16, 2 fp16.
+int launch_dequantize(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,
+                      int64_t d_in, int bits, int groupsize, const int32_t* perm, int out_dtype, void* out,
+                      cudaStream_t stream, DevStatus* st);
+
 // permute.cu (act-order): the processing order from diag(H), the permuted
 // Hessian, and the column permutation of a row-major matrix (in place allowed).
 int launch_act_order_perm(const float* H, int64_t d, int32_t* perm, cudaStream_t stream);

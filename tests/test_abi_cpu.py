@@ -201,6 +201,22 @@ def test_dequant_gemv_rejects_bad_arguments(lib):
     assert call(perm=ctypes.c_void_p(0x10002), ws=FAKE, ws_bytes=4096) == 1
 
 
+def test_dequantize_rejects_bad_arguments(lib):
+    f = lib.gptq_dequantize
+    ok = dict(codes=FAKE, scales=FAKE, zeros=FAKE, d_out=64, d_in=512, bits=3, g=128, perm=None, dt=1, out=FAKE)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["codes"], a["scales"], a["zeros"], a["d_out"], a["d_in"], a["bits"], a["g"], a["perm"], a["dt"],
+                 a["out"], None)
+    assert call(bits=5) == 1 and call(bits=1) == 1
+    assert call(dt=3) == 1 and call(dt=-1) == 1
+    assert call(d_in=300) == 1 and call(g=100) == 1 and call(d_out=0) == 1
+    assert call(codes=None) == 1 and call(out=None) == 1
+    assert call(codes=ctypes.c_void_p(0x10002)) == 1 and call(out=MIS) == 1
+    assert call(perm=MIS) == 1 and call(scales=ctypes.c_void_p(0x10001)) == 1
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError):
         _native._lib = None
