@@ -27,11 +27,13 @@
 //   into warp-level fp16 MMAs (m16n8k16: 16 rows x 8 tokens, exact products,
 //   fp32 accumulation).  Each column block is then scaled in fp32 as
 //   2^e s (sum c x - z sum x); a shared-memory reduction over the 8 warps
-//   finishes y in a fixed order.  A lane's scales, zeros and block sums are
-//   loaded one stage ahead of their use.
+//   finishes y in a fixed order.  The block's scale / zero pairs (one padded
+//   word per row and group) and the tokens' block sums are staged in shared
+//   memory once, so the loop reads nothing else from global memory.
 // A word's nibbles are taken in pairs (p, p + 4) -- the two halves of a packed
-// fp16 register -- and x is stored in the same pairing, so no permute is left
-// in the inner loop.
+// fp16 register -- and x is stored in the same pairing, with the four lanes'
+// 16-byte chunks interleaved, so no permute is left in the inner loop and the
+// x reads are free of bank conflicts.
 #include <algorithm>
 
 #include "common.cuh"
@@ -95,8 +97,6 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-
-__device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
 // One warp's share of a column block, in registers: 16 bytes of codes of each
 // of the lane's 4 rows (g + 8 i) and 64 bytes of its token's x.
