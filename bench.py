@@ -240,6 +240,9 @@ def run_profile_case():
         y = torch.empty((m, d_out), dtype=torch.float32, device="cuda")
         for _ in range(2):
             api.dequant_gemv(codes, scales, zeros, 4, 128, xt, y)
+    # ... and the weights rebuilt from that stored form in bf16 (470 MB written)
+    wq = torch.empty((d_out, d_in), dtype=torch.bfloat16, device="cuda")
+    api.dequantize(codes, scales, zeros, 4, 128, wq)
     api.get_status()
     print("profile case done")
     return 0
