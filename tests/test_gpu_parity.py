@@ -409,3 +409,56 @@ def test_mlp28672_full_size_sampled_rows():
     be within 0.5% of the oracle's."""
     frac = _full_size_check(synth.mlp28672(), n_rows_sample=16, match=0.0)
     print(f"mlp28672: {frac:.4f} of sampled codes identical")
+
+
+@pytest.mark.slow
+def test_max_d_in_properties():
+    """d_in = 32768, the largest the library takes (H, U 4.3 GB each), with
+    fewer calibration rows than columns (H singular; the damping makes it
+    definite).  The fp64 oracle of this size does not fit the host, so the
+    checks are properties that hold at any size: H entries against exact
+    dot products, U^T U (H + lambda I) v = v in fp64 for random v, codes on
+    their recorded grid, and the GPTQ loss below RTN's."""
+    d_out, d_in, n = 96, 32768, 16384
+    p = synth.custom("maxd", d_out, d_in, n, bits=4, groupsize=128, x_dtype="bf16", n_batches=2, rho=0.9,
+                     layer=32768)
+    xs = [p.x_batch(b) for b in range(p.n_batches)]
+    lq = _gpu_pipeline(p, [to_dev_x(p, x) for x in xs], want_q=True)
+    xf = np.concatenate([synth.x_as_f32(p, x) for x in xs]).astype(np.float64)
+    del xs
+    rng = np.random.default_rng(3)
+    a = rng.integers(0, d_in, 64)
+    b = np.maximum(a, rng.integers(0, d_in, 64))
+    b[:8] = a[:8]                                       # some diagonal entries
+    Hg = lq.H
+    got = Hg[torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()].cpu().numpy().astype(np.float64)
+    want = 2.0 * np.einsum("ra,ra->a", xf[:, a], xf[:, b])
+    assert np.max(np.abs(got - want) / np.abs(want).max()) <= 1e-5
+    del xf
+    # U^T U (H + lambda I) v = v, in fp64 on the GPU
+    Hs = torch.triu(Hg).double()
+    Hs = Hs + torch.triu(Hs, 1).T
+    lam = p.percdamp * float(torch.diagonal(Hs).mean())
+    U = lq.U.double()
+    assert torch.count_nonzero(torch.tril(lq.U, -1)) == 0
+    for seed in range(3):
+        v = torch.randn(d_in, dtype=torch.float64, device="cuda", generator=torch.Generator("cuda").manual_seed(seed))
+        r = U.T @ (U @ (Hs @ v + lam * v))
+        assert float(torch.linalg.norm(r - v) / torch.linalg.norm(v)) <= 1e-3
+    # the stored form rebuilds Q exactly, and GPTQ beats RTN on the layer loss
+    out = torch.empty((d_out, d_in), dtype=torch.float32, device="cuda")
+    api.dequantize(lq.codes, lq.scales, lq.zeros, 4, 128, out)
+    api.get_status()
+    assert torch.equal(out, lq.Q)
+    W = torch.from_numpy(p.W).cuda().double()
+    codes = torch.zeros((d_out, d_in // 8), dtype=torch.int32, device="cuda")
+    sc = torch.zeros((d_out, d_in // 128), dtype=torch.float16, device="cuda")
+    zr = torch.zeros_like(sc)
+    Qr = torch.zeros((d_out, d_in), dtype=torch.float32, device="cuda")
+    api.rtn_layer(torch.from_numpy(p.W).cuda(), 4, 128, codes, sc, zr, Qr)
+    api.get_status()
+
+    def loss(Q):
+        D = W - Q.double()
+        return float(0.5 * torch.sum((D @ Hs) * D))
+    assert loss(lq.Q) < loss(Qr)
