@@ -243,6 +243,9 @@ def run_profile_case():
     # ... and the weights rebuilt from that stored form in bf16 (470 MB written)
     wq = torch.empty((d_out, d_in), dtype=torch.bfloat16, device="cuda")
     api.dequantize(codes, scales, zeros, 4, 128, wq)
+    # ... and with a column permutation undone
+    perm = torch.randperm(d_in, device="cuda", generator=gen).to(torch.int32)
+    api.dequantize(codes, scales, zeros, 4, 128, wq, perm=perm)
     api.get_status()
     print("profile case done")
     return 0
@@ -562,6 +565,13 @@ def gemv_timing(dev, stream, flush, args, api, hbm_gbs):
     nbytes = d_out * d_in // 2 + 2 * d_out * ng * 2 + d_out * d_in * 2
     gbs = nbytes / (us * 1e-6) / 1e9
     out["dequantize_bf16"] = {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs}
+    # the same with act-order undone (a random permutation of the columns)
+    perm = torch.randperm(d_in, device=dev, generator=gen).to(torch.int32)
+    us = timed(lambda: api.dequantize(codes, scales, zeros, 4, g, wq, perm=perm))
+    api.get_status(stream)
+    nbytes += d_in * 4
+    gbs = nbytes / (us * 1e-6) / 1e9
+    out["dequantize_bf16_perm"] = {"us": us, "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm_gbs}
     return out
 
 

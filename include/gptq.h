@@ -323,7 +323,10 @@ int gptq_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uint1
  *   perm    device int32 [d_in], 16-byte aligned, or NULL.  An entry outside
  *           [0, d_in) is recorded as GPTQ_ERR_INVALID_ARG and skipped; a
  *           column that no entry reaches is NaN.
- *   out_dtype  0 fp32 (exact), 1 bf16, 2 fp16 (both rounded to nearest even).
+ *   out_dtype  0 fp32: s (c - z) rounded once (exact whenever it fits 24
+ *              bits, as it always does for the integer zero points the
+ *              quantizer writes); 1 bf16, 2 fp16: that fp32 value rounded to
+ *              nearest even.
  *   out     device [d_out, d_in] of that type, row-major, 16-byte aligned.
  * ---------------------------------------------------------------------- */
 int gptq_dequantize(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, int64_t d_out,

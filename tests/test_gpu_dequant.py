@@ -100,3 +100,40 @@ def test_dequantize_bad_permutation_entry_is_reported():
     perm[3] = -7
     with pytest.raises(api.GPTQError):
         _run(words, s, z, 4, -1, d_in, perm, torch.float32)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("d_out,d_in,g", [(1, 128, -1), (7, 384, 128), (3, 32768, 256)])
+def test_dequantize_edge_shapes(bits, d_out, d_in, g):
+    """One row of the narrowest width, a ragged row count, and the widest rows
+    (the permuted path's largest shared-memory footprint), with and without a
+    permutation."""
+    words, s, z = _stored(d_out, d_in, bits, g, d_out * 100 + bits)
+    for with_perm in (False, True):
+        perm = np.random.default_rng(d_in + bits).permutation(d_in) if with_perm else None
+        want = _expected(words, s, z, bits, g, d_in, perm)
+        got = _run(words, s, z, bits, g, d_in, perm, torch.float32).cpu().numpy()
+        assert np.array_equal(got.astype(np.float64), want)
+        got = _run(words, s, z, bits, g, d_in, perm, torch.bfloat16).cpu()
+        assert torch.equal(got, torch.from_numpy(want.astype(np.float32)).bfloat16())
+
+
+@pytest.mark.parametrize("with_perm", [False, True])
+def test_dequantize_rounds_once(with_perm):
+    """Zero points off the integers (any fp16 grid a caller brings): each value
+    is the exact s (c - z) rounded once to fp32, then to nearest even for
+    fp16 / bf16.  The products here need up to 25 significant bits, so fp32
+    rounding does occur."""
+    d_out, d_in, g = 64, 1024, 128
+    words, s, z = _stored(d_out, d_in, 4, g, 17)
+    rng = np.random.default_rng(18)
+    z = rng.uniform(-8.0, 24.0, size=z.shape).astype(np.float16)
+    perm = np.random.default_rng(19).permutation(d_in) if with_perm else None
+    want = _expected(words, s, z, 4, g, d_in, perm)           # exact in fp64
+    want32 = want.astype(np.float32)
+    assert np.any(want32.astype(np.float64) != want)            # some values do round
+    got = _run(words, s, z, 4, g, d_in, perm, torch.float32).cpu().numpy()
+    assert np.array_equal(got, want32)
+    for dt in (torch.bfloat16, torch.float16):
+        got = _run(words, s, z, 4, g, d_in, perm, dt).cpu()
+        assert torch.equal(got, torch.from_numpy(want32).to(dt))
