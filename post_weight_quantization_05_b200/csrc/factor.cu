@@ -66,18 +66,26 @@ __global__ void damp_lambda_kernel(const float* __restrict__ H, int d, float per
 }
 
 // A[i][j] = H[d-1-i][d-1-j] (+ lambda on the diagonal) for j <= i: the lower
-// triangle of P (H + lambda I) P, read from the upper triangle of H.
-__global__ void reverse_damp_kernel(const float* __restrict__ H, int d, const float* __restrict__ lam,
-                                    float* __restrict__ A) {
+// triangle of P (H + lambda I) P, read from the upper triangle of H.  One
+// block per row i; each thread moves four columns, read as one reversed
+// float4 of H's row d-1-i (d is a multiple of 128, so both sides stay
+// aligned).  The float4 that holds the diagonal also writes up to three
+// entries above it, which nothing reads.
+__global__ void __launch_bounds__(256)
+    reverse_damp_kernel(const float* __restrict__ H, int d, const float* __restrict__ lam, float* __restrict__ A) {
+    const int i = blockIdx.x;
     const float l = *lam;
-    const size_t total = size_t(d) * d;
-    for (size_t idx = size_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += size_t(gridDim.x) * blockDim.x) {
-        const int i = int(idx / d), j = int(idx % d);
-        if (j > i) continue;
-        float v = H[size_t(d - 1 - i) * d + (d - 1 - j)];
-        if (i == j) v += l;
-        A[idx] = v;
+    const float* src = H + size_t(d - 1 - i) * d;
+    float4* dst = reinterpret_cast<float4*>(A + size_t(i) * d);
+    for (int j4 = threadIdx.x; 4 * j4 <= i; j4 += blockDim.x) {
+        const float4 h = *reinterpret_cast<const float4*>(src + (d - 4 - 4 * j4));   // columns d-4-4j4 .. d-1-4j4
+        float4 v = make_float4(h.w, h.z, h.y, h.x);
+        const int k = i - 4 * j4;                                                      // the diagonal's place, if < 4
+        if (k == 0) v.x += l;
+        else if (k == 1) v.y += l;
+        else if (k == 2) v.z += l;
+        else if (k == 3) v.w += l;
+        dst[j4] = v;
     }
 }
 
@@ -451,24 +459,39 @@ static int aux_stream(AuxStream** out) {
 }
 
 // U[r][c] = Z[d-1-c][d-1-r] for r <= c (U = P L'^-1 P = P Z^T P), 0 below the
-// diagonal; NaN everywhere if the factorization failed.  32 x 32 tiles are
-// transposed through shared memory so that both sides stay coalesced.
-__global__ void write_u_kernel(const float* __restrict__ Z, int d, const int* __restrict__ info,
-                               float* __restrict__ U) {
-    __shared__ float tile[32][33];
-    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+// diagonal; NaN everywhere if the factorization failed.  A block writes a
+// 64 x 64 tile of U: the matching tile of Z (rows d-c0-64 .., columns
+// d-r0-64 ..) comes in as float4 rows into shared memory (row stride 65, so
+// that the reversed, transposed reads below hit at most two ways of a bank),
+// and goes out as float4 rows of U.  Tiles wholly below the diagonal read
+// nothing.
+constexpr int UT = 64;
+__global__ void __launch_bounds__(256)
+    write_u_kernel(const float* __restrict__ Z, int d, const int* __restrict__ info, float* __restrict__ U) {
+    __shared__ float tile[UT][UT + 1];
+    const int r0 = blockIdx.y * UT, c0 = blockIdx.x * UT, t = threadIdx.x;
     const bool bad = *info != 0;
-    const bool below = c0 + 31 < r0;    // tile entirely in the strict lower triangle
+    const bool below = c0 + UT - 1 < r0;
     if (!below && !bad) {
-        for (int cc = threadIdx.y; cc < 32; cc += blockDim.y)
-            tile[cc][threadIdx.x] = Z[size_t(d - 1 - (c0 + cc)) * d + (d - 1 - (r0 + threadIdx.x))];
+        const float* zt = Z + size_t(d - c0 - UT) * d + (d - r0 - UT);
+        for (int idx = t; idx < UT * UT / 4; idx += 256) {
+            const int zr = idx / (UT / 4), zc = (idx % (UT / 4)) * 4;
+            const float4 v = *reinterpret_cast<const float4*>(zt + size_t(zr) * d + zc);
+            tile[zr][zc] = v.x; tile[zr][zc + 1] = v.y; tile[zr][zc + 2] = v.z; tile[zr][zc + 3] = v.w;
+        }
     }
     __syncthreads();
-    for (int rr = threadIdx.y; rr < 32; rr += blockDim.y) {
-        const int r = r0 + rr, c = c0 + threadIdx.x;
-        float v = (!below && c >= r) ? tile[threadIdx.x][rr] : 0.0f;
-        if (bad) v = __int_as_float(0x7fc00000);
-        U[size_t(r) * d + c] = v;
+    for (int idx = t; idx < UT * UT / 4; idx += 256) {
+        const int rl = idx / (UT / 4), cl = (idx % (UT / 4)) * 4;
+        const int r = r0 + rl;
+        float o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int c = c0 + cl + q;
+            // U[r][c] = Z[d-1-c][d-1-r] = tile[(d-1-c) - (d-c0-UT)][(d-1-r) - (d-r0-UT)]
+            o[q] = bad ? __int_as_float(0x7fc00000) : (!below && c >= r) ? tile[UT - 1 - (cl + q)][UT - 1 - rl] : 0.0f;
+        }
+        *reinterpret_cast<float4*>(U + size_t(r) * d + c0 + cl) = make_float4(o[0], o[1], o[2], o[3]);
     }
 }
 
@@ -488,7 +511,6 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     float* lam = reinterpret_cast<float*>(base + L.scal_off);
     int* info = info_user ? info_user : reinterpret_cast<int*>(base + L.scal_off + 64);
     const int nblk = d / NB;
-    const int ew_blocks = int(std::min<int64_t>((int64_t(d) * d + 255) / 256, 148 * 32));
 
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -513,7 +535,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         return GPTQ_ERR_CUDA;
 
     damp_lambda_kernel<<<1, 1024, 0, stream>>>(H, d, percdamp, lam, info, st); count_launch();
-    reverse_damp_kernel<<<ew_blocks, 256, 0, stream>>>(H, d, lam, A); count_launch();
+    reverse_damp_kernel<<<d, 256, 0, stream>>>(H, d, lam, A); count_launch();
     // fork: the inverse (stream `as`) starts from a zeroed Z; `ss` takes the
     // trailing updates beyond the next NEAR block columns
     const cudaStream_t ss = aux->side;
@@ -603,7 +625,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         cudaEventRecord(aux->join_side, ss) != cudaSuccess ||
         cudaStreamWaitEvent(stream, aux->join_side, 0) != cudaSuccess)
         return GPTQ_ERR_CUDA;
-    write_u_kernel<<<dim3(d / 32, d / 32), dim3(32, 8), 0, stream>>>(Z, d, info, U); count_launch();
+    write_u_kernel<<<dim3(d / UT, d / UT), 256, 0, stream>>>(Z, d, info, U); count_launch();
     // back to the caller's stream
     if (cudaEventRecord(aux->join, stream) != cudaSuccess || cudaStreamWaitEvent(caller, aux->join, 0) != cudaSuccess)
         return GPTQ_ERR_CUDA;
