@@ -276,29 +276,38 @@ __global__ void __launch_bounds__(GATHER_THREADS, 1)
     }
 }
 
+// The gather kernel's shared memory: ip (16-bit, padded to 16 bytes) and
+// d_in + 1 slots; 196,612 bytes at the largest d_in (32768).
+inline size_t gather_smem(int d_in) { return ((size_t(d_in) * 2 + 15) & ~size_t(15)) + size_t(d_in + 1) * 4; }
+
 template <int BITS, int OUT>
 int launch_typed(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros, const int32_t* perm,
                  Shape sh, void* out, cudaStream_t stream, DevStatus* st) {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return GPTQ_ERR_CUDA;
     uint4* o = static_cast<uint4*>(out);
     if (!perm) {
         const int64_t n_chunks = (sh.vpr + CHUNK - 1) / CHUNK;
         const int64_t blocks = (sh.d_out + ROWS - 1) / ROWS * n_chunks;      // <= 2^22 * 16
         dequant_vec_kernel<BITS, OUT><<<unsigned(blocks), VEC_THREADS, 0, stream>>>(codes, scales, zeros, sh, o);
     } else {
-        const size_t smem = ((size_t(sh.d_in) * 2 + 15) & ~size_t(15)) + size_t(sh.d_in + 1) * 4;   // <= 192 KB + 4
-        if (cudaFuncSetAttribute(dequant_gather_kernel<BITS, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(smem)) != cudaSuccess)
-            return GPTQ_ERR_CUDA;
+        // once per device: the shared-memory limit for the largest d_in, and the SM count
+        static bool ready[64] = {};
+        static int sms[64] = {};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
+        if (!ready[dev]) {
+            if (cudaFuncSetAttribute(dequant_gather_kernel<BITS, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(gather_smem(32768))) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            ready[dev] = true;
+        }
+        const size_t smem = gather_smem(sh.d_in);
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dequant_gather_kernel<BITS, OUT>, GATHER_THREADS,
                                                           smem) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         const int64_t units = OUT == 0 ? sh.d_out : (sh.d_out + 1) / 2;     // rows per block step: 1 or 2
-        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(units, int64_t(sms) * std::max(per_sm, 1)));
+        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(units, int64_t(sms[dev]) * std::max(per_sm, 1)));
         dequant_gather_kernel<BITS, OUT><<<unsigned(blocks), GATHER_THREADS, smem, stream>>>(codes, scales, zeros,
                                                                                              perm, sh, o, st);
     }

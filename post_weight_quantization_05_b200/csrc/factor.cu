@@ -416,12 +416,17 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
     }
 }
 
-// Three internal streams and a few events per device (created on first use).
+// Three internal streams and a few events per set (created on first use).
 // The factorization's critical chain runs on a high-priority stream; the
 // inverse's block steps run on another, each as soon as the factorization has
 // finished the block column it needs; the trailing update beyond the next
 // NEAR block columns runs on a low-priority stream, so that the next diagonal
 // blocks are factored while it proceeds (look-ahead) and get the SMs first.
+// Each device has AUX_SETS sets.  A caller stream keeps the set it was given
+// first, so that factorizations called on different streams (independent
+// layers) run concurrently; once every set is taken, further caller streams
+// share them in turn, and calls on a shared set enqueue one at a time.
+constexpr int AUX_SETS = 4;
 struct AuxStream {
     cudaStream_t main = nullptr;    // the factorization's critical chain (highest priority)
     cudaStream_t s = nullptr;       // inverse steps
@@ -429,15 +434,29 @@ struct AuxStream {
     static constexpr int RING = 4;
     cudaEvent_t fork = nullptr, step = nullptr, join = nullptr, join_side = nullptr, filled = nullptr;
     cudaEvent_t far_done[RING] = {};   // the far update of step k, slot k % RING
+    std::mutex enqueue;                // one call enqueues on this set at a time
+    cudaStream_t owner = nullptr;      // the caller stream the set was given to
+    bool taken = false;
 };
 
-static int aux_stream(AuxStream** out) {
+static int aux_stream(cudaStream_t caller, AuxStream** out) {
     static std::mutex mu;
-    static AuxStream per_dev[64];
+    static AuxStream per_dev[64][AUX_SETS];
+    static int next_shared[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
     std::lock_guard<std::mutex> lock(mu);
-    AuxStream& a = per_dev[dev];
+    AuxStream* pick = nullptr;
+    for (int i = 0; i < AUX_SETS && !pick; ++i)
+        if (per_dev[dev][i].taken && per_dev[dev][i].owner == caller) pick = &per_dev[dev][i];
+    for (int i = 0; i < AUX_SETS && !pick; ++i)
+        if (!per_dev[dev][i].taken) {
+            pick = &per_dev[dev][i];
+            pick->taken = true;
+            pick->owner = caller;
+        }
+    if (!pick) pick = &per_dev[dev][next_shared[dev]++ % AUX_SETS];
+    AuxStream& a = *pick;
     if (!a.s) {
         int least = 0, greatest = 0;
         if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
@@ -522,12 +541,11 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         attr_set[dev] = true;
     }
 
-    // One call enqueues at a time (per process): the auxiliary stream and its
-    // events are shared by every call on a device.
-    static std::mutex enqueue_mu;
-    std::lock_guard<std::mutex> enqueue_lock(enqueue_mu);
+    // The internal streams and events of this caller stream's set; calls that
+    // share a set enqueue one at a time.
     AuxStream* aux = nullptr;
-    if (aux_stream(&aux)) return GPTQ_ERR_CUDA;
+    if (aux_stream(stream, &aux)) return GPTQ_ERR_CUDA;
+    std::lock_guard<std::mutex> enqueue_lock(aux->enqueue);
     const cudaStream_t as = aux->s;
     const cudaStream_t caller = stream;
     stream = aux->main;

@@ -13,7 +13,8 @@ kernel as the block runs (a forward hook per layer), then each layer is
 quantized (factorization, blocked sweep, packing; act-order if asked), its
 weight is replaced by the dequantized Q, and the quantized block runs once
 more to produce the next block's inputs.  All layers of a block are
-calibrated on the same pass of the unquantized block.
+calibrated on the same pass of the unquantized block, and quantized
+concurrently, each on a stream of its own.
 """
 from __future__ import annotations
 
@@ -23,6 +24,9 @@ import torch
 from torch import nn
 
 from . import api
+
+
+_STREAMS: dict = {}   # device -> streams for the layers' quantization
 
 
 @dataclasses.dataclass
@@ -38,9 +42,10 @@ class QuantizedLinear:
 
 class BlockSequential:
     def __init__(self, bits: int = 4, groupsize: int = -1, percdamp: float = 0.01, act_order: bool = False,
-                 keep_hessian: bool = False):
+                 keep_hessian: bool = False, max_tokens: int = 32768):
         self.bits, self.groupsize, self.percdamp = bits, groupsize, percdamp
         self.act_order, self.keep_hessian = act_order, keep_hessian
+        self.max_tokens = max_tokens
 
     @staticmethod
     def linears(block: nn.Module):
@@ -53,7 +58,7 @@ class BlockSequential:
         first one.  The weights of every nn.Linear are replaced by their
         dequantized values.  Returns one dict per block (layer name ->
         QuantizedLinear) and the last block's outputs."""
-        xs = list(inputs)
+        xs, groups = self._merge(list(inputs))
         report = []
         for block in blocks:
             layers = self.linears(block)
@@ -80,13 +85,59 @@ class BlockSequential:
             finally:
                 for h in hooks:
                     h.remove()
+            # The layers' factorizations and sweeps are independent: each runs
+            # on a stream of its own (the library gives every caller stream its
+            # own internal streams), forked from and joined back to the
+            # calibration stream.
             out = {}
-            for name, m in layers:
+            main = stream if stream is not None else torch.cuda.current_stream()
+            ready = torch.cuda.Event()
+            ready.record(main)
+            done = []
+            for (name, m), side in zip(layers, self._streams(len(layers))):
+                side.wait_event(ready)
                 lq = quant[name]
-                lq.finish(stream)
-                m.weight.copy_(lq.Q.to(m.weight.dtype))
+                with torch.cuda.stream(side):
+                    lq.finish(side)
+                    m.weight.copy_(lq.Q.to(m.weight.dtype))
+                ev = torch.cuda.Event()
+                ev.record(side)
+                done.append(ev)
                 out[name] = QuantizedLinear(lq.codes, lq.scales, lq.zeros, lq.perm,
                                             lq.H if self.keep_hessian else None)
+            for ev in done:
+                main.wait_event(ev)
             report.append(out)
-            xs = [block(x) for x in xs]
-        return report, xs
+            with torch.cuda.stream(main):
+                xs = [block(x) for x in xs]
+        return report, [part for x, g in zip(xs, groups) for part in x.split(g)]
+
+    def _merge(self, xs):
+        """Consecutive batches of the same sequence shape joined into one,
+        up to max_tokens tokens each: one forward (and one Hessian call per
+        layer) instead of several.  H is the same sum over the same rows.
+        Returns the joined batches and, for each, the sizes of its parts."""
+        out, groups, cur, n = [], [], [], 0
+        for x in xs:
+            t = x.numel() // x.shape[-1]
+            if cur and (x.shape[1:] != cur[0].shape[1:] or n + t > self.max_tokens):
+                out.append(torch.cat(cur) if len(cur) > 1 else cur[0])
+                groups.append([c.shape[0] for c in cur])
+                cur, n = [], 0
+            cur.append(x)
+            n += t
+        if cur:
+            out.append(torch.cat(cur) if len(cur) > 1 else cur[0])
+            groups.append([c.shape[0] for c in cur])
+        return out, groups
+
+    @staticmethod
+    def _streams(n):
+        """n streams of the current device, created once per process and
+        reused, so that each keeps the library's internal streams it was
+        given."""
+        dev = torch.cuda.current_device()
+        pool = _STREAMS.setdefault(dev, [])
+        while len(pool) < n:
+            pool.append(torch.cuda.Stream(dev))
+        return pool[:n]
