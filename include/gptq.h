@@ -135,6 +135,13 @@ int gptq_hessian_accumulate_batches(const void* const* X, const int64_t* n, int 
  *            and finite.  The status word gets GPTQ_ERR_NOT_PD (or
  *            GPTQ_ERR_NONFINITE for a NaN/Inf pivot).
  *   ws       >= gptq_prepare_hinv_workspace_size(d_in) bytes.
+ * The work forks from `stream` onto three library-owned streams (the
+ * factorization's chain, its look-ahead updates, the inverse) and joins back
+ * before the call's last kernel; later work on `stream` sees U complete.  A
+ * device has four such sets.  A caller stream keeps the set it got first, so
+ * calls on up to four different streams run concurrently (independent
+ * layers); further streams share the sets, and calls sharing a set run one
+ * after the other.
  * ---------------------------------------------------------------------- */
 size_t gptq_prepare_hinv_workspace_size(int64_t d_in);
 int gptq_prepare_hinv(const float* H, int64_t d_in, float percdamp, float* U,

@@ -234,8 +234,9 @@ _OUT_DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, bits: int, groupsize: int,
                out: torch.Tensor, perm: torch.Tensor | None = None, stream=None):
-    """out = the weights rebuilt from the stored form, in W's column order
-    (fp32 exact; bf16 / fp16 rounded)."""
+    """out = the weights rebuilt from the stored form, in W's column order:
+    s (c - z) rounded once to fp32 (exact for integer zero points), or that
+    value rounded to nearest even in bf16 / fp16."""
     d_out, d_in = out.shape
     ng = n_groups(d_in, groupsize)
     _need(codes, torch.int32, (d_out, d_in * bits // 32), "codes")
