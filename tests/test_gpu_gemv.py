@@ -98,6 +98,19 @@ def test_gemv_act_order_permutation(d_out, d_in, g, m):
     _check(y, words, s, z, g, xf, perm)
 
 
+@pytest.mark.parametrize("g,m,with_perm", [(128, 8, False), (128, 8, True), (-1, 1, False)])
+def test_gemv_widest_rows(g, m, with_perm):
+    """d_in = 32768, the widest the library takes: the most column blocks,
+    the largest staged scale table (256 groups) and, at m = 8, the largest
+    block data of x (the ring drops to two stages); 70 rows, a ragged tile."""
+    d_out, d_in = 70, 32768
+    words, s, z = _stored_form(d_out, d_in, g, 11 + m)
+    xbits, xf = _tokens(m, d_in, 13)
+    perm = np.random.default_rng(4).permutation(d_in) if with_perm else None
+    y = _run(words, s, z, g, xbits, perm)
+    _check(y, words, s, z, g, xf, perm)
+
+
 @pytest.mark.parametrize("m", [1, 8])
 def test_gemv_full_size_sampled_rows(m):
     """The 8192 x 28672 g128 layer (the largest of the workloads), every
