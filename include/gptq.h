@@ -141,7 +141,9 @@ int gptq_hessian_accumulate_batches(const void* const* X, const int64_t* n, int 
  * device has four such sets.  A caller stream keeps the set it got first, so
  * calls on up to four different streams run concurrently (independent
  * layers); further streams share the sets, and calls sharing a set run one
- * after the other.
+ * after the other.  A set's streams and events are created by the first call
+ * that gets it; a caller that records these calls into a stream capture
+ * makes one call on that stream before the capture begins.
  * ---------------------------------------------------------------------- */
 size_t gptq_prepare_hinv_workspace_size(int64_t d_in);
 int gptq_prepare_hinv(const float* H, int64_t d_in, float percdamp, float* U,
