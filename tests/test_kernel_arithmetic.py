@@ -1,0 +1,60 @@
+"""Arithmetic facts the stored-form kernels rely on, checked on the host
+against exact integer and rational arithmetic (no GPU):
+
+- the group index of column k as a reciprocal multiply,
+  floor((k / 128) / (g / 128)) = ((k >> 7) * ceil(2^16 / (g / 128))) >> 16,
+  for every k < 32768 and every group g = 128 q, q <= 256;
+- the code-to-float conversion through the exponent field,
+  bits(0x4B000000 | c) - 2^23 = c for c < 2^23;
+- the product of two fp16 numbers is exact in fp32;
+- s c - s z formed from those exact products and rounded once equals the
+  exact s (c - z) rounded once to fp32 (what one fused multiply-add gives).
+"""
+from fractions import Fraction
+
+import numpy as np
+
+
+def test_group_index_reciprocal_is_exact():
+    n = np.arange(256, dtype=np.int64)[:, None]            # k >> 7 for k < 32768
+    q = np.arange(1, 257, dtype=np.int64)[None, :]         # group / 128
+    inv = -(-65536 // q)                                    # ceil(2^16 / q)
+    assert np.array_equal((n * inv) >> 16, n // q)
+
+
+def test_exponent_field_conversion_is_exact():
+    c = np.arange(0, 1 << 12, dtype=np.uint32)              # codes (8-bit and well beyond)
+    f = (np.uint32(0x4B000000) | c).view(np.float32) - np.float32(8388608.0)
+    assert np.array_equal(f, c.astype(np.float32))
+
+
+def _fp16_sample(rng, n, lo, hi):
+    return rng.uniform(lo, hi, n).astype(np.float16)
+
+
+def test_fp16_products_are_exact_in_fp32():
+    rng = np.random.default_rng(0)
+    s = np.concatenate([_fp16_sample(rng, 4000, 1e-6, 1.0), np.array([6.1e-5, 65504.0], np.float16)])
+    z = np.concatenate([_fp16_sample(rng, 4000, -300.0, 300.0), np.array([-2048.0, 2048.0], np.float16)])
+    p32 = s.astype(np.float32) * z.astype(np.float32)
+    exact = [Fraction(float(a)) * Fraction(float(b)) for a, b in zip(s, z)]
+    assert all(Fraction(float(p)) == e for p, e in zip(p32, exact))
+
+
+def test_one_rounding_of_the_dequantized_value():
+    rng = np.random.default_rng(1)
+    n = 20000
+    s = _fp16_sample(rng, n, 1e-5, 0.05)
+    z = _fp16_sample(rng, n, -8.0, 24.0)                     # off the integers: rounding happens
+    c = rng.integers(0, 256, n).astype(np.float32)
+    s32, z32 = s.astype(np.float32), z.astype(np.float32)
+    # both products are exact in fp32, so one fp32 subtraction rounds the exact difference once
+    got = s32 * c - s32 * z32
+    rounded = 0
+    for i in range(n):
+        exact = Fraction(float(s[i])) * (Fraction(int(c[i])) - Fraction(float(z[i])))
+        want = np.float32(float(exact))                        # fp64 holds it exactly; one rounding to fp32
+        assert Fraction(float(np.float64(float(exact)))) == exact
+        assert got[i] == want, (i, float(s[i]), float(z[i]), int(c[i]))
+        rounded += Fraction(float(want)) != exact
+    assert rounded > 0                                         # the check has teeth: some values do round
