@@ -8,7 +8,10 @@ against exact integer and rational arithmetic (no GPU):
   bits(0x4B000000 | c) - 2^23 = c for c < 2^23;
 - the product of two fp16 numbers is exact in fp32;
 - s c - s z formed from those exact products and rounded once equals the
-  exact s (c - z) rounded once to fp32 (what one fused multiply-add gives).
+  exact s (c - z) rounded once to fp32 (what one fused multiply-add gives);
+- the 4-bit product's fp16 conversion constants give exact codes from either
+  nibble, and its power-of-two scaling of bf16 x into fp16 is exact over the
+  range it claims.
 """
 from fractions import Fraction
 
@@ -58,3 +61,33 @@ def test_one_rounding_of_the_dequantized_value():
         assert got[i] == want, (i, float(s[i]), float(z[i]), int(c[i]))
         rounded += Fraction(float(want)) != exact
     assert rounded > 0                                         # the check has teeth: some values do round
+
+
+def test_fp16_code_conversion_constants():
+    """The 4-bit product's conversion: a code c in the low nibble of a half
+    ORed into 0x6400 is 1024 + c, and adding 0xE400 (-1024) gives c; in the
+    high nibble it is 1024 + 16 c, and times 0x2C00 (1/16) plus 0xD400 (-64)
+    gives c.  Every intermediate is exact in fp16."""
+    h = lambda bits: np.array([bits], dtype=np.uint16).view(np.float16)[0]  # noqa: E731
+    k_sub, k_s16, k_sub64 = h(0xE400), h(0x2C00), h(0xD400)
+    assert (float(k_sub), float(k_s16), float(k_sub64)) == (-1024.0, 1.0 / 16, -64.0)
+    for c in range(16):
+        lo = h(0x6400 | c)
+        hi = h(0x6400 | (c << 4))
+        assert float(lo) == 1024 + c and float(np.float16(lo + k_sub)) == c
+        assert float(hi) == 1024 + 16 * c
+        t = np.float16(hi * k_s16)                          # 64 + c, exact
+        assert float(t) == 64 + c and float(np.float16(t + k_sub64)) == c
+
+
+def test_scaled_bf16_values_are_exact_in_fp16():
+    """The product scales each 128-column block of bf16 x by a power of two
+    that puts its largest magnitude in [2^14, 2^15): every bf16 value from
+    2^-28 of that maximum up to it then lies in fp16's normal range
+    [2^-14, 2^15], where fp16's 11-bit significand holds bf16's 8 bits."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    v = (bits << 16).view(np.float32)                        # every bf16 value
+    a = np.abs(v)
+    sel = np.isfinite(v) & (a >= 2.0 ** -14) & (a < 2.0 ** 15)
+    assert np.array_equal(v[sel].astype(np.float16).astype(np.float32), v[sel])
+    assert 2.0 ** 14 * 2.0 ** -28 == 2.0 ** -14               # the range's floor for a block max of 2^14
