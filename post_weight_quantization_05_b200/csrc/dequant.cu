@@ -19,6 +19,7 @@
 // block keeps the inverse permutation in shared memory, decodes one or two
 // rows in processing order into shared memory, and gathers each output
 // column from there.  Bound by HBM: bits / 8 bytes per weight in, 2 or 4 out.
+#include <atomic>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -290,15 +291,17 @@ int launch_typed(const uint32_t* codes, const uint16_t* scales, const uint16_t* 
         dequant_vec_kernel<BITS, OUT><<<unsigned(blocks), VEC_THREADS, 0, stream>>>(codes, scales, zeros, sh, o);
     } else {
         // once per device: the shared-memory limit for the largest d_in, and the SM count
-        static bool ready[64] = {};
-        static int sms[64] = {};
+        static std::atomic<bool> ready[64];   // zero-initialized (static storage)
+        static std::atomic<int> sms[64];
         int dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
         if (!ready[dev]) {
+            int n = 0;
             if (cudaFuncSetAttribute(dequant_gather_kernel<BITS, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      int(gather_smem(32768))) != cudaSuccess ||
-                cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
+            sms[dev] = n;
             ready[dev] = true;
         }
         const size_t smem = gather_smem(sh.d_in);
@@ -307,7 +310,7 @@ int launch_typed(const uint32_t* codes, const uint16_t* scales, const uint16_t* 
                                                           smem) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         const int64_t units = OUT == 0 ? sh.d_out : (sh.d_out + 1) / 2;     // rows per block step: 1 or 2
-        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(units, int64_t(sms[dev]) * std::max(per_sm, 1)));
+        const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(units, int64_t(sms[dev].load()) * std::max(per_sm, 1)));
         dequant_gather_kernel<BITS, OUT><<<unsigned(blocks), GATHER_THREADS, smem, stream>>>(codes, scales, zeros,
                                                                                              perm, sh, o, st);
     }

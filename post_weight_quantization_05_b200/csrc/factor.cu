@@ -18,6 +18,7 @@
 //   (both on the tensor cores, tgemm).  Z = L'^-T is built block column by
 //   block column alongside (right-looking forward substitution on the
 //   identity, transposed), and U is written by reversing both indices.
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -531,7 +532,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     int* info = info_user ? info_user : reinterpret_cast<int*>(base + L.scal_off + 64);
     const int nblk = d / NB;
 
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {

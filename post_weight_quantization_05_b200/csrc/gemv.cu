@@ -34,6 +34,7 @@
 // fp16 register -- and x is stored in the same pairing, with the four lanes'
 // 16-byte chunks interleaved, so no permute is left in the inner loop and the
 // x reads are free of bank conflicts.
+#include <atomic>
 #include <algorithm>
 
 #include "common.cuh"
@@ -440,7 +441,7 @@ int launch_dequant_gemv(const uint32_t* codes, const uint16_t* scales, const uin
     const size_t smem = ring_bytes + side;
     constexpr size_t SMEM_CAP = size_t(160) * 1024;   // largest case (m = 8, d_in = 32768): about 112 KB
     if (smem > SMEM_CAP) return GPTQ_ERR_UNSUPPORTED;
-    static bool attr_done[64] = {};
+    static std::atomic<bool> attr_done[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {

@@ -29,6 +29,7 @@
 //    contraction then runs over the six leading cross products
 //    (hh, hm, mh, mm, hl, lh), which the K loop walks one after another.
 //  - No TMA load uses multicast (each CTA loads its own halves).
+#include <atomic>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -289,7 +290,7 @@ int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, voi
     p.late_wait = (after_own_launch && dtype != GPTQ_F32) ? 1 : 0;
     p.T = int((d + BNP - 1) / BNP);
     p.tiles = p.T * (p.T + 1) / 2;
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {

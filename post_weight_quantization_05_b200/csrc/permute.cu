@@ -13,6 +13,7 @@
 //                         dst[r][perm[k]] = src[r][k]  (back to the original
 //                         order); in place when src == dst
 // All three are bound by HBM (or L2) traffic, not arithmetic.
+#include <atomic>
 #include "common.cuh"
 #include "kernels.h"
 
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(ROW_THREADS)
 constexpr size_t MAX_ROW_SMEM = 32768 * sizeof(float);
 
 int allow_big_rows(const void* fn, int slot) {
-    static bool done[64][3] = {};
+    static std::atomic<bool> done[64][3];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
     if (dev >= 0 && dev < 64 && done[dev][slot]) return GPTQ_OK;

@@ -18,6 +18,7 @@
 // the same time (broadcast).  The block's E is written for the lazy trailing
 // product on the tensor cores.  The codes are packed in registers
 // (compile-time bit positions) and stored as vectors.
+#include <atomic>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -416,7 +417,7 @@ __global__ void transpose_upper_kernel(const float* __restrict__ U, int d, float
 
 template <int BITS>
 int run_sweep(const SweepArgs& a, cudaStream_t stream) {
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {

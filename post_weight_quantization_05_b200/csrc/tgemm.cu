@@ -31,6 +31,7 @@
 // 32 columns at a time (128-byte swizzle, conflict-free) and writes it with one
 // TMA store, or one TMA reduce-add when accumulating, so C leaves the SM as
 // whole lines and is never read by the SM.  No TMA load uses multicast.
+#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -317,18 +318,21 @@ PFN_encodeTiled g_enc = nullptr;
 template <bool PRESPLIT>
 int launch_variant(const tg::Maps& maps, const tg::Args& g, cudaStream_t stream) {
     using C = tg::Cfg<PRESPLIT>;
-    static bool attr_set[64] = {};
-    static int sms[64] = {};
+    static std::atomic<bool> attr_set[64];
+    static std::atomic<int> sms[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
     if (dev < 64 && !attr_set[dev]) {
+        int n = 0;
         if (cudaFuncSetAttribute(tg::tgemm_kernel<PRESPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(C::SMEM_BYTES)) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return GPTQ_ERR_CUDA;
+        sms[dev] = n;
         attr_set[dev] = true;
     }
-    const int grid = std::max(1, std::min(g.tiles, dev < 64 && sms[dev] > 0 ? sms[dev] : 148));
+    const int n_sms = dev < 64 ? sms[dev].load() : 0;
+    const int grid = std::max(1, std::min(g.tiles, n_sms > 0 ? n_sms : 148));
     if (launch_pdl(tg::tgemm_kernel<PRESPLIT>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, maps, g) !=
         cudaSuccess)
         return GPTQ_ERR_CUDA;
