@@ -436,12 +436,17 @@ def stage_rooflines(p, stages, burst, sustained, hbm):
     nb = d_in // B
     h_flops = p.n * d_in * (d_in + 1)                        # upper triangle incl. diagonal, 2 per MAC
     h_tf = h_flops / (stages["hessian_16_batches"] / 1e3) / 1e12
-    # factorization: Cholesky (d^3/3) + triangular inverse (d^3/3) + U from the inverse (d^3/3), 2 per MAC
-    f_flops = 2.0 * d_in ** 3
+    # factorization as run: one Cholesky (d^3/3 flops) and one triangular inverse (d^3/3); U is
+    # the inverse with both indices reversed (no flops).  The pages' literal chain would be 4/3 d^3.
+    f_flops = 2.0 * d_in ** 3 / 3.0
     f_tf = f_flops / (stages["prepare_hinv"] / 1e3) / 1e12
-    # sweep: each block reads its W columns and U diagonal block, writes E (tf32 hi / lo) and the codes;
+    # sweep, algorithmic: W read and E written once (fp32 each), the codes, the grid (fp16 scale and
+    # zero per row and group) and the U diagonal blocks.  As built E is written twice (its tf32 part
+    # and the remainder, for the three-pass trailing products): 4 more bytes per weight issued.
+    ng = p.d_in // p.groupsize if p.groupsize > 0 else 1
+    sweep_bytes = d_out * d_in * (4 + 4 + p.bits / 8) + d_out * ng * 4 + nb * B * B * 4
+    sweep_issued = sweep_bytes + d_out * d_in * 4
     # trailing products: sum over blocks of 2 d_out (d_in - B (i + 1)) B
-    sweep_bytes = d_out * d_in * (4 + 8 + p.bits / 8) + nb * B * B * 4
     t_flops = sum(2.0 * d_out * (d_in - B * (i + 1)) * B for i in range(nb))
     q_s = stages["quantize_layer"] / 1e3
     return {
@@ -450,15 +455,18 @@ def stage_rooflines(p, stages, burst, sustained, hbm):
         "prepare_hinv": {"bound": "latency: 32 dependent 128-column steps", "achieved": f_tf, "unit": "TFLOP/s",
                          "peak": sustained, "frac": f_tf / sustained,
                          "issued_tflops": 3 * f_tf,
-                         "work": "2 d^3 flops (Cholesky, triangular inverse, U), 3 tf32 passes issued for each"},
+                         "work": "2/3 d^3 flops (Cholesky d^3/3, triangular inverse d^3/3), 3 tf32 passes "
+                                 "issued for their products"},
         "quantize_layer": {"bound": "latency: 32 dependent sweep blocks, each followed by its trailing product",
                            "sweep_gbs_over_stage": sweep_bytes / q_s / 1e9, "hbm_peak_gbs": hbm,
                            "sweep_frac_over_stage": sweep_bytes / q_s / 1e9 / hbm,
+                           "sweep_issued_gbs_over_stage": sweep_issued / q_s / 1e9,
                            "trailing_tflops_over_stage": t_flops / q_s / 1e12, "tensor_peak": sustained,
                            "trailing_frac_over_stage": t_flops / q_s / 1e12 / sustained,
                            "trailing_issued_tflops_over_stage": 3 * t_flops / q_s / 1e12,
-                           "work": f"sweep {sweep_bytes / 1e6:.1f} MB, trailing products {t_flops:.3e} flops "
-                                   "(3 tf32 passes issued), both over the whole stage time"},
+                           "work": f"sweep {sweep_bytes / 1e6:.1f} MB algorithmic ({sweep_issued / 1e6:.1f} MB "
+                                   f"issued), trailing products {t_flops:.3e} flops (3 tf32 passes issued), "
+                                   "both over the whole stage time"},
     }
 
 
