@@ -155,6 +155,13 @@ def cpu_sample(problem, x0, rows=64):
     import oracle
     from post_weight_quantization_05_b200 import synth
     cores = len(os.sched_getaffinity(0))
+    try:   # the oracle's parallel work is its BLAS / LAPACK calls: report that pool's threads
+        from threadpoolctl import threadpool_info
+        pools = [i.get("num_threads") or 0 for i in threadpool_info() if i.get("user_api") == "blas"]
+        if pools:
+            cores = min(cores, max(pools))
+    except Exception:   # noqa: BLE001 -- without threadpoolctl the affinity count stands
+        pass
     xf = synth.x_as_f32(problem, x0)
     t0 = time.perf_counter()
     H = oracle.hessian([xf])
