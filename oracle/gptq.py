@@ -55,7 +55,7 @@ __all__ = [
     "grid_params", "quant_codes", "dequant", "gptq_quantize", "rtn_quantize",
     "pack_codes", "unpack_codes", "layer_loss_direct", "layer_loss_hessian",
     "obq_fixed_order_row", "least_squares_refit", "act_order_perm", "gptq_quantize_act_order",
-    "dequant_gemv",
+    "dequant_gemv", "gptq_quantize_deferred",
 ]
 
 FP16_MIN_NORMAL = 2.0 ** -14
@@ -220,6 +220,61 @@ def gptq_quantize(W, U, bits: int = 4, blocksize: int = 128, groupsize: int = -1
         out["W_at"] = W_at
         out["E"] = E_all
     return out
+
+
+def gptq_quantize_deferred(W, U, bits: int = 4, blocksize: int = 128, groupsize: int = -1,
+                           superblock: int = 4):
+    """A cross-check, not the pages' order: the same sweep with the trailing
+    update deferred.  After each block, E updates only the rest of its
+    super-block (`superblock` blocks); the columns beyond the super-block get
+    one product with the super-block's whole E.  The trailing update is
+    linear, so in exact arithmetic every column holds the same values when it
+    is quantized as in gptq_quantize.  A group grid is taken from the columns
+    of its group, which must therefore not reach past the super-block: the
+    group size has to divide superblock * blocksize (or the grid is per row).
+    Returns codes, scales, zeros and Q as gptq_quantize does."""
+    W = np.array(W, dtype=np.float64, copy=True)
+    U = np.asarray(U, dtype=np.float64)
+    d_out, d_in = W.shape
+    B = int(blocksize)
+    SB = int(superblock) * B
+    if groupsize > 0 and SB % groupsize != 0:
+        raise ValueError("the group size must divide the super-block width")
+    n_groups = 1 if groupsize <= 0 else -(-d_in // groupsize)
+    scales = np.zeros((d_out, n_groups), dtype=np.float32)
+    zeros = np.zeros((d_out, n_groups), dtype=np.float32)
+    codes = np.zeros((d_out, d_in), dtype=np.int64)
+    Q = np.zeros((d_out, d_in), dtype=np.float64)
+    if groupsize <= 0:
+        s, z = grid_params(*_row_minmax(W), bits)
+        scales[:, 0], zeros[:, 0] = s, z
+    for s1 in range(0, d_in, SB):
+        s2 = min(s1 + SB, d_in)
+        E_sb = np.zeros((d_out, s2 - s1), dtype=np.float64)
+        for i1 in range(s1, s2, B):
+            i2 = min(i1 + B, s2)
+            W1 = W[:, i1:i2].copy()
+            for j in range(i2 - i1):
+                col = i1 + j
+                if groupsize > 0 and col % groupsize == 0:    # the group lies inside [col, s2)
+                    g_end = min(col + groupsize, d_in)
+                    cur = np.concatenate([W1[:, j:], W[:, i2:s2]], axis=1)[:, :g_end - col]
+                    s, z = grid_params(*_row_minmax(cur), bits)
+                    scales[:, col // groupsize], zeros[:, col // groupsize] = s, z
+                w = W1[:, j]
+                c = quant_codes(w, s, z, bits)
+                q = dequant(c, s, z)
+                codes[:, col] = c
+                Q[:, col] = q
+                err = (w - q) / U[col, col]
+                W1[:, j:] -= np.outer(err, U[col, col:i2])
+                E_sb[:, col - s1] = err
+            W[:, i1:i2] = W1
+            if i2 < s2:                                       # the rest of the super-block only
+                W[:, i2:s2] -= E_sb[:, i1 - s1:i2 - s1] @ U[i1:i2, i2:s2]
+        if s2 < d_in:                                         # the far tail, once per super-block
+            W[:, s2:] -= E_sb @ U[s1:s2, s2:]
+    return {"codes": codes, "scales": scales, "zeros": zeros, "Q": Q}
 
 
 # ---------------------------------------------------------------------------

@@ -188,6 +188,32 @@ def test_obq_elimination_form_equals_sweep():
             assert np.max(np.abs(w_at - out["W_at"][r])) < 1e-12
 
 
+def test_deferred_trailing_update_is_exact():
+    """The deferred trailing update (each block's E applied to the rest of its
+    super-block, the far tail once per super-block with the super-block's
+    whole E) gives the per-block sweep's codes and grids, and Q to 1e-10: the
+    update is linear.  One super-block spanning the whole layer (no far
+    update at all) and one block per super-block (every update a far one)
+    are both covered.  A group that would reach past its super-block is
+    refused."""
+    W, X = _small_problem(d_out=20, d_in=96, n=400, seed=21)
+    H, Hd, lam, U = _factor(X)
+    checked = 0
+    for g in (-1, 16, 32):
+        ref = oracle.gptq_quantize(W, U, 4, 8, groupsize=g)
+        for K in (1, 2, 4, 12):                              # super-blocks of 8, 16, 32, 96 columns
+            if g > 0 and (8 * K) % g:
+                with pytest.raises(ValueError):
+                    oracle.gptq_quantize_deferred(W, U, 4, 8, groupsize=g, superblock=K)
+                continue
+            out = oracle.gptq_quantize_deferred(W, U, 4, 8, groupsize=g, superblock=K)
+            assert np.array_equal(out["codes"], ref["codes"]), (g, K)
+            assert np.array_equal(out["scales"], ref["scales"]) and np.array_equal(out["zeros"], ref["zeros"])
+            assert np.max(np.abs(out["Q"] - ref["Q"])) < 1e-10
+            checked += 1
+    assert checked == 4 + 3 + 2
+
+
 def test_lazy_batch_is_exact():
     """T3: B = 1 (unblocked), B = 4 and B = 128 give the same result."""
     W, X = _small_problem(d_out=20, d_in=48, n=200, seed=9)
