@@ -55,7 +55,8 @@ __all__ = [
     "grid_params", "quant_codes", "dequant", "gptq_quantize", "rtn_quantize",
     "pack_codes", "unpack_codes", "layer_loss_direct", "layer_loss_hessian",
     "obq_fixed_order_row", "least_squares_refit", "act_order_perm", "gptq_quantize_act_order",
-    "dequant_gemv", "gptq_quantize_deferred",
+    "dequant_gemv", "gptq_quantize_deferred", "grid_params_working_precision",
+    "quant_codes_working_precision",
 ]
 
 FP16_MIN_NORMAL = 2.0 ** -14
@@ -140,6 +141,26 @@ def grid_params(wmin, wmax, bits: int):
     return s, z
 
 
+def grid_params_working_precision(wmin, wmax, bits: int):
+    """Scale and zero as the page's minimal quantizer forms them ([wiki]
+    "최소 구현"): scale = max(wmax - wmin, 1e-8) / maxq and zero =
+    round(-wmin / scale), both kept in the working precision (fp64 here), with
+    no fp16 storage.  This is reading B, used only to compare the oracle with a
+    direct run of those steps; the codes the library stores use reading R5."""
+    maxq = float(2 ** bits - 1)
+    wmin = np.asarray(wmin, dtype=np.float64)
+    wmax = np.asarray(wmax, dtype=np.float64)
+    s = np.maximum(wmax - wmin, 1e-8) / maxq
+    return s, np.rint(-wmin / s)
+
+
+def quant_codes_working_precision(w, s, z, bits: int) -> np.ndarray:
+    """c = clamp(round(w / s) + z, 0, maxq) in fp64 (reading B)."""
+    maxq = float(2 ** bits - 1)
+    t = np.rint(np.asarray(w, dtype=np.float64) / np.asarray(s, dtype=np.float64))
+    return np.clip(t + np.asarray(z, dtype=np.float64), 0.0, maxq).astype(np.int64)
+
+
 def quant_codes(w, s, z, bits: int) -> np.ndarray:
     """Integer codes c = clamp(rint(w/s) + z, 0, maxq), decided in fp32 (R4)."""
     maxq = np.float32(2 ** bits - 1)
@@ -165,14 +186,20 @@ def _row_minmax(A):
 # batch of B columns followed by one matrix product for the rest)
 # ---------------------------------------------------------------------------
 def gptq_quantize(W, U, bits: int = 4, blocksize: int = 128, groupsize: int = -1,
-                  return_trace: bool = False):
+                  return_trace: bool = False, grid: str = "fp16"):
     """Algorithm 1 step by step, vectorised over rows.
+
+    grid = "fp16" (the default): reading R5, the grid the library stores.
+    grid = "working": reading B, the page's minimal quantizer's own grid (one
+    per row, scale and zero kept in fp64, decisions in fp64); per-row grids
+    only.  It exists to compare the oracle with a direct run of those steps.
 
     W [d_out, d_in] (any float, widened to fp64), U upper [d_in, d_in] with
     U^T U = (H + lambda I)^-1.  Returns a dict with codes (int64 [d_out, d_in]),
     scales/zeros (float32 values of the fp16 grid, [d_out, n_groups]),
     Q (fp64 dequantized weights) and, if return_trace, the weight each column
-    had when it was quantized (W_at) and the error matrix E [d_out, d_in]."""
+    had when it was quantized (W_at), the error matrix E [d_out, d_in] and the
+    fp32 min / max each grid was set from (gmin, gmax [d_out, n_groups])."""
     W = np.array(W, dtype=np.float64, copy=True)
     U = np.asarray(U, dtype=np.float64)
     d_out, d_in = W.shape
@@ -184,9 +211,22 @@ def gptq_quantize(W, U, bits: int = 4, blocksize: int = 128, groupsize: int = -1
     Q = np.zeros((d_out, d_in), dtype=np.float64)
     W_at = np.zeros((d_out, d_in), dtype=np.float64) if return_trace else None
     E_all = np.zeros((d_out, d_in), dtype=np.float64) if return_trace else None
+    gmin = np.zeros((d_out, n_groups), dtype=np.float32)   # the fp32 min / max each grid was set from
+    gmax = np.zeros((d_out, n_groups), dtype=np.float32)
 
-    if groupsize <= 0:                                   # reading R6: original W
-        s, z = grid_params(*_row_minmax(W), bits)
+    working = grid == "working"
+    if working:
+        if groupsize > 0:
+            raise ValueError("the working-precision grid is one grid per row")
+        scales = scales.astype(np.float64)
+        zeros = zeros.astype(np.float64)
+        s, z = grid_params_working_precision(W.min(axis=1), W.max(axis=1), bits)
+        scales[:, 0], zeros[:, 0] = s, z
+    elif grid != "fp16":
+        raise ValueError(grid)
+    elif groupsize <= 0:                                 # reading R6: original W
+        gmin[:, 0], gmax[:, 0] = _row_minmax(W)
+        s, z = grid_params(gmin[:, 0], gmax[:, 0], bits)
         scales[:, 0], zeros[:, 0] = s, z
 
     for i1 in range(0, d_in, B):
@@ -198,10 +238,12 @@ def gptq_quantize(W, U, bits: int = 4, blocksize: int = 128, groupsize: int = -1
             if groupsize > 0 and col % groupsize == 0:    # R6: latest updated weights
                 g_end = min(col + groupsize, d_in)
                 cur = np.concatenate([W1[:, j:], W[:, i2:]], axis=1)[:, :g_end - col]
-                s, z = grid_params(*_row_minmax(cur), bits)
-                scales[:, col // groupsize], zeros[:, col // groupsize] = s, z
+                gi = col // groupsize
+                gmin[:, gi], gmax[:, gi] = _row_minmax(cur)
+                s, z = grid_params(gmin[:, gi], gmax[:, gi], bits)
+                scales[:, gi], zeros[:, gi] = s, z
             w = W1[:, j]
-            c = quant_codes(w, s, z, bits)
+            c = quant_codes_working_precision(w, s, z, bits) if working else quant_codes(w, s, z, bits)
             q = dequant(c, s, z)
             codes[:, col] = c
             Q[:, col] = q
@@ -219,6 +261,8 @@ def gptq_quantize(W, U, bits: int = 4, blocksize: int = 128, groupsize: int = -1
     if return_trace:
         out["W_at"] = W_at
         out["E"] = E_all
+        out["gmin"], out["gmax"] = gmin, gmax
+        out["bits"] = int(bits)
     return out
 
 

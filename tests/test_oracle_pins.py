@@ -632,3 +632,94 @@ def test_planted_gemv_mistakes_are_caught(mistake, monkeypatch, golden_dir):
         except AssertionError:
             caught += 1
     assert caught >= 1
+
+
+# ---------------------------------------------------------------- the page's own minimal quantizer
+def _page_minimal_quantizer_f64(W, X, bits, blocksize, percdamp):
+    """The steps of [wiki] "최소 구현" run directly in torch float64 on the CPU
+    (a second, independent restatement: torch's own Cholesky, Cholesky-inverse
+    and products, nothing from the oracle): one asymmetric grid per row from
+    the original weights, H = 2 X^T X damped by percdamp of its mean diagonal,
+    the upper Cholesky factor of its inverse, then per block the column loop
+    (quantize, error over the diagonal entry, in-block correction) and one
+    product for the columns after the block.  Returns the dequantized weights."""
+    import torch
+    W = torch.tensor(np.asarray(W, dtype=np.float64))
+    X = torch.tensor(np.asarray(X, dtype=np.float64))
+    d = W.shape[1]
+    top = float(2 ** bits - 1)
+    lo, hi = W.amin(dim=1), W.amax(dim=1)
+    step = torch.clamp(hi - lo, min=1e-8) / top
+    offset = torch.round(-lo / step)
+    H = 2.0 * (X.T @ X)
+    H = H + percdamp * torch.diagonal(H).mean() * torch.eye(d, dtype=torch.float64)
+    R = torch.linalg.cholesky(torch.cholesky_inverse(torch.linalg.cholesky(H)), upper=True)
+    Q = torch.zeros_like(W)
+    for a in range(0, d, blocksize):
+        b = min(a + blocksize, d)
+        panel = W[:, a:b].clone()
+        errs = torch.zeros_like(panel)
+        for k in range(b - a):
+            col = panel[:, k]
+            lvl = torch.clamp(torch.round(col / step) + offset, 0.0, top)
+            qcol = step * (lvl - offset)
+            Q[:, a + k] = qcol
+            e = (col - qcol) / R[a + k, a + k]
+            panel[:, k:] -= torch.outer(e, R[a + k, a + k:b])
+            errs[:, k] = e
+        W[:, b:] -= errs @ R[a:b, b:]
+    return Q.numpy()
+
+
+@pytest.mark.parametrize("d_out,d_in,n,bits,blocksize", [(48, 64, 400, 4, 128), (40, 96, 500, 3, 32),
+                                                         (32, 64, 300, 2, 16)])
+def test_oracle_reproduces_the_page_minimal_quantizer(d_out, d_in, n, bits, blocksize):
+    """T6: with the page's own grid (scale and zero kept in the working
+    precision, reading B) the oracle gives the same dequantized weights as the
+    page's minimal quantizer run in float64, up to the order of rounding."""
+    rng = np.random.default_rng(60 + d_in + bits)
+    X = synth.ar1_rows(rng, n, d_in, 0.9).astype(np.float64)
+    W = rng.standard_normal((d_out, d_in)) * 0.02
+    Q_page = _page_minimal_quantizer_f64(W, X, bits, blocksize, 0.01)
+    Hd, _ = oracle.damp(oracle.hessian([X]), 0.01)
+    U = oracle.hinv_upper_factor(Hd)
+    out = oracle.gptq_quantize(W, U, bits, blocksize, -1, grid="working")
+    assert np.max(np.abs(out["Q"] - Q_page)) <= 1e-12
+    # and the stored-grid default differs from it only through the fp16 grid:
+    # the same sweep on the page's grid values would be the page's result
+    s, z = oracle.grid_params_working_precision(W.min(1), W.max(1), bits)
+    assert np.array_equal(out["scales"][:, 0], s) and np.array_equal(out["zeros"][:, 0], z)
+
+
+def test_page_minimal_quantizer_restatement_is_not_the_fp16_grid():
+    """Control: the two readings of the grid really differ (so the comparison
+    above checks the sweep, not a coincidence of grids)."""
+    rng = np.random.default_rng(7)
+    X = synth.ar1_rows(rng, 400, 64, 0.9).astype(np.float64)
+    W = rng.standard_normal((48, 64)) * 0.02
+    Q_page = _page_minimal_quantizer_f64(W, X, 4, 128, 0.01)
+    Hd, _ = oracle.damp(oracle.hessian([X]), 0.01)
+    out = oracle.gptq_quantize(W, oracle.hinv_upper_factor(Hd), 4, 128, -1)
+    assert np.max(np.abs(out["Q"] - Q_page)) > 1e-6
+
+
+def test_planted_sweep_mistake_breaks_the_page_cross_check(monkeypatch):
+    """Planted in the oracle: the in-block correction skips the next column.
+    The cross-check with the page's quantizer must catch it."""
+    rng = np.random.default_rng(61)
+    X = synth.ar1_rows(rng, 400, 64, 0.9).astype(np.float64)
+    W = rng.standard_normal((48, 64)) * 0.02
+    Q_page = _page_minimal_quantizer_f64(W, X, 4, 128, 0.01)
+    Hd, _ = oracle.damp(oracle.hessian([X]), 0.01)
+    U = oracle.hinv_upper_factor(Hd)
+    real_outer = np.outer
+
+    def outer_skipping_next(a, b):
+        o = real_outer(a, b)
+        if o.shape[1] > 1:
+            o[:, 1] = 0.0
+        return o
+    monkeypatch.setattr(np, "outer", outer_skipping_next)
+    out = oracle.gptq_quantize(W, U, 4, 128, -1, grid="working")
+    monkeypatch.setattr(np, "outer", real_outer)
+    assert np.max(np.abs(out["Q"] - Q_page)) > 1e-6
