@@ -199,6 +199,31 @@ def test_prepare_hinv(d, rho):
     assert rel_fro(U, Uref) <= U_TOL
 
 
+@pytest.mark.parametrize("d", [2048, 4096])
+def test_prepare_hinv_is_deterministic(d):
+    """The factorization's streams update shared block columns: U must still
+    be the same bits on every call (here three calls, on two streams)."""
+    p = synth.custom("det", 8, d, 2 * d, rho=0.9, x_dtype="bf16", layer=3 * d)
+    H = torch.zeros((d, d), dtype=torch.float32, device="cuda")
+    api.hessian_accumulate(to_dev_x(p, p.x_batch(0)), H)
+    ws = api.workspace(api.prepare_hinv_workspace_size(d), "cuda")
+    Us = []
+    side = torch.cuda.Stream()
+    for i in range(3):
+        U = torch.empty((d, d), dtype=torch.float32, device="cuda")
+        if i == 1:
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                api.prepare_hinv(H, U, ws, 0.01, None)
+            torch.cuda.current_stream().wait_stream(side)
+        else:
+            api.prepare_hinv(H, U, ws, 0.01, None)
+        api.get_status()
+        Us.append(U)
+    assert torch.equal(Us[0].view(torch.int32), Us[1].view(torch.int32))
+    assert torch.equal(Us[0].view(torch.int32), Us[2].view(torch.int32))
+
+
 def test_prepare_hinv_not_positive_definite():
     d = 256
     Ht = torch.zeros((d, d), dtype=torch.float32, device="cuda")    # X == 0 -> H = 0, lambda = 0
@@ -364,7 +389,13 @@ def _oracle_h_syrk(p, xs):
     return np.triu(Hu) + np.triu(Hu, 1).T
 
 
-def _full_size_check(p, n_rows_sample=48, seed=0, match=CODE_MATCH):
+def _full_size_check(p, n_rows_sample=48, seed=0, match=CODE_MATCH, sweep_rows=64):
+    """End to end at full size (the launch configuration the benchmark uses):
+    H and U against the fp64 oracle in full, codes and loss on sampled rows.
+    Then the sweep alone at the same shape: the GPU's sweep and the oracle's
+    on one common U (the oracle's, rounded to fp32, fed to both) for
+    `sweep_rows` sampled rows, held to the code criteria without exception.
+    Returns (end-to-end identical fraction, sweep-alone identical fraction)."""
     xs = synth.x_batches_threaded(p, 8)
     lq = _gpu_pipeline(p, [to_dev_x(p, x) for x in xs], want_q=False)
     H = _oracle_h_syrk(p, xs)
@@ -372,6 +403,7 @@ def _full_size_check(p, n_rows_sample=48, seed=0, match=CODE_MATCH):
     assert rel_fro(upper(lq.H.cpu().numpy()), upper(H)) <= H_TOL
     Hd, _ = oracle.damp(H, p.percdamp)
     U = oracle.hinv_upper_factor_ul(Hd)
+    del Hd
     assert rel_fro(lq.U.cpu().numpy(), U) <= U_TOL
     rows = np.random.default_rng(seed).choice(p.d_out, size=n_rows_sample, replace=False)
     ref = oracle.gptq_quantize(p.W[rows], U, p.bits, 128, p.groupsize, return_trace=True)
@@ -383,14 +415,32 @@ def _full_size_check(p, n_rows_sample=48, seed=0, match=CODE_MATCH):
     lg = oracle.layer_loss_hessian(p.W[rows], Qg, H)
     lo = oracle.layer_loss_hessian(p.W[rows], ref["Q"], H)
     assert abs(lg / lo - 1.0) <= LOSS_TOL, (lg, lo)
-    return frac
+    del lq
+    torch.cuda.empty_cache()
+    # the sweep alone on one common U
+    U32 = U.astype(np.float32)
+    del U
+    srows = np.random.default_rng(seed + 1).choice(p.d_out, size=sweep_rows, replace=False)
+    ref_s = oracle.gptq_quantize(p.W[srows], U32.astype(np.float64), p.bits, 128, p.groupsize, return_trace=True)
+    codes, scales, zeros, _, _ = _gpu_quantize(p.W[srows], U32, p.bits, p.groupsize, want_q=False)
+    got_s = unpack_gpu_codes(codes, p.bits, p.d_in)
+    ss, zs = fp16_values(scales), fp16_values(zeros)
+    frac_s = check_codes(got_s, ref_s, p.name + " (sweep alone)", groupsize=p.groupsize, gpu_scales=ss,
+                         gpu_zeros=zs)
+    Qs = dequant_rows(got_s, ss, zs, p.groupsize)
+    lg = oracle.layer_loss_hessian(p.W[srows], Qs, H)
+    lo = oracle.layer_loss_hessian(p.W[srows], ref_s["Q"], H)
+    assert abs(lg / lo - 1.0) <= LOSS_TOL, (lg, lo)
+    print(f"{p.name}: end to end {frac:.5f} of sampled codes identical; sweep alone {frac_s:.5f}")
+    return frac, frac_s
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("which,bits", [("up", 4), ("down", 3)])
+@pytest.mark.parametrize("which,bits", [("up", 3), ("up", 4), ("down", 3), ("down", 4)])
 def test_mlp11008_full_size_sampled_rows(which, bits):
     """The Llama-7B MLP pair with heavy-tailed (Student-t) activations and 1%
-    outlier channels x20, 65536 calibration rows."""
+    outlier channels x20, 65536 calibration rows: up- and down-projection, each
+    at 3 and 4 bits."""
     _full_size_check(synth.mlp11008(which, bits))
 
 
@@ -403,12 +453,13 @@ def test_mlp28672_full_size_sampled_rows():
     the compensated weights), and the GPU's H -- fp32 accumulation, relative
     error ~6e-7, well inside its 1e-5 bound -- already moves about one row in
     eight across a near-tie even with an exact factorization.  So for this
-    workload the identical-code fraction is reported, not asserted; every row
-    must still agree with the oracle up to its first difference, that first
-    difference must be a one-level flip at a near-tie, and the layer loss must
-    be within 0.5% of the oracle's."""
-    frac = _full_size_check(synth.mlp28672(), n_rows_sample=16, match=0.0)
-    print(f"mlp28672: {frac:.4f} of sampled codes identical")
+    workload the end-to-end identical-code fraction is reported, not asserted;
+    every row must still agree with the oracle up to its first difference,
+    that first difference must be a one-level flip at a near-tie, and the
+    layer loss must be within 0.5% of the oracle's.  The sweep alone, on one
+    common U, is held to the full code criteria (>= 99.9% identical)."""
+    frac, frac_s = _full_size_check(synth.mlp28672(), n_rows_sample=16, match=0.0)
+    assert frac_s >= CODE_MATCH
 
 
 @pytest.mark.slow

@@ -1,13 +1,16 @@
 """The allocation-free quantize entry point (gptq_quantize_layer_noalloc).
 
 Some callers cannot allocate device memory at the point where they quantize:
-code recording into a CUDA stream capture, where cudaMalloc is not allowed,
-or a framework whose memory pool owns every device buffer and hands out only
-inputs and outputs.  This entry point takes no workspace and keeps its scratch
-in a fixed array inside the library.  These tests call it through the C ABI
-and compare it with gptq_quantize_layer (which takes a caller workspace) on
-the same inputs, twice in a row so that the second call starts from the
-scratch the first one left behind.  This file is named to be collected last.
+a framework whose memory pool owns every device buffer and hands out only
+inputs and outputs, or a serving process that reserves its whole memory
+budget at start-up and may not call cudaMalloc afterwards (the call can fail
+once the budget is taken, and it synchronizes the device).  This entry point
+takes no workspace and keeps its scratch in a fixed array inside the library.
+These tests call it through the C ABI and compare it with gptq_quantize_layer
+(which takes a caller workspace) on the same inputs, twice in a row so that
+the second call starts from the scratch the first one left behind.  Both run
+the same kernels on the same inputs, so their results must be identical bit
+for bit.  This file is named to be collected last.
 """
 import ctypes
 
@@ -17,7 +20,7 @@ import torch
 
 import oracle
 from post_weight_quantization_05_b200 import _native, api, build_lib, synth
-from parity_util import CODE_MATCH, check_codes, fp16_values, unpack_gpu_codes
+from parity_util import check_codes, fp16_values, unpack_gpu_codes
 
 pytestmark = pytest.mark.gpu
 
@@ -69,17 +72,13 @@ def test_noalloc_matches_workspace_entry_point(lib, d_out, d_in, bits, groupsize
                                              _ptr(got[0]), _ptr(got[1]), _ptr(got[2]), _ptr(got[3]), stream)
         assert rc == 0
         assert api.get_status() == (0, 0)
-        c_ref = unpack_gpu_codes(ref[0], bits, d_in)
+        # the same kernels on the same inputs: identical bits everywhere
+        assert torch.equal(got[0], ref[0])
+        assert torch.equal(got[1].view(torch.int16), ref[1].view(torch.int16))
+        assert torch.equal(got[2].view(torch.int16), ref[2].view(torch.int16))
+        assert torch.equal(got[3].view(torch.int32), ref[3].view(torch.int32))
+        assert torch.equal(W_na.view(torch.int32), W_ref.view(torch.int32))
         c_got = unpack_gpu_codes(got[0], bits, d_in)
-        # same kernels on the same inputs: held to the code-parity tolerance the
-        # other tests use (in practice identical)
-        frac = float(np.mean(c_got == c_ref))
-        assert frac >= CODE_MATCH and np.abs(c_got - c_ref).max() <= 1
-        assert np.array_equal(fp16_values(got[1]), fp16_values(ref[1]))
-        assert np.array_equal(fp16_values(got[2]), fp16_values(ref[2]))
-        q_ref, q_got = ref[3].cpu().numpy(), got[3].cpu().numpy()
-        assert np.isfinite(q_got).all()
-        assert np.mean(q_got == q_ref) >= CODE_MATCH
         # and against the oracle, like the workspace path
         ref_o = oracle.gptq_quantize(p.W, U, bits, 128, groupsize, return_trace=True)
         check_codes(c_got, ref_o, "noalloc", groupsize=groupsize, gpu_scales=fp16_values(got[1]),
