@@ -137,7 +137,9 @@ int gptq_hessian_accumulate_batches(const void* const* X, const int64_t* n, int 
  *   ws       >= gptq_prepare_hinv_workspace_size(d_in) bytes.
  * The work forks from `stream` onto three library-owned streams (the
  * factorization's chain, its look-ahead updates, the inverse) and joins back
- * before the call's last kernel; later work on `stream` sees U complete.  A
+ * before the call's last kernel; later work on `stream` sees U complete.
+ * Deterministic: every element receives its updates in a fixed order, so the
+ * same H gives the same U bit for bit on every call.  A
  * device has four such sets.  A caller stream keeps the set it got first, so
  * calls on up to four different streams run concurrently (independent
  * layers); further streams share the sets, and calls sharing a set run one
@@ -189,9 +191,11 @@ int gptq_quantize_layer(float* W, int64_t d_out, int64_t d_in, const float* U,
 /* ------------------------------------------------------------------------
  * Stages 3-5 without a caller workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory where
- * they quantize -- code recording into a CUDA stream capture (cudaMalloc is
- * not allowed there) or a host framework whose memory pool owns every device
- * buffer and hands out only inputs and outputs.
+ * they quantize -- a host framework whose memory pool owns every device
+ * buffer and hands out only inputs and outputs, or a serving process that
+ * reserves its memory budget at start-up and may not call cudaMalloc later
+ * (the call can fail once the budget is taken, and it synchronizes the
+ * device).
  *
  * Same arguments, results and errors as gptq_quantize_layer, minus ws and
  * ws_bytes.  The scratch it needs (E [d_out, 128] and U^T [d_in, d_in], each

@@ -583,12 +583,8 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         const int k0 = k * NB;
         float* dk = Dinv + size_t(k) * NB * NB;
         // Block k needs every far update j <= k - NEAR - 1 (side stream, see
-        // below).  One wait every NEAR steps, for the far update of two steps
-        // back, covers all of them (the side stream runs in order) and keeps
-        // the other steps' kernels back to back for programmatic launch.
-        if (k % NEAR == 0 && k >= 2 &&
-            cudaStreamWaitEvent(stream, aux->far_done[(k - 2) % AuxStream::RING], 0) != cudaSuccess)
-            return GPTQ_ERR_CUDA;
+        // below); the wait before step k - 1's near update (below) has already
+        // ordered them before this kernel.
         if (launch_pdl(potrf_diag_kernel, dim3(1), dim3(DIAG_THREADS), DIAG_SMEM, stream, static_cast<const float*>(A), d,
                        k0, dk, Z, info, st) != cudaSuccess)
             return GPTQ_ERR_CUDA;
@@ -607,14 +603,19 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
             return GPTQ_ERR_CUDA;
         if (rest > 0) {
             // the next NEAR block columns (they hold the next diagonal blocks) on
-            // `stream` ...
+            // `stream` ...  Column block k + NEAR enters this window now: until
+            // step k - 1 it was updated by the side stream.  Waiting for step
+            // k - 1's far update (the side stream runs in order, so it is the
+            // last one) makes every element receive its updates in step order,
+            // so U does not depend on how the two streams interleave.
+            if (k >= 1 && cudaStreamWaitEvent(stream, aux->far_done[(k - 1) % AuxStream::RING], 0) != cudaSuccess)
+                return GPTQ_ERR_CUDA;
             const int near_cols = std::min(rest, NEAR * NB);
             float* next = A + size_t(k0 + NB) * d + k0 + NB;
             rc = launch_tgemm(rest, near_cols, NB, -1.0f, panel, nullptr, d, panel, nullptr, d, true, next, d, true,
                               stream, st);
             if (rc) return rc;
-            // ... the columns after them on `ss` (reduce-adds into regions the
-            // next update may also be adding to: each element's add is atomic)
+            // ... the columns after them on `ss`, beside the next steps' chain
             if (rest > NEAR * NB) {
                 if (cudaStreamWaitEvent(ss, aux->step, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
                 const int f0 = k0 + (NEAR + 1) * NB;

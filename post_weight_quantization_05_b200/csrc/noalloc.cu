@@ -3,10 +3,11 @@
 // workspace.
 //
 // Who needs it: code that must not allocate device memory at the point where
-// it quantizes -- for example a caller recording into a CUDA stream capture,
-// where cudaMalloc is not allowed, or a host framework whose memory pool owns
-// every device buffer and hands out only inputs and outputs.  Such a caller
-// passes W, U and the outputs and nothing else.
+// it quantizes -- for example a host framework whose memory pool owns every
+// device buffer and hands out only inputs and outputs, or a serving process
+// that reserves its memory budget at start-up and may not call cudaMalloc
+// later (the call can fail once the budget is taken, and it synchronizes the
+// device).  Such a caller passes W, U and the outputs and nothing else.
 //
 // The scratch is one file-scope device array of kNoAllocScratchBytes, held
 // by every GPU that loads this library until the process exits.  It holds the
