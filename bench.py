@@ -45,23 +45,33 @@ WORKLOAD = ("attn4096: W [4096,4096] bf16 ~N(0,0.02^2), X [262144,4096] bf16 AR(
             "in 16 batches of 16384, 4-bit, groupsize 128, B=128, percdamp 0.01")
 
 
-def syrk_traffic_per_launch():
-    """DRAM bytes (read + write) of one X^T X launch from the committed ncu
-    summary, or None if the kernel's sources changed since that capture."""
+def source_hash(files, recorded=None):
+    """sha256 (16 hex digits) over the named files of the CUDA sources, in
+    order; with `recorded` (a dict file -> hash recorded when a profile was
+    captured), over those recorded per-file hashes instead."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "syrk_pair_kernel_attn4096.md")
-    try:
-        text = open(path).read()
-    except OSError:
-        return None
-    vals = dict(line.split(": ", 1) for line in text.splitlines() if line.startswith(("traffic_", "kernel_source")))
     h = hashlib.sha256()
-    for f in ("hessian.cu", "common.cuh"):
-        with open(os.path.join(ROOT, "post_weight_quantization_05_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    if vals.get("kernel_source_hash") != h.hexdigest()[:16]:
+    for f in files:
+        if recorded is not None:
+            h.update(recorded[f].encode())
+        else:
+            with open(os.path.join(ROOT, "post_weight_quantization_05_b200", "csrc", f), "rb") as fh:
+                h.update(hashlib.sha256(fh.read()).hexdigest()[:16].encode())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name):
+    """DRAM bytes (read + write) per launch of a kernel from its committed
+    profile record (profiles/<name>.json, written by profile_summary.py from
+    the ncu capture), or None if the kernel's sources changed since."""
+    try:
+        with open(os.path.join(ROOT, "profiles", name + ".json")) as f:
+            rec = json.load(f)
+        if rec["source_hash"] != source_hash(rec["source_files"]):
+            return None
+        return int(rec["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
         return None
-    return int(vals["traffic_bytes_per_launch"])
 
 
 def peaks():
@@ -146,61 +156,104 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-# --------------------------------------------------------------------------- the oracle (CPU) sample
-def cpu_sample(problem, x0, rows=64):
-    """Time the fp64 oracle on a bounded sample of the workload: one of the
-    16 calibration batches (x16), the full factorization, and the sweep on
-    `rows` of the 4096 rows (x 4096/rows).  Returns (seconds per layer
-    estimate, description, cores)."""
-    import oracle
-    from post_weight_quantization_05_b200 import synth
+# --------------------------------------------------------------------------- the oracle on the host cores
+def oracle_cores():
+    """Threads the oracle's parallel work (its BLAS / LAPACK calls) runs on,
+    capped by the process's CPU affinity; its own Python loops run on one."""
     cores = len(os.sched_getaffinity(0))
-    try:   # the oracle's parallel work is its BLAS / LAPACK calls: report that pool's threads
+    try:
         from threadpoolctl import threadpool_info
         pools = [i.get("num_threads") or 0 for i in threadpool_info() if i.get("user_api") == "blas"]
         if pools:
             cores = min(cores, max(pools))
     except Exception:   # noqa: BLE001 -- without threadpoolctl the affinity count stands
         pass
-    xf = synth.x_as_f32(problem, x0)
+    return cores
+
+
+def oracle_full_layer(problem, xs_host):
+    """The fp64 oracle on the whole workload, once, unsampled: H over every
+    calibration row, the damping and the pages' factorization chain, and the
+    sweep over every row.  Returns (seconds per stage, cores)."""
+    import oracle
+    from post_weight_quantization_05_b200 import synth
     t0 = time.perf_counter()
-    H = oracle.hessian([xf])
+    H = None
+    for xb in xs_host:
+        xf = synth.x_as_f32(problem, xb)
+        if H is None:
+            H = np.zeros((problem.d_in, problem.d_in), dtype=np.float64)
+        oracle.hessian_accumulate(H, xf)
+        del xf
     t_h = time.perf_counter() - t0
     t0 = time.perf_counter()
     Hd, _ = oracle.damp(H, problem.percdamp)
     U = oracle.hinv_upper_factor(Hd)
     t_u = time.perf_counter() - t0
+    del Hd, H
     t0 = time.perf_counter()
-    oracle.gptq_quantize(problem.W[:rows], U, problem.bits, problem.blocksize, problem.groupsize)
+    oracle.gptq_quantize(problem.W, U, problem.bits, problem.blocksize, problem.groupsize)
     t_s = time.perf_counter() - t0
-    est = t_h * problem.n_batches + t_u + t_s * (problem.d_out / rows)
-    desc = (f"oracle fp64 on 1/{problem.n_batches} of the calibration rows (H, x{problem.n_batches}), "
-            f"full damp+factor chain, sweep on {rows}/{problem.d_out} rows (x{problem.d_out // rows}); "
-            f"measured {t_h:.1f}+{t_u:.1f}+{t_s:.1f} s")
-    return est, desc, cores
+    return {"hessian": t_h, "damp_factor": t_u, "sweep": t_s, "total": t_h + t_u + t_s}, oracle_cores()
+
+
+CYCLE = 16      # reference-arm steps per layer
 
 
 def run_reference(args):
-    """--impl reference: the oracle on the host cores, same metric/config."""
+    """--impl reference: the fp64 oracle on the host cores, same metric and
+    config.  One step is 1/16 of the layer, unsampled: the H of one of the 16
+    calibration batches and the sweep of 256 of the 4096 rows; every 16th
+    step also runs the damping and the pages' factorization chain on the H
+    accumulated over the previous 16 steps.  16 steps are one whole layer.
+    The sweeps use the U of the previous complete cycle (the first cycle's
+    comes from an untimed set-up factorization); rows are independent given
+    U, so the sweep's work does not depend on which U it uses."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    import oracle
     from post_weight_quantization_05_b200 import synth
     p = synth.attn4096()
-    x0 = p.x_batch(0)
-    for _ in range(args.warmup):
-        pass   # the oracle has no warm-up state; the sample below is timed as is
-    ests = []
-    desc = cores = None
-    for _ in range(max(1, args.steps)):
-        est, desc, cores = cpu_sample(p, x0)
-        ests.append(est)
-    sec = statistics.mean(ests)
-    value = p.d_out * p.d_in / sec
+    rows = p.d_out // CYCLE
+    xs = synth.x_batches_threaded(p, min(16, os.cpu_count() or 8))
+    # set-up (untimed): a U to sweep with in the first cycle
+    Hd, _ = oracle.damp(oracle.hessian([synth.x_as_f32(p, xs[0])]), p.percdamp)
+    U = oracle.hinv_upper_factor(Hd)
+    del Hd
+    H = np.zeros((p.d_in, p.d_in), dtype=np.float64)
+    times, stage = [], {"hessian": 0.0, "damp_factor": 0.0, "sweep": 0.0}
+    n_fact = 0
+    for i in range(args.steps):
+        b = i % CYCLE
+        t0 = time.perf_counter()
+        oracle.hessian_accumulate(H, synth.x_as_f32(p, xs[b]))
+        t1 = time.perf_counter()
+        oracle.gptq_quantize(p.W[b * rows:(b + 1) * rows], U, p.bits, p.blocksize, p.groupsize)
+        t2 = time.perf_counter()
+        t3 = t2
+        if b == CYCLE - 1:
+            Hd, _ = oracle.damp(H, p.percdamp)
+            U = oracle.hinv_upper_factor(Hd)
+            del Hd
+            H[:] = 0.0
+            n_fact += 1
+            t3 = time.perf_counter()
+        stage["hessian"] += t1 - t0
+        stage["sweep"] += t2 - t1
+        stage["damp_factor"] += t3 - t2
+        times.append(t3 - t0)
+    total = sum(times)
+    value = p.d_out * p.d_in * (len(times) / CYCLE) / total
+    cores = oracle_cores()
+    desc = (f"fp64 oracle, unsampled, in steps of 1/{CYCLE} layer: each step the H of one 16384-row batch and "
+            f"the sweep of {rows} of the {p.d_out} rows; every {CYCLE}th step the damping and the "
+            f"chol -> inverse -> chol chain ({n_fact} in these {len(times)} steps); {CYCLE} steps = one layer")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD},
+            "stage_s": stage,
             "cpu_baseline": {"value": value, "unit": "weights/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -218,6 +271,13 @@ def run_profile_case():
 
     from post_weight_quantization_05_b200 import api, build_lib, synth
     build_lib.build()
+    # the sources this capture runs, recorded beside it for the profile records
+    csrc = os.path.join(ROOT, "post_weight_quantization_05_b200", "csrc")
+    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+    import hashlib
+    with open(os.path.join(ROOT, "gpurun_out", "profile_sources.json"), "w") as f:
+        json.dump({fn: hashlib.sha256(open(os.path.join(csrc, fn), "rb").read()).hexdigest()[:16]
+                   for fn in sorted(os.listdir(csrc)) if fn.endswith((".cu", ".cuh", ".h"))}, f, indent=1)
     torch.cuda.set_device(0)
     p = synth.attn4096(n_batches=1)
     x = torch.from_numpy(p.x_batch(0).view(np.int16)).cuda().view(torch.bfloat16)
@@ -270,6 +330,8 @@ def main():
     ap.add_argument("--no-act-order", action="store_true")
     ap.add_argument("--no-gemv", action="store_true")
     ap.add_argument("--no-whole-model", action="store_true")
+    ap.add_argument("--no-shapes", action="store_true",
+                    help="skip the timings of the 11008-wide MLP pair and the 8192 x 28672 layer")
     ap.add_argument("--profile-case", action="store_true",
                     help="small case for ncu captures: one 16384-row batch of the same layer, 3 passes, no timing")
     args = ap.parse_args()
@@ -365,26 +427,33 @@ def main():
     ms_per_step = total_ms / args.steps
     value = job_throughput(p.d_out * p.d_in, world, args.steps, total_ms)
 
-    # roofline of the dominant kernel: the X^T X launch (one per batch)
+    # roofline of the dominant kernel: the X^T X launch (one per batch).  The
+    # timed region lasts well under a second (steps x ~6 ms), far from the
+    # seconds-long power-capped loop of the sustained figure: the burst peak applies.
     burst, sustained, hbm, src = peaks()
     n_b = p.batch_rows
     flops_per_launch = n_b * p.d_in * (p.d_in + 1)       # upper triangle incl. diagonal, 2 flops per MAC
     h_launch_avg = statistics.mean(h_launch_ms)
     achieved = flops_per_launch / (h_launch_avg / 1e3) / 1e12
+    timed_s = sum(step_ms) / 1e3
     roof = {"kernel": "hess::syrk_pair_kernel (tcgen05 cta_group::2)", "bound": "tensor", "achieved": achieved,
-            "peak": sustained, "unit": "TFLOP/s", "frac": achieved / sustained,
-            "peak_kind": f"bf16 dense sustained ({src})", "traffic": syrk_traffic_per_launch(),
+            "peak": burst, "unit": "TFLOP/s", "frac": achieved / burst,
+            "peak_kind": f"bf16 dense burst ({src}): the timed region lasts {timed_s:.2f} s",
+            "frac_of_sustained": achieved / sustained,
+            "traffic": profiled_traffic("syrk_pair_kernel_attn4096"),
             "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             "algorithmic_per_launch": f"{flops_per_launch:.4e} flop ({n_b}x{p.d_in}x{p.d_in + 1})",
+            "algorithmic_bytes_per_launch": n_b * p.d_in * 2 + 2 * (p.d_in * (p.d_in + 1) // 2) * 4,
             "avg_launch_ms": h_launch_avg}
 
-    stages = {"widen_W+zero_H": statistics.mean(begin_ms), "hessian_16_batches": statistics.mean(h_ms),
+    # stages: "begin" = widen W to its fp32 working copy and zero H; "hessian" = the 16 batches
+    stages = {"begin": statistics.mean(begin_ms), "hessian": statistics.mean(h_ms),
               "prepare_hinv": statistics.mean(prep_ms), "quantize_layer": statistics.mean(quant_ms)}
-    stages_median = {"widen_W+zero_H": statistics.median(begin_ms), "hessian_16_batches": statistics.median(h_ms),
+    stages_median = {"begin": statistics.median(begin_ms), "hessian": statistics.median(h_ms),
                      "prepare_hinv": statistics.median(prep_ms), "quantize_layer": statistics.median(quant_ms),
                      "step": statistics.median(step_ms),
                      "quantize_only": statistics.median([a + b for a, b in zip(prep_ms, quant_ms)])}
-    stage_roof = stage_rooflines(p, stages, burst, sustained, hbm)
+    stage_roof = stage_rooflines(p, stages, burst, hbm)
 
     # ---- the same layer with act-order (columns by descending diag(H))
     act = None
@@ -406,11 +475,18 @@ def main():
     if not args.no_e2e:
         e2e = end_to_end(p, xs_host, w_bits, lq, dev, args, world, dist if world > 1 else None)
 
+    # ---- the other layer shapes of the scope, timed the same way
+    shapes = None
+    if not args.no_shapes:
+        shapes = shape_timings(dev, stream, flush, args, api, burst, hbm)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        est, desc, cores = cpu_sample(p, xs_host[0])
-        cpu = {"value": p.d_out * p.d_in / est, "unit": "weights/s", "cores": cores, "kind": "oracle",
-               "sample": desc}
+        st_s, cores = oracle_full_layer(p, xs_host)
+        cpu = {"value": p.d_out * p.d_in / st_s["total"], "unit": "weights/s", "cores": cores, "kind": "oracle",
+               "sample": "the whole layer once, unsampled: H over all 262144 rows, damping and the pages' "
+                         "chol -> inverse -> chol chain, the sweep over all 4096 rows (fp64)",
+               "stage_s": st_s}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
@@ -424,8 +500,8 @@ def main():
                 "quantize_only_ms": stages["prepare_hinv"] + stages["quantize_layer"],
                 "stage_roofline": stage_roof, "roofline": roof,
                 "cpu_baseline": cpu,
-                "e2e": e2e, "gpu_launches": launches, "clocks": clk, "act_order": act, "dequant_gemv": gemv, "whole_model": whole,
-                "input_generation_s": gen_s}
+                "e2e": e2e, "gpu_launches": launches, "clocks": clk, "act_order": act, "dequant_gemv": gemv,
+                "whole_model": whole, "shapes": shapes, "input_generation_s": gen_s}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -433,16 +509,16 @@ def main():
     return 0
 
 
-def stage_rooflines(p, stages, burst, sustained, hbm):
+def stage_rooflines(p, stages, peak, hbm):
     """Each stage's algorithmic work over its own live event time, against
-    the measured peak of what bounds it.  The factorization and the sweep are
-    chains of dependent 128-column steps: their fractions say how far the
-    chain's latency keeps them from the hardware's rate, not how fast a
-    single kernel runs."""
+    the measured peak of what bounds it (bf16 burst for the tensor stages).
+    The factorization and the sweep are chains of dependent 128-column steps:
+    their fractions say how far the chain's latency keeps them from the
+    hardware's rate, not how fast a single kernel runs."""
     d_out, d_in, B = p.d_out, p.d_in, p.blocksize
     nb = d_in // B
     h_flops = p.n * d_in * (d_in + 1)                        # upper triangle incl. diagonal, 2 per MAC
-    h_tf = h_flops / (stages["hessian_16_batches"] / 1e3) / 1e12
+    h_tf = h_flops / (stages["hessian"] / 1e3) / 1e12
     # factorization as run: one Cholesky (d^3/3 flops) and one triangular inverse (d^3/3); U is
     # the inverse with both indices reversed (no flops).  The pages' literal chain would be 4/3 d^3.
     f_flops = 2.0 * d_in ** 3 / 3.0
@@ -457,24 +533,93 @@ def stage_rooflines(p, stages, burst, sustained, hbm):
     t_flops = sum(2.0 * d_out * (d_in - B * (i + 1)) * B for i in range(nb))
     q_s = stages["quantize_layer"] / 1e3
     return {
-        "hessian": {"bound": "tensor", "achieved": h_tf, "unit": "TFLOP/s", "peak": sustained,
-                    "frac": h_tf / sustained, "peak_kind": "bf16 dense sustained (measured)"},
-        "prepare_hinv": {"bound": "latency: 32 dependent 128-column steps", "achieved": f_tf, "unit": "TFLOP/s",
-                         "peak": sustained, "frac": f_tf / sustained,
-                         "issued_tflops": 3 * f_tf,
+        "hessian": {"bound": "tensor", "achieved": h_tf, "unit": "TFLOP/s", "peak": peak,
+                    "frac": h_tf / peak, "peak_kind": "bf16 dense burst (measured)"},
+        "prepare_hinv": {"bound": f"latency: {nb} dependent 128-column steps", "achieved": f_tf, "unit": "TFLOP/s",
+                         "peak": peak, "frac": f_tf / peak, "issued_tflops": 3 * f_tf,
                          "work": "2/3 d^3 flops (Cholesky d^3/3, triangular inverse d^3/3), 3 tf32 passes "
                                  "issued for their products"},
-        "quantize_layer": {"bound": "latency: 32 dependent sweep blocks, each followed by its trailing product",
+        "quantize_layer": {"bound": f"latency: {nb} dependent sweep blocks and their trailing products",
                            "sweep_gbs_over_stage": sweep_bytes / q_s / 1e9, "hbm_peak_gbs": hbm,
                            "sweep_frac_over_stage": sweep_bytes / q_s / 1e9 / hbm,
                            "sweep_issued_gbs_over_stage": sweep_issued / q_s / 1e9,
-                           "trailing_tflops_over_stage": t_flops / q_s / 1e12, "tensor_peak": sustained,
-                           "trailing_frac_over_stage": t_flops / q_s / 1e12 / sustained,
+                           "trailing_tflops_over_stage": t_flops / q_s / 1e12, "tensor_peak": peak,
+                           "trailing_frac_over_stage": t_flops / q_s / 1e12 / peak,
                            "trailing_issued_tflops_over_stage": 3 * t_flops / q_s / 1e12,
                            "work": f"sweep {sweep_bytes / 1e6:.1f} MB algorithmic ({sweep_issued / 1e6:.1f} MB "
                                    f"issued), trailing products {t_flops:.3e} flops (3 tf32 passes issued), "
                                    "both over the whole stage time"},
     }
+
+
+def time_layer(p, X_dev, W_dev, lq, stream, flush, steps, warmup, api):
+    """`warmup` untimed then `steps` timed runs of the whole layer (widen W
+    and zero H, H over every batch, damping and factorization, sweep and
+    packing), L2 flushed before each; device events between the stages.
+    Returns per-stage lists of ms."""
+    import torch
+
+    def one(evs):
+        evs[0].record(stream)
+        lq.begin(W_dev)
+        evs[1].record(stream)
+        lq.add_batches(X_dev)
+        evs[2].record(stream)
+        api.prepare_hinv(lq.H, lq.U, lq.ws_hinv, p.percdamp, lq.info)
+        evs[3].record(stream)
+        api.quantize_layer(lq.W, lq.U, p.bits, p.blocksize, p.groupsize, lq.codes, lq.scales, lq.zeros, lq.ws_q)
+        evs[4].record(stream)
+
+    runs = []
+    for i in range(warmup + steps):
+        flush.zero_()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        one(evs)
+        if i >= warmup:
+            runs.append(evs)
+    torch.cuda.synchronize()
+    api.get_status(stream)
+    return {"step": [e[0].elapsed_time(e[4]) for e in runs], "begin": [e[0].elapsed_time(e[1]) for e in runs],
+            "hessian": [e[1].elapsed_time(e[2]) for e in runs],
+            "prepare_hinv": [e[2].elapsed_time(e[3]) for e in runs],
+            "quantize_layer": [e[3].elapsed_time(e[4]) for e in runs]}
+
+
+def shape_timings(dev, stream, flush, args, api, peak, hbm):
+    """The scope's other layer shapes through the same timed step: the
+    11008-wide MLP pair (up 11008 x 4096 and down 4096 x 11008, 65536
+    heavy-tailed calibration rows, per-row grid, 3 and 4 bits) and the
+    8192 x 28672 layer (65536 rows in 8 batches, 4-bit, groups of 128).
+    Median ms per stage over the timed runs, weights/s, stage rooflines."""
+    import torch
+    from post_weight_quantization_05_b200 import synth
+    out = {}
+    steps = max(1, min(args.steps, 5))
+    warmup = max(1, min(args.warmup, 3))
+    cases = [("mlp28672", [synth.mlp28672()])]
+    cases += [(f"mlp11008_{w}", [synth.mlp11008(w, b) for b in (4, 3)]) for w in ("up", "down")]
+    for name, problems in cases:
+        p0 = problems[0]
+        xs = synth.x_batches_threaded(p0, min(16, os.cpu_count() or 8))
+        X_dev = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in xs]
+        del xs
+        for p in problems:
+            W_dev = torch.from_numpy(synth.f32_to_bf16_bits(p.W).view(np.int16)).to(dev).view(torch.bfloat16)
+            lq = api.LayerQuantizer(p.d_out, p.d_in, p.bits, p.groupsize, p.blocksize, p.percdamp, device=dev)
+            t = time_layer(p, X_dev, W_dev, lq, stream, flush, steps, warmup, api)
+            med = {k: statistics.median(v) for k, v in t.items()}
+            key = f"{name}_{p.bits}bit" if len(problems) > 1 else name
+            out[key] = {"d_out": p.d_out, "d_in": p.d_in, "n": p.n, "batches": p.n_batches, "bits": p.bits,
+                        "groupsize": p.groupsize, "ms_per_layer": med["step"],
+                        "weights_per_s": p.d_out * p.d_in / (med["step"] / 1e3),
+                        "quantize_only_ms": med["prepare_hinv"] + med["quantize_layer"],
+                        "stages_ms_median": med, "steps": steps, "warmup": warmup,
+                        "stage_roofline": stage_rooflines(p, med, peak, hbm)}
+            del lq, W_dev
+            torch.cuda.empty_cache()
+        del X_dev
+        torch.cuda.empty_cache()
+    return out
 
 
 def act_order_timing(p, X_dev, W_dev, dev, stream, flush, args, api):

@@ -18,8 +18,8 @@ def _layer():
 
 
 def test_stage_work_matches_closed_forms():
-    stages = {"hessian_16_batches": 4.0, "prepare_hinv": 2.0, "quantize_layer": 1.0}    # ms
-    r = bench.stage_rooflines(_layer(), stages, burst=1600.0, sustained=1400.0, hbm=6500.0)
+    stages = {"hessian": 4.0, "prepare_hinv": 2.0, "quantize_layer": 1.0}    # ms
+    r = bench.stage_rooflines(_layer(), stages, peak=1600.0, hbm=6500.0)
     # X^T X: the upper triangle with its diagonal, 2 flops per multiply-add
     assert r["hessian"]["achieved"] == pytest.approx(N * D * (D + 1) / 4e-3 / 1e12)
     assert N * D * (D + 1) == pytest.approx(4.40e12, rel=1e-3)
@@ -38,13 +38,13 @@ def test_stage_work_matches_closed_forms():
     assert q["trailing_tflops_over_stage"] == pytest.approx(t / 1e-3 / 1e12)
     assert q["trailing_issued_tflops_over_stage"] == pytest.approx(3 * t / 1e-3 / 1e12)
     for k, v in (("hessian", r["hessian"]), ("prepare_hinv", r["prepare_hinv"])):
-        assert v["frac"] == pytest.approx(v["achieved"] / 1400.0), k
+        assert v["frac"] == pytest.approx(v["achieved"] / 1600.0), k
 
 
 def test_per_row_grid_counts_one_group():
     p = _layer()
     p.groupsize = -1
-    stages = {"hessian_16_batches": 1.0, "prepare_hinv": 1.0, "quantize_layer": 1.0}
-    r = bench.stage_rooflines(p, stages, burst=1.0, sustained=1.0, hbm=1.0)
+    stages = {"hessian": 1.0, "prepare_hinv": 1.0, "quantize_layer": 1.0}
+    r = bench.stage_rooflines(p, stages, peak=1.0, hbm=1.0)
     sweep = D * D * 8.5 + D * 4 + (D // B) * B * B * 4
     assert r["quantize_layer"]["sweep_gbs_over_stage"] == pytest.approx(sweep / 1e-3 / 1e9)
