@@ -163,7 +163,14 @@ int gptq_prepare_hinv(const float* H, int64_t d_in, float percdamp, float* U,
  * For each block i = 0, B, 2B, ... and each column j of the block:
  *   c = clamp(rint(w_j / s) + z, 0, maxq);  q = s (c - z);
  *   E[:, j-i] = (w_j - q) / U[j][j];  W[:, j:i+B] -= E[:, j-i] U[j, j:i+B];
- * then W[:, i+B:] -= E U[i:i+B, i+B:].
+ * then W[:, i+B:] -= E U[i:i+B, i+B:].  That trailing update is applied in
+ * the deferred super-block form, exact in real arithmetic: blocks are taken
+ * in super-blocks of S columns (S = d_in if d_in <= 1024; else 1024, or the
+ * largest multiple of groupsize up to 1024, or B for groups wider than
+ * 1024); after each block its E updates only the rest of its super-block,
+ * and after a super-block's last block the columns beyond it get one product
+ * with the whole super-block's E (S deep).  The order is fixed: the same
+ * inputs give the same bits on every call.
  * Grid: s32 = max(wmax - wmin, 1e-8) / maxq (fp32), s = fp16(s32) (2^-14 if
  * that rounds to 0), z = fp16(rint(-wmin / s)); per row from the original W
  * (groupsize = -1), or per group of `groupsize` columns from the current W
@@ -198,14 +205,15 @@ int gptq_quantize_layer(float* W, int64_t d_out, int64_t d_in, const float* U,
  * device).
  *
  * Same arguments, results and errors as gptq_quantize_layer, minus ws and
- * ws_bytes.  The scratch it needs (E [d_out, 128] and U^T [d_in, d_in], each
- * kept as two fp32 arrays -- the tf32-rounded part and the remainder -- for
- * the tensor-core trailing product, each array rounded up to 256 bytes)
- * lives in one 40 MiB device array inside the library, which every GPU that
- * loads the library holds until the process exits.  Sizes that need more than
- * 40 MiB (about d_out * 1024 + d_in * d_in * 8 bytes) return
- * GPTQ_ERR_UNSUPPORTED and launch nothing: e.g. d_in = 2048 works for d_out
- * up to 8192, d_in = 3072 does not fit.
+ * ws_bytes.  The scratch it needs (E [d_out, min(d_in, 1024)] and U^T
+ * [d_in, d_in], each kept as two fp32 arrays -- the tf32-rounded part and the
+ * remainder -- for the tensor-core trailing products, each array rounded up to
+ * 256 bytes) lives in one 40 MiB device array inside the library, which every
+ * GPU that loads the library holds until the process exits.  Sizes that need
+ * more than 40 MiB (about d_out * min(d_in, 1024) * 8 + d_in * d_in * 8
+ * bytes) return GPTQ_ERR_UNSUPPORTED and launch nothing: e.g. d_in = 1024
+ * works for d_out up to 4096, d_in = 2048 for d_out up to 1024, d_in = 512 for
+ * d_out up to 9728; d_in = 2304 does not fit at all.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress with that device current); make that first call
  *    before any stream capture begins.

@@ -11,7 +11,7 @@
 //
 // The scratch is one file-scope device array of kNoAllocScratchBytes, held
 // by every GPU that loads this library until the process exits.  It holds the
-// per-block error matrix E [d_out, 128] fp32 and U^T [d_in, d_in] fp32, the
+// super-block error matrix E [d_out, min(d_in, 1024)] fp32 and U^T [d_in, d_in] fp32, the
 // same two pieces gptq_quantize_layer keeps in its workspace.  Host code may
 // not use the array's name as a device pointer, so its device address is
 // looked up once per device (cudaGetSymbolAddress, with that device current)

@@ -157,8 +157,9 @@ struct SweepArgs {
     uint16_t* scales;
     uint16_t* zeros;
     float* Q;
-    float* E;     // [d_out, B] hi parts of the block's E (tf32-rounded)
-    float* E_lo;  // [d_out, B] remainders
+    float* E;     // [d_out, e_ld] hi parts of the super-block's E (tf32-rounded)
+    float* E_lo;  // [d_out, e_ld] remainders
+    int e_ld;     // super-block width: block i0's E goes to columns i0 % e_ld ..
     DevStatus* st;
 };
 
@@ -336,8 +337,8 @@ __global__ void __launch_bounds__(SWEEP_THREADS) sweep_block_kernel(const __grid
 
     if (active) {
         // E leaves pre-split for the trailing product's tensor cores
-        float* erow = a.E + size_t(r) * B + wc;
-        float* elo = a.E_lo + size_t(r) * B + wc;
+        float* erow = a.E + size_t(r) * a.e_ld + i0 % a.e_ld + wc;
+        float* elo = a.E_lo + size_t(r) * a.e_ld + i0 % a.e_ld + wc;
 #pragma unroll
         for (int j = 0; j < SUB; j += 4) {
             float4 hi, lo;
@@ -415,6 +416,20 @@ __global__ void transpose_upper_kernel(const float* __restrict__ U, int d, float
     }
 }
 
+// The blocks in order, each followed by its share of the trailing update.
+// Deferred super-block form (exact reformulation of the pages' lazy update:
+// the trailing update is linear, so each column still holds, when the sweep
+// reaches it, every earlier block's correction): the blocks are taken in
+// super-blocks of a.e_ld columns.  After block i0, its E updates only the
+// rest of its super-block, W[:, i0+B:s2] -= E_i0 U[i0:i0+B, i0+B:s2]; after
+// the super-block's last block, the columns beyond it get one product with
+// the super-block's whole E, W[:, s2:] -= E_sb U[s1:s2, s2:] (K = e_ld).  The
+// far tail of W is then read and written once per super-block instead of
+// once per block, and each product is e_ld deep instead of B.  With e_ld = B
+// this is exactly the per-block form.  A group grid is set from the columns
+// of its group, which therefore must lie inside one super-block (e_ld is a
+// multiple of the group size).  Everything runs on one stream, in a fixed
+// order, so the result does not depend on timing.
 template <int BITS>
 int run_sweep(const SweepArgs& a, cudaStream_t stream) {
     static std::atomic<bool> attr_set[64];
@@ -430,18 +445,30 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
     if (make_map_2d_f32(&tmU, a.U, uint64_t(a.d_in), uint64_t(a.d_in), uint64_t(a.d_in), B, B, false))
         return GPTQ_ERR_CUDA;
     const int blocks = (a.d_out + SUB - 1) / SUB;
-    for (int i0 = 0; i0 < a.d_in; i0 += B) {
-        if (launch_pdl(sweep_block_kernel<BITS>, dim3(blocks), dim3(SWEEP_THREADS), SMEM, stream, tmU, a, i0) !=
-            cudaSuccess)
-            return GPTQ_ERR_CUDA;
-        count_launch();
-        const int tail = a.d_in - i0 - B;
-        if (tail > 0) {
-            // W[:, i0+B:] -= E * U[i0:i0+B, i0+B:]   (U[i0+k][i0+B+n] = Ut[i0+B+n][i0+k])
-            float* c = a.W + i0 + B;
-            const size_t ut = size_t(i0 + B) * a.d_in + i0;
-            const int rc = launch_tgemm(a.d_out, tail, B, -1.0f, a.E, a.E_lo, B, a.Ut + ut, a.Ut_lo + ut, a.d_in,
-                                        true, c, a.d_in, false, stream, a.st);
+    const int sbw = a.e_ld;
+    for (int s1 = 0; s1 < a.d_in; s1 += sbw) {
+        const int s2 = std::min(s1 + sbw, a.d_in);
+        for (int i0 = s1; i0 < s2; i0 += B) {
+            if (launch_pdl(sweep_block_kernel<BITS>, dim3(blocks), dim3(SWEEP_THREADS), SMEM, stream, tmU, a, i0) !=
+                cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            count_launch();
+            const int near = s2 - i0 - B;
+            if (near > 0) {
+                // W[:, i0+B:s2] -= E_i0 U[i0:i0+B, i0+B:s2]   (U[i0+k][i0+B+n] = Ut[i0+B+n][i0+k])
+                const size_t ut = size_t(i0 + B) * a.d_in + i0;
+                const int rc = launch_tgemm(a.d_out, near, B, -1.0f, a.E + (i0 - s1), a.E_lo + (i0 - s1), sbw,
+                                            a.Ut + ut, a.Ut_lo + ut, a.d_in, true, a.W + i0 + B, a.d_in, false,
+                                            stream, a.st);
+                if (rc) return rc;
+            }
+        }
+        const int far = a.d_in - s2;
+        if (far > 0) {
+            // W[:, s2:] -= E_sb U[s1:s2, s2:]
+            const size_t ut = size_t(s2) * a.d_in + s1;
+            const int rc = launch_tgemm(a.d_out, far, s2 - s1, -1.0f, a.E, a.E_lo, sbw, a.Ut + ut, a.Ut_lo + ut,
+                                        a.d_in, true, a.W + s2, a.d_in, false, stream, a.st);
             if (rc) return rc;
         }
     }
@@ -450,13 +477,32 @@ int run_sweep(const SweepArgs& a, cudaStream_t stream) {
 
 }  // namespace sweep
 
-// E hi, E lo [d_out, B] fp32, then U^T hi, U^T lo [d_in, d_in] fp32 (each 256-byte aligned)
+// Width of the super-blocks of the deferred trailing update: up to
+// kSuperBlockCols columns, a multiple of the block and of the group size; the
+// whole layer when it is narrower; the per-block form (B) for groups wider
+// than kSuperBlockCols.
+#ifndef GPTQ_SUPERBLOCK_COLS
+#define GPTQ_SUPERBLOCK_COLS 1024
+#endif
+constexpr int kSuperBlockCols = GPTQ_SUPERBLOCK_COLS;   // a build-time tuning knob (128: per-block form)
+static_assert(kSuperBlockCols % 128 == 0 && kSuperBlockCols >= 128 && kSuperBlockCols <= 8192, "super-block width");
+int superblock_cols(int64_t d_in, int groupsize) {
+    if (d_in <= kSuperBlockCols) return int(d_in);
+    if (groupsize <= 0) return kSuperBlockCols;
+    if (groupsize > kSuperBlockCols) return sweep::B;
+    return (kSuperBlockCols / groupsize) * groupsize;
+}
+
+// E hi, E lo [d_out, min(d_in, kSuperBlockCols)] fp32, then U^T hi, U^T lo
+// [d_in, d_in] fp32 (each 256-byte aligned)
 namespace {
-size_t e_bytes(int64_t d_out) { return (size_t(d_out) * sweep::B * sizeof(float) + 255) & ~size_t(255); }
+size_t e_bytes(int64_t d_out, int64_t d_in) {
+    return (size_t(d_out) * size_t(std::min<int64_t>(d_in, kSuperBlockCols)) * sizeof(float) + 255) & ~size_t(255);
+}
 }  // namespace
 
 size_t sweep_workspace_bytes(int64_t d_out, int64_t d_in) {
-    return 2 * e_bytes(d_out) + 2 * size_t(d_in) * size_t(d_in) * sizeof(float);
+    return 2 * e_bytes(d_out, d_in) + 2 * size_t(d_in) * size_t(d_in) * sizeof(float);
 }
 
 int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int bits, int groupsize,
@@ -477,8 +523,9 @@ int launch_quantize(float* W, int64_t d_out, int64_t d_in, const float* U, int b
     a.Q = Q;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     a.E = reinterpret_cast<float*>(wsb);
-    a.E_lo = reinterpret_cast<float*>(wsb + e_bytes(d_out));
-    float* Ut = reinterpret_cast<float*>(wsb + 2 * e_bytes(d_out));
+    a.E_lo = reinterpret_cast<float*>(wsb + e_bytes(d_out, d_in));
+    a.e_ld = superblock_cols(d_in, groupsize);
+    float* Ut = reinterpret_cast<float*>(wsb + 2 * e_bytes(d_out, d_in));
     float* Ut_lo = Ut + size_t(d_in) * size_t(d_in);
     a.Ut = Ut;
     a.Ut_lo = Ut_lo;

@@ -50,7 +50,9 @@ def test_workspace_sizes(lib):
     assert lib.gptq_hessian_workspace_size(_native.GPTQ_F32, 1000, 512) == 3 * 1000 * 512 * 2
     assert lib.gptq_prepare_hinv_workspace_size(512) >= 2 * 512 * 512 * 4
     assert lib.gptq_prepare_hinv_workspace_size(100) == 0          # d_in % 128 != 0
-    assert lib.gptq_quantize_workspace_size(300, 512, 128) == 2 * ((300 * 128 * 4 + 255) // 256) * 256 + 2 * 512 * 512 * 4
+    # E [d_out, min(d_in, 1024)] and U^T [d_in, d_in], each as a tf32 part and a remainder
+    assert lib.gptq_quantize_workspace_size(300, 512, 128) == 2 * ((300 * 512 * 4 + 255) // 256) * 256 + 2 * 512 * 512 * 4
+    assert lib.gptq_quantize_workspace_size(300, 4096, 128) == 2 * 300 * 1024 * 4 + 2 * 4096 * 4096 * 4
     assert lib.gptq_quantize_workspace_size(300, 512, 64) == 0
 
 
