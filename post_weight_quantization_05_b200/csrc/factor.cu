@@ -28,9 +28,15 @@ namespace gptq {
 namespace factor {
 
 constexpr int NB = 128;
-// Block columns the critical stream updates after each panel (the rest of the
-// trailing update goes to the side stream).
-constexpr int NEAR = 3;
+// Block columns per super-panel.  Inside a super-panel the factorization is
+// right-looking by 128-column blocks; the columns beyond it get the
+// super-panel's whole update at once, as one product SUPER * 128 deep.  A
+// build-time tuning knob.
+#ifndef GPTQ_FACTOR_SUPER
+#define GPTQ_FACTOR_SUPER 8
+#endif
+constexpr int SUPER = GPTQ_FACTOR_SUPER;
+static_assert(SUPER >= 1 && SUPER * 128 <= 8192, "super-panel width");
 
 struct Layout {
     size_t a_off, y_off, dinv_off, scal_off, total;
@@ -420,9 +426,9 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
 // Three internal streams and a few events per set (created on first use).
 // The factorization's critical chain runs on a high-priority stream; the
 // inverse's block steps run on another, each as soon as the factorization has
-// finished the block column it needs; the trailing update beyond the next
-// NEAR block columns runs on a low-priority stream, so that the next diagonal
-// blocks are factored while it proceeds (look-ahead) and get the SMs first.
+// finished the block column it needs; the update of the columns beyond the
+// next super-panel runs on a low-priority stream, beside the next
+// super-panel's chain (look-ahead).
 // Each device has AUX_SETS sets.  A caller stream keeps the set it was given
 // first, so that factorizations called on different streams (independent
 // layers) run concurrently; once every set is taken, further caller streams
@@ -431,10 +437,10 @@ constexpr int AUX_SETS = 4;
 struct AuxStream {
     cudaStream_t main = nullptr;    // the factorization's critical chain (highest priority)
     cudaStream_t s = nullptr;       // inverse steps
-    cudaStream_t side = nullptr;    // trailing updates beyond the next NEAR block columns
+    cudaStream_t side = nullptr;    // updates of the columns beyond the next super-panel
     static constexpr int RING = 4;
     cudaEvent_t fork = nullptr, step = nullptr, join = nullptr, join_side = nullptr, filled = nullptr;
-    cudaEvent_t far_done[RING] = {};   // the far update of step k, slot k % RING
+    cudaEvent_t far_done[RING] = {};   // the far update of super-panel p, slot p % RING
     std::mutex enqueue;                // one call enqueues on this set at a time
     cudaStream_t owner = nullptr;      // the caller stream the set was given to
     bool taken = false;
@@ -556,7 +562,7 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
     damp_lambda_kernel<<<1, 1024, 0, stream>>>(H, d, percdamp, lam, info, st); count_launch();
     reverse_damp_kernel<<<d, 256, 0, stream>>>(H, d, lam, A); count_launch();
     // fork: the inverse (stream `as`) starts from a zeroed Z; `ss` takes the
-    // trailing updates beyond the next NEAR block columns
+    // updates of the columns beyond the next super-panel
     const cudaStream_t ss = aux->side;
     if (cudaEventRecord(aux->fork, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->fork, 0) != cudaSuccess ||
         cudaStreamWaitEvent(ss, aux->fork, 0) != cudaSuccess)
@@ -570,75 +576,93 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         return GPTQ_ERR_CUDA;
 
     // Cholesky of A (lower), blocked right-looking, products on the tensor
-    // cores.  Step k on `stream`: factor the diagonal block, solve the panel,
-    // update the next NEAR block columns; the rest of the trailing update goes
-    // to `ss`.
+    // cores, in super-panels of SUPER block columns [p0, p1):
+    //  - step k of the super-panel, on `stream`: factor the diagonal block,
+    //    solve the panel below it, then update the super-panel's later block
+    //    columns (all rows below);
+    //  - after the super-panel: the next super-panel's columns [p1, h1) get
+    //    the whole super-panel's update, one product (p1 - p0) deep, on
+    //    `stream`; the columns from h1 on get theirs on `ss`, beside the next
+    //    super-panel's steps.
+    // Every element of A thus receives its updates in a fixed order (by
+    // super-panel, then by step): `ss` runs in order, and `stream` waits for
+    // the previous super-panel's far update before it first touches the
+    // columns that update covered.  So U does not depend on how the streams
+    // interleave.
     // Z = L^-T (upper) on `as`: block step i needs only L's block column i and
     // Dinv_i, so it runs as soon as the factorization has them:
     //   Z[i][i] = Dinv_i^T;  Z[0:i0, i] <- Z[0:i0, i] Dinv_i^T;
-    //   Z[0:i0+NB, i0+NB:] -= Z[0:i0+NB, i] L[i0+NB:, i]^T
-    // (the transpose of the block forward substitution Y = L^-1; working on Z
-    // keeps every tensor-core operand K-major).
-    for (int k = 0; k < nblk; ++k) {
-        const int k0 = k * NB;
-        float* dk = Dinv + size_t(k) * NB * NB;
-        // Block k needs every far update j <= k - NEAR - 1 (side stream, see
-        // below); the wait before step k - 1's near update (below) has already
-        // ordered them before this kernel.
-        if (launch_pdl(potrf_diag_kernel, dim3(1), dim3(DIAG_THREADS), DIAG_SMEM, stream, static_cast<const float*>(A), d,
-                       k0, dk, Z, info, st) != cudaSuccess)
-            return GPTQ_ERR_CUDA;
-        count_launch();
-        const int rest = d - k0 - NB;
-        float* panel = A + size_t(k0 + NB) * d + k0;
-        int rc;
-        if (rest > 0) {
-            // panel <- panel * Dinv_k^T.  In place is safe: N = NB is one output
-            // tile column, so each CTA reads only the rows it writes, all before
-            // its epilogue.
-            rc = launch_tgemm(rest, NB, NB, 1.0f, panel, nullptr, d, dk, nullptr, NB, false, panel, d, false, stream, st);
-            if (rc) return rc;
-        }
-        if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->step, 0) != cudaSuccess)
-            return GPTQ_ERR_CUDA;
-        if (rest > 0) {
-            // the next NEAR block columns (they hold the next diagonal blocks) on
-            // `stream` ...  Column block k + NEAR enters this window now: until
-            // step k - 1 it was updated by the side stream.  Waiting for step
-            // k - 1's far update (the side stream runs in order, so it is the
-            // last one) makes every element receive its updates in step order,
-            // so U does not depend on how the two streams interleave.
-            if (k >= 1 && cudaStreamWaitEvent(stream, aux->far_done[(k - 1) % AuxStream::RING], 0) != cudaSuccess)
+    //   Z[0:i0+NB, i0+NB:p1] -= Z[0:i0+NB, i] L[i0+NB:p1, i]^T,
+    // and after each super-panel Z[0:p1, p1:] -= Z[0:p1, p0:p1] L[p1:, p0:p1]^T
+    // (the transpose of the block forward substitution Y = L^-1, deferred the
+    // same way; Z's entries below the diagonal are zero, so the full row range
+    // adds nothing; working on Z keeps every tensor-core operand K-major).
+    int rc;
+    for (int pb0 = 0, sp = 0; pb0 < nblk; pb0 += SUPER, ++sp) {
+        const int pb1 = std::min(nblk, pb0 + SUPER);
+        const int p0 = pb0 * NB, p1 = pb1 * NB;
+        for (int k = pb0; k < pb1; ++k) {
+            const int k0 = k * NB;
+            float* dk = Dinv + size_t(k) * NB * NB;
+            if (launch_pdl(potrf_diag_kernel, dim3(1), dim3(DIAG_THREADS), DIAG_SMEM, stream, static_cast<const float*>(A),
+                           d, k0, dk, Z, info, st) != cudaSuccess)
                 return GPTQ_ERR_CUDA;
-            const int near_cols = std::min(rest, NEAR * NB);
-            float* next = A + size_t(k0 + NB) * d + k0 + NB;
-            rc = launch_tgemm(rest, near_cols, NB, -1.0f, panel, nullptr, d, panel, nullptr, d, true, next, d, true,
-                              stream, st);
-            if (rc) return rc;
-            // ... the columns after them on `ss`, beside the next steps' chain
-            if (rest > NEAR * NB) {
-                if (cudaStreamWaitEvent(ss, aux->step, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
-                const int f0 = k0 + (NEAR + 1) * NB;
-                float* far = A + size_t(f0) * d + f0;
-                const float* prow = panel + size_t(NEAR) * NB * d;
-                rc = launch_tgemm(rest - NEAR * NB, rest - NEAR * NB, NB, -1.0f, prow, nullptr, d, prow, nullptr, d,
-                                  true, far, d, true, ss, st);
+            count_launch();
+            const int rest = d - k0 - NB;
+            float* panel = A + size_t(k0 + NB) * d + k0;
+            if (rest > 0) {
+                // panel <- panel * Dinv_k^T.  In place is safe: N = NB is one output
+                // tile column, so each CTA reads only the rows it writes, all before
+                // its epilogue.
+                rc = launch_tgemm(rest, NB, NB, 1.0f, panel, nullptr, d, dk, nullptr, NB, false, panel, d, false, stream, st);
                 if (rc) return rc;
             }
-            if (cudaEventRecord(aux->far_done[k % AuxStream::RING], ss) != cudaSuccess) return GPTQ_ERR_CUDA;
+            if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(as, aux->step, 0) != cudaSuccess)
+                return GPTQ_ERR_CUDA;
+            const int ncols = p1 - k0 - NB;   // the super-panel's later columns
+            if (ncols > 0) {
+                rc = launch_tgemm(rest, ncols, NB, -1.0f, panel, nullptr, d, panel, nullptr, d, true,
+                                  A + size_t(k0 + NB) * d + k0 + NB, d, true, stream, st);
+                if (rc) return rc;
+            }
+            // inverse block step k on the auxiliary stream (Z's diagonal block k
+            // was written by the diagonal kernel)
+            if (k > 0) {
+                float* zi = Z + k0;   // in place is safe for the same reason as the panel
+                rc = launch_tgemm(k0, NB, NB, 1.0f, zi, nullptr, d, dk, nullptr, NB, false, zi, d, false, as, st);
+                if (rc) return rc;
+            }
+            if (ncols > 0) {
+                rc = launch_tgemm(k0 + NB, ncols, NB, -1.0f, Z + k0, nullptr, d, panel, nullptr, d, true, Z + k0 + NB, d,
+                                  false, as, st);
+                if (rc) return rc;
+            }
         }
-        // inverse block step k on the auxiliary stream (Z's diagonal block k
-        // was written by the diagonal kernel)
-        if (k > 0) {
-            float* zi = Z + k0;   // in place is safe for the same reason as the panel
-            rc = launch_tgemm(k0, NB, NB, 1.0f, zi, nullptr, d, dk, nullptr, NB, false, zi, d, false, as, st);
+        if (p1 >= d) break;
+        // the super-panel's update of the columns after it
+        const int h1 = std::min(d, p1 + SUPER * NB);   // end of the next super-panel
+        const int kd = p1 - p0;
+        const float* lp = A + size_t(p1) * d + p0;     // L[p1:, p0:p1]
+        if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(ss, aux->step, 0) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        if (h1 < d) {
+            // columns [h1, d) on `ss`
+            const float* lh = A + size_t(h1) * d + p0;
+            rc = launch_tgemm(d - h1, d - h1, kd, -1.0f, lh, nullptr, d, lh, nullptr, d, true,
+                              A + size_t(h1) * d + h1, d, true, ss, st);
             if (rc) return rc;
         }
-        if (rest > 0) {
-            float* zc = Z + k0 + NB;
-            rc = launch_tgemm(k0 + NB, rest, NB, -1.0f, Z + k0, nullptr, d, panel, nullptr, d, true, zc, d, false, as, st);
-            if (rc) return rc;
-        }
+        if (cudaEventRecord(aux->far_done[sp % AuxStream::RING], ss) != cudaSuccess) return GPTQ_ERR_CUDA;
+        // columns [p1, h1) on `stream`, after the previous super-panel's far
+        // update (which covered them)
+        if (sp > 0 && cudaStreamWaitEvent(stream, aux->far_done[(sp - 1) % AuxStream::RING], 0) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        rc = launch_tgemm(d - p1, h1 - p1, kd, -1.0f, lp, nullptr, d, lp, nullptr, d, true, A + size_t(p1) * d + p1, d,
+                          true, stream, st);
+        if (rc) return rc;
+        // Z's columns after the super-panel
+        rc = launch_tgemm(p1, d - p1, kd, -1.0f, Z + p0, nullptr, d, lp, nullptr, d, true, Z + p1, d, false, as, st);
+        if (rc) return rc;
     }
     // join both auxiliary streams
     if (cudaEventRecord(aux->join, as) != cudaSuccess || cudaStreamWaitEvent(stream, aux->join, 0) != cudaSuccess ||
