@@ -45,12 +45,17 @@ constexpr int EPI_WARPS = 8;              // 4 TMEM lane quadrants x 2 column ha
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr int BMH = 128;                   // H rows per CTA (the pair covers 256)
 constexpr int BNP = 256;                   // H columns per pair (128 loaded by each CTA)
-constexpr int STAGES = 6;
+#ifndef GPTQ_HESS_STAGES
+#define GPTQ_HESS_STAGES 6
+#endif
+constexpr int STAGES = GPTQ_HESS_STAGES;   // a build-time tuning knob
 constexpr int A_BYTES = BMH * BK * 2;      // 16 KB
 constexpr int B_BYTES = (BNP / 2) * BK * 2;  // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BNP;         // two accumulator buffers
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + size_t(STAGES) * STAGE_BYTES + 256 /*barriers*/;
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+static_assert((2 * STAGES + 4) * 8 + 4 <= 256, "barrier area");
 
 // Pair protocol: CTA r (r = 0, 1) loads a-columns a0 + 128 r .. + 127 and
 // b-columns b0 + 128 r .. + 127 of each slab; both CTAs' TMA loads complete on
@@ -67,6 +72,42 @@ struct Params {
     int late_wait;  // the previous kernel in the stream is this kernel on another batch
 };
 
+// Launch order of the tiles (ta, tb), ta <= tb.  Pairs that run at the same
+// time should read few distinct column slabs of X, so that a slab comes from
+// HBM once and from L2 for the other tiles that use it (a slab is n_b x 256
+// bf16: 4 MB at 8192 rows, so X of a 28672-wide layer is 112 slabs, far more
+// than L2 holds).  Tiles are therefore taken in super-tiles of SUPER x SUPER
+// tiles (about one wave of 74 pairs at SUPER = 8, reading at most 16 slabs),
+// super-tiles by column J and then row I <= J, and inside a super-tile
+// column-major with ta <= tb.  The order does not change any tile's
+// arithmetic.
+constexpr int SUPER = 8;
+__device__ __forceinline__ void tile_of(int t, int T, int& ta, int& tb) {
+    const int ns = (T + SUPER - 1) / SUPER;
+    for (int J = 0; J < ns; ++J) {
+        const int b0 = J * SUPER, b1 = min(T, b0 + SUPER);
+        for (int I = 0; I <= J; ++I) {
+            const int a0 = I * SUPER, a1 = min(T, a0 + SUPER);
+            int cnt = 0;   // tiles of this super-tile with ta <= tb
+            for (int b = b0; b < b1; ++b) cnt += max(0, min(a1, b + 1) - a0);
+            if (t >= cnt) {
+                t -= cnt;
+                continue;
+            }
+            for (int b = b0; b < b1; ++b) {
+                const int na = max(0, min(a1, b + 1) - a0);
+                if (t < na) {
+                    ta = a0 + t;
+                    tb = b;
+                    return;
+                }
+                t -= na;
+            }
+        }
+    }
+    ta = tb = 0;   // not reached for t < T (T + 1) / 2
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     syrk_pair_kernel(const __grid_constant__ CUtensorMap tmX, const Params p, float* __restrict__ H,
                      DevStatus* st) {
@@ -79,15 +120,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
 
     const uint32_t rank = cluster_ctarank();
-    // tile (ta, tb), ta <= tb, column-major over tb
     int ta = 0, tb = 0;
-    {
-        int t = int(blockIdx.x >> 1), acc = 0;
-        for (tb = 0; tb < p.T; ++tb) {
-            if (t < acc + tb + 1) { ta = t - acc; break; }
-            acc += tb + 1;
-        }
-    }
+    tile_of(int(blockIdx.x >> 1), p.T, ta, tb);
     const int a0 = ta * BNP + int(rank) * BMH;   // this CTA's H rows
     const int b0 = tb * BNP;                     // the pair's H columns
     const int warp = threadIdx.x >> 5;
