@@ -12,6 +12,14 @@ Tolerances (stated once, used by every parity test):
            those are bounded by the fraction and the loss criteria.  (An fp32
            restatement of the sweep on the CPU shows the same cascades,
            including later codes two levels apart.)
+           With group grids taken from the latest weights a flip does not die
+           out: the later groups' grids come from the differently compensated
+           weights, so the rest of the row follows another trajectory.  If
+           decisions flip at a rate rho, the expected differing fraction of a
+           row of d_in codes is rho * d_in / 2, which fp32 arithmetic (rho about
+           5.5e-7 against the fp64 oracle) keeps under 0.1% only up to about
+           3600 columns.  For group grids the identical fraction is therefore
+           held to 1 - RHO_MAX * d_in / 2 where that is below 99.9%.
   loss     ||W X^T - W^ X^T||^2 within 0.5% (relative) of the oracle's
   grid     per-row scales/zeros (from the original W) and RTN: bit-exact;
            group scales/zeros: bit-exact given the GPU's own group min/max.
@@ -35,6 +43,10 @@ CODE_MATCH = 0.999
 LOSS_TOL = 0.005
 TIE_TOL = 5e-3
 GRID_TIE_REL = 1e-4
+# Flips per decision allowed for group grids (see check_codes): four times the
+# rate measured for the fp32 sweep against the fp64 oracle on one common U
+# (5.5e-7 at 8192 x 28672, groups of 128).
+RHO_MAX = 2e-6
 
 
 def rel_fro(a, b):
@@ -98,12 +110,13 @@ def check_codes(got, ref, what="", match=CODE_MATCH, bits=None, groupsize=-1, gp
     """`ref` is the oracle's output dict (with the trace when available)."""
     got = np.asarray(got)
     rc = np.asarray(ref["codes"])
+    d_in = rc.shape[1]
     diff = np.abs(got - rc)
     frac = float(np.mean(diff == 0))
-    assert frac >= match, f"{what}: only {frac:.6f} of codes identical"
+    need = match if groupsize <= 0 else min(match, 1.0 - RHO_MAX * d_in / 2)
+    assert frac >= need, f"{what}: only {frac:.6f} of codes identical (need {need:.6f})"
     if "W_at" not in ref:
         return frac
-    d_in = rc.shape[1]
     g = d_in if groupsize <= 0 else groupsize
     s_full = np.repeat(np.asarray(ref["scales"], np.float64), g, axis=1)[:, :d_in]
     z_full = np.repeat(np.asarray(ref["zeros"], np.float64), g, axis=1)[:, :d_in]
@@ -125,6 +138,18 @@ def check_codes(got, ref, what="", match=CODE_MATCH, bits=None, groupsize=-1, gp
         dist = abs((t - np.floor(t)) - 0.5)
         assert dist <= TIE_TOL, f"{what}: row {r} col {j} flipped away from a tie (distance {dist:.2e})"
     return frac
+
+
+def decision_stats(got, ref_codes):
+    """Per-decision agreement along the sweep.  In each row the codes up to
+    and including its first difference were decided from identical states;
+    returns (rows with a difference, decisions taken from identical states).
+    Their ratio is the rate at which the two sides' arithmetic decides a
+    code differently, without the cascade that follows a flip."""
+    diff = np.asarray(got) != np.asarray(ref_codes)
+    any_d = diff.any(axis=1)
+    first = np.where(any_d, np.argmax(diff, axis=1) + 1, diff.shape[1])
+    return int(any_d.sum()), int(first.sum())
 
 
 def dequant_rows(codes, scales, zeros, groupsize):

@@ -114,3 +114,12 @@ def test_grid_tie_tolerance_is_below_an_fp16_step():
     # the accepted distance from the rounding boundary is a small part of one
     # fp16 step (2^-10 relative at most), so a scale from a wrong range fails
     assert GRID_TIE_REL < 0.25 * 2.0 ** -10
+
+
+def test_decision_stats_counts_prefixes():
+    from parity_util import decision_stats
+    ref = np.zeros((3, 10), dtype=np.int64)
+    got = ref.copy()
+    got[0, 4:] = 1          # first difference at column 4: 5 decisions from identical states
+    got[2, 0] = 1           # at column 0: 1 decision
+    assert decision_stats(got, ref) == (2, 5 + 10 + 1)
