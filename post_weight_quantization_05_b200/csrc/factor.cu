@@ -38,19 +38,45 @@ constexpr int NB = 128;
 constexpr int SUPER = GPTQ_FACTOR_SUPER;
 static_assert(SUPER >= 1 && SUPER * 128 <= 8192, "super-panel width");
 
+// Workspace: A (the reversed damped H, then L'), Z (= L'^-T), the diagonal
+// blocks' inverses, and the operands of the once-per-super-panel products
+// pre-split into tf32 parts and remainders: a super-panel's block columns of
+// L' (two buffers, so that one super-panel's can be written while the
+// previous one's are still read) and of Z, each [d, min(d, SUPER * NB)] fp32.
 struct Layout {
-    size_t a_off, y_off, dinv_off, scal_off, total;
+    size_t a_off, y_off, dinv_off, ls_off, zs_off, scal_off, total;
+    size_t sp_elems;   // elements of one pre-split array
 };
 
 __host__ __device__ inline Layout layout(int64_t d) {
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     Layout L;
+    L.sp_elems = size_t(d) * size_t(d < SUPER * NB ? d : SUPER * NB);
     L.a_off = 0;
     L.y_off = up(L.a_off + size_t(d) * d * sizeof(float));
     L.dinv_off = up(L.y_off + size_t(d) * d * sizeof(float));
-    L.scal_off = up(L.dinv_off + size_t(d) * NB * sizeof(float));
+    L.ls_off = up(L.dinv_off + size_t(d) * NB * sizeof(float));          // [2 buffers][hi, lo]
+    L.zs_off = up(L.ls_off + 4 * L.sp_elems * sizeof(float));             // [hi, lo]
+    L.scal_off = up(L.zs_off + 2 * L.sp_elems * sizeof(float));
     L.total = L.scal_off + 256;
     return L;
+}
+
+// hi[r][c] + lo[r][c] = src[r * ld + c] (tf32 part and remainder), r < rows,
+// c < cols (a multiple of 4); hi and lo are dense [rows, cols].
+__global__ void split_cols_kernel(const float* __restrict__ src, int ld, int rows, int cols, float* __restrict__ hi,
+                                  float* __restrict__ lo) {
+    const int c4 = cols / 4;
+    const size_t n = size_t(rows) * c4;
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x) {
+        const int r = int(i / c4), c = int(i % c4) * 4;
+        const float4 v = *reinterpret_cast<const float4*>(src + size_t(r) * ld + c);
+        float4 h, l;
+        split_tf32(v.x, h.x, l.x); split_tf32(v.y, h.y, l.y);
+        split_tf32(v.z, h.z, l.z); split_tf32(v.w, h.w, l.w);
+        *reinterpret_cast<float4*>(hi + size_t(r) * cols + c) = h;
+        *reinterpret_cast<float4*>(lo + size_t(r) * cols + c) = l;
+    }
 }
 
 // lambda = percdamp * mean(diag H); also resets *info.
@@ -441,6 +467,7 @@ struct AuxStream {
     static constexpr int RING = 4;
     cudaEvent_t fork = nullptr, step = nullptr, join = nullptr, join_side = nullptr, filled = nullptr;
     cudaEvent_t far_done[RING] = {};   // the far update of super-panel p, slot p % RING
+    cudaEvent_t zfar_done[2] = {};     // Z's far update of super-panel p, slot p % 2
     std::mutex enqueue;                // one call enqueues on this set at a time
     cudaStream_t owner = nullptr;      // the caller stream the set was given to
     bool taken = false;
@@ -479,6 +506,8 @@ static int aux_stream(cudaStream_t caller, AuxStream** out) {
             return GPTQ_ERR_CUDA;
         for (int i = 0; i < AuxStream::RING; ++i)
             if (cudaEventCreateWithFlags(&a.far_done[i], cudaEventDisableTiming) != cudaSuccess) return GPTQ_ERR_CUDA;
+        for (int i = 0; i < 2; ++i)
+            if (cudaEventCreateWithFlags(&a.zfar_done[i], cudaEventDisableTiming) != cudaSuccess) return GPTQ_ERR_CUDA;
     }
     *out = &a;
     return GPTQ_OK;
@@ -639,17 +668,32 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
             }
         }
         if (p1 >= d) break;
-        // the super-panel's update of the columns after it
+        // the super-panel's update of the columns after it, from its operands
+        // pre-split into tf32 parts and remainders (the products' fast form):
+        // L'[p1:, p0:p1] into buffer sp % 2 (on `stream`, once the super-panel
+        // two back no longer reads that buffer), Z[0:p1, p0:p1] (on `as`)
         const int h1 = std::min(d, p1 + SUPER * NB);   // end of the next super-panel
         const int kd = p1 - p0;
-        const float* lp = A + size_t(p1) * d + p0;     // L[p1:, p0:p1]
-        if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(ss, aux->step, 0) != cudaSuccess)
+        const int lrows = d - p1;
+        float* ls_hi = reinterpret_cast<float*>(base + L.ls_off) + size_t(sp % 2) * 2 * L.sp_elems;
+        float* ls_lo = ls_hi + L.sp_elems;
+        float* zs_hi = reinterpret_cast<float*>(base + L.zs_off);
+        float* zs_lo = zs_hi + L.sp_elems;
+        const unsigned split_blocks = 148 * 8;
+        if (sp >= 2 && cudaStreamWaitEvent(stream, aux->zfar_done[sp % 2], 0) != cudaSuccess) return GPTQ_ERR_CUDA;
+        split_cols_kernel<<<split_blocks, 256, 0, stream>>>(A + size_t(p1) * d + p0, d, lrows, kd, ls_hi, ls_lo);
+        count_launch();
+        split_cols_kernel<<<split_blocks, 256, 0, as>>>(Z + p0, d, p1, kd, zs_hi, zs_lo);
+        count_launch();
+        if (cudaEventRecord(aux->step, stream) != cudaSuccess || cudaStreamWaitEvent(ss, aux->step, 0) != cudaSuccess ||
+            cudaStreamWaitEvent(as, aux->step, 0) != cudaSuccess)
             return GPTQ_ERR_CUDA;
         if (h1 < d) {
             // columns [h1, d) on `ss`
-            const float* lh = A + size_t(h1) * d + p0;
-            rc = launch_tgemm(d - h1, d - h1, kd, -1.0f, lh, nullptr, d, lh, nullptr, d, true,
-                              A + size_t(h1) * d + h1, d, true, ss, st);
+            const float* hh = ls_hi + size_t(h1 - p1) * kd;
+            const float* hl = ls_lo + size_t(h1 - p1) * kd;
+            rc = launch_tgemm(d - h1, d - h1, kd, -1.0f, hh, hl, kd, hh, hl, kd, true, A + size_t(h1) * d + h1, d,
+                              true, ss, st);
             if (rc) return rc;
         }
         if (cudaEventRecord(aux->far_done[sp % AuxStream::RING], ss) != cudaSuccess) return GPTQ_ERR_CUDA;
@@ -657,12 +701,13 @@ int launch_prepare_hinv(const float* H, int64_t d64, float percdamp, float* U, i
         // update (which covered them)
         if (sp > 0 && cudaStreamWaitEvent(stream, aux->far_done[(sp - 1) % AuxStream::RING], 0) != cudaSuccess)
             return GPTQ_ERR_CUDA;
-        rc = launch_tgemm(d - p1, h1 - p1, kd, -1.0f, lp, nullptr, d, lp, nullptr, d, true, A + size_t(p1) * d + p1, d,
-                          true, stream, st);
+        rc = launch_tgemm(lrows, h1 - p1, kd, -1.0f, ls_hi, ls_lo, kd, ls_hi, ls_lo, kd, true, A + size_t(p1) * d + p1,
+                          d, true, stream, st);
         if (rc) return rc;
         // Z's columns after the super-panel
-        rc = launch_tgemm(p1, d - p1, kd, -1.0f, Z + p0, nullptr, d, lp, nullptr, d, true, Z + p1, d, false, as, st);
+        rc = launch_tgemm(p1, lrows, kd, -1.0f, zs_hi, zs_lo, kd, ls_hi, ls_lo, kd, true, Z + p1, d, false, as, st);
         if (rc) return rc;
+        if (cudaEventRecord(aux->zfar_done[sp % 2], as) != cudaSuccess) return GPTQ_ERR_CUDA;
     }
     // join both auxiliary streams
     if (cudaEventRecord(aux->join, as) != cudaSuccess || cudaStreamWaitEvent(stream, aux->join, 0) != cudaSuccess ||

@@ -13,8 +13,10 @@
 //    shared memory -- no transpose pass over X.
 //  - A cluster of two CTAs (two SMs) owns a tile and runs it as cta_group::2
 //    MMAs (M = 256, N = 256, K = 16, fp32 accumulators in TMEM): CTA r loads
-//    64 calibration rows of its 128 a-columns and of its 128 of the 256
-//    b-columns per stage (32 KB, six stages in flight), and the pair's MMA
+//    128 calibration rows of its 128 a-columns and of its 128 of the 256
+//    b-columns per stage (64 KB, three stages in flight; measured: 64-row
+//    stages with six in flight ran 9% slower, 32-row stages 64% slower, so
+//    the per-stage handshakes cost more than the shallower ring), and the pair's MMA
 //    reads both CTAs' halves.  Per SM that is two thirds of the bytes a
 //    single-CTA 128 x 256 tile would stream for the same MMA work, which is
 //    what lets the loads stay ahead of the tensor cores.  One thread per CTA
@@ -38,20 +40,30 @@
 namespace gptq {
 namespace hess {
 
-constexpr int BK = 64;            // calibration rows per stage
-constexpr int CHUNK = 8;          // k-steps (of BK rows) summed in TMEM before promotion
-constexpr int CHUNK_BYTES = 64 * BK * 2;  // one TMA box: 64 columns x 64 rows of bf16
+// Build-time tuning knobs: calibration rows per stage, rows summed in TMEM
+// before each promotion to fp32 registers, stages in the ring (default: a
+// 192 KB ring).
+#ifndef GPTQ_HESS_BK
+#define GPTQ_HESS_BK 128
+#endif
+#ifndef GPTQ_HESS_PROMOTE_ROWS
+#define GPTQ_HESS_PROMOTE_ROWS 512
+#endif
+constexpr int BK = GPTQ_HESS_BK;            // calibration rows per stage
+constexpr int CHUNK = GPTQ_HESS_PROMOTE_ROWS / BK;   // k-steps (of BK rows) summed in TMEM before promotion
+static_assert(BK % 16 == 0 && BK <= 256 && CHUNK >= 1 && CHUNK * BK == GPTQ_HESS_PROMOTE_ROWS, "Hessian k-steps");
+constexpr int CHUNK_BYTES = 64 * BK * 2;  // one TMA box: 64 columns x BK rows of bf16
 constexpr int EPI_WARPS = 8;              // 4 TMEM lane quadrants x 2 column halves
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr int BMH = 128;                   // H rows per CTA (the pair covers 256)
 constexpr int BNP = 256;                   // H columns per pair (128 loaded by each CTA)
-#ifndef GPTQ_HESS_STAGES
-#define GPTQ_HESS_STAGES 6
-#endif
-constexpr int STAGES = GPTQ_HESS_STAGES;   // a build-time tuning knob
-constexpr int A_BYTES = BMH * BK * 2;      // 16 KB
-constexpr int B_BYTES = (BNP / 2) * BK * 2;  // 16 KB
+constexpr int A_BYTES = BMH * BK * 2;      // 32 KB at BK = 128
+constexpr int B_BYTES = (BNP / 2) * BK * 2;  // 32 KB at BK = 128
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+#ifndef GPTQ_HESS_STAGES
+#define GPTQ_HESS_STAGES (196608 / STAGE_BYTES)
+#endif
+constexpr int STAGES = GPTQ_HESS_STAGES;
 constexpr int TMEM_COLS = 2 * BNP;         // two accumulator buffers
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + size_t(STAGES) * STAGE_BYTES + 256 /*barriers*/;
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
