@@ -466,10 +466,11 @@ def test_mlp28672_full_size_sampled_rows():
     must agree with the oracle up to its first difference, that first
     difference must be a one-level flip at a near-tie (or a grid rounding
     tie), and the layer loss must be within 0.5% of the oracle's; end to end
-    the identical fraction is reported.  The sweep alone is held to the group
-    grids' fraction bound (1 - 2e-6 * 28672 / 2 = 97.1%), to at most 1e-4
-    flips per decision taken from identical states, and to >= 99.9% identical
-    codes over the leading 4096 columns (the width of the benchmark layer)."""
+    the identical fraction is reported.  The sweep alone is held to the
+    general code criteria (tests/parity_util.py: at most 1e-5 flips per
+    decision taken from identical states, plus 2), to at most 1e-4 flips per
+    decision here as well, and to >= 99.9% identical codes over the leading
+    4096 columns (the width of the benchmark layer)."""
     frac, frac_s, got_s, ref_s = _full_size_check(synth.mlp28672(), n_rows_sample=16, match=0.0)
     flips, decisions = decision_stats(got_s, ref_s["codes"])
     assert flips / decisions <= 1e-4
