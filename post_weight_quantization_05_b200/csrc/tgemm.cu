@@ -310,6 +310,197 @@ __global__ void __launch_bounds__(Cfg<PRESPLIT>::THREADS, 1)
     if (warp == 0) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
+// ---------------------------------------------------------------------------
+// The same pre-split three-pass product on SM pairs, for long contractions
+// (the far updates, K = 256 .. 8192).  A cluster of two CTAs owns a 256 x 256
+// output tile and runs it as cta_group::2 MMAs (M = 256, N = 256, K = 8):
+// CTA r loads rows 128 r .. 128 r + 127 of the tile's A rows and of its Bt
+// rows (its half of N), all four operand parts per 32-wide K chunk (64 KB per
+// stage, three stages); both CTAs' loads complete on CTA 0's barrier; CTA 0
+// issues the MMAs, whose commits arrive on both CTAs' barriers; each CTA's
+// TMEM holds its 128 rows x 256 columns (two accumulators, 512 columns).
+// Per SM this streams half the operand bytes of a 128 x 128 tile for the
+// same MMA work, which keeps shared memory below its bandwidth: the single-CTA
+// kernel's three passes over 128 x 128 tiles read and write about 200 bytes
+// of shared memory per clock at full tensor rate, against about 106 here.
+// Persistent: cluster c walks tiles c, c + clusters, ...; no TMA load uses
+// multicast.
+constexpr int PBM = 256, PBN = 256;              // pair tile
+constexpr int P_ROWS = 128;                      // A rows and Bt rows each CTA loads per chunk
+constexpr int P_PART = P_ROWS * BKC * 4;         // 16 KB
+constexpr int P_STAGE = 4 * P_PART;              // A_hi, B_hi, A_lo, B_lo
+constexpr int P_STAGES = 3;
+constexpr int P_EPI_WARP0 = 4;                   // warp % 4 = TMEM lane quadrant
+constexpr int P_THREADS = 32 * (P_EPI_WARP0 + EPI_WARPS);
+constexpr int P_TMEM_COLS = 2 * PBN;
+constexpr size_t P_SMEM_BYTES = 1024 + size_t(P_STAGES) * P_STAGE + size_t(SLAB_BUFS) * SLAB_BYTES + 256;
+static_assert(P_SMEM_BYTES <= 232448, "shared memory");
+
+__host__ __device__ constexpr uint32_t idesc_tf32_pair() {
+    return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(PBN >> 3) << 17) |
+           (static_cast<uint32_t>(PBM >> 4) << 24);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
+    tgemm_pair_kernel(const __grid_constant__ Maps maps, const Args g) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* cbuf = smem + size_t(P_STAGES) * P_STAGE;                                   // [SLAB_BUFS][128 rows][128 B]
+    uint64_t* full = reinterpret_cast<uint64_t*>(cbuf + size_t(SLAB_BUFS) * SLAB_BYTES);  // CTA 0: both halves landed
+    uint64_t* empty = full + P_STAGES;   // both CTAs: the pair's MMAs are done with the stage
+    uint64_t* tfull = empty + P_STAGES;  // [2] both CTAs: accumulator complete
+    uint64_t* tempty = tfull + 2;        // [2] CTA 0: accumulator drained by both CTAs
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    int* epi_abort = reinterpret_cast<int*>(tmem_slot + 1);
+
+    const uint32_t rank = cluster_ctarank();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cl = int(blockIdx.x >> 1), ncl = int(gridDim.x >> 1);
+    const int nk = g.K / BKC;
+    const int my_tiles = g.tiles > cl ? (g.tiles - cl + ncl - 1) / ncl : 0;
+
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&maps.a);
+        tma_prefetch_desc(&maps.b);
+        tma_prefetch_desc(&maps.a_lo);
+        tma_prefetch_desc(&maps.b_lo);
+        tma_prefetch_desc(&maps.c);
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 2 * EPI_WARPS);
+        }
+        *epi_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc_pair(tmem_slot, P_TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();          // barriers of both CTAs initialized, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs)
+            const uint32_t fb0 = mapa_shared(&full[0], 0);
+            int gc = 0;
+            bool ok = true;
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                int tm, tn;
+                tile_coords(cl + lt * ncl, g, tm, tn);
+                const int ar = tm * PBM + int(rank) * P_ROWS, br = tn * PBN + int(rank) * P_ROWS;
+                for (int c = 0; c < nk; ++c, ++gc) {
+                    const int s = gc % P_STAGES;
+                    const uint32_t round = uint32_t(gc / P_STAGES);
+                    if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, g.st, 311)) { ok = false; break; }
+                    uint8_t* base = smem + size_t(s) * P_STAGE;
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * P_STAGE);
+                    const uint32_t fb = fb0 + uint32_t(s) * 8u;
+                    tma_load_2d_pair(base, &maps.a, c * BKC, ar, fb);
+                    tma_load_2d_pair(base + P_PART, &maps.b, c * BKC, br, fb);
+                    tma_load_2d_pair(base + 2 * P_PART, &maps.a_lo, c * BKC, ar, fb);
+                    tma_load_2d_pair(base + 3 * P_PART, &maps.b_lo, c * BKC, br, fb);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer (CTA 0)
+            constexpr uint32_t idesc = idesc_tf32_pair();
+            int gc = 0;
+            bool ok = true;
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                const int acc = lt & 1;
+                const uint32_t use = uint32_t(lt >> 1);
+                if (use > 0 && !mbar_wait_cluster(&tempty[acc], (use - 1) & 1u, g.st, 317)) break;
+                tc_fence_after();
+                const uint32_t dt = tmem_base + uint32_t(acc * PBN);
+                for (int c = 0; c < nk; ++c, ++gc) {
+                    const int s = gc % P_STAGES;
+                    const uint32_t round = uint32_t(gc / P_STAGES);
+                    if (!mbar_wait(&full[s], round & 1u, g.st, 314)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_hi = smem_u32(smem + size_t(s) * P_STAGE), b_hi = a_hi + P_PART;
+                    const uint32_t a_lo = a_hi + 2 * P_PART, b_lo = a_hi + 3 * P_PART;
+#pragma unroll
+                    for (int kk = 0; kk < BKC / 8; ++kk) {
+                        const uint64_t dah = sdesc_sw128(a_hi + kk * 32, 16, 1024);
+                        const uint64_t dal = sdesc_sw128(a_lo + kk * 32, 16, 1024);
+                        const uint64_t dbh = sdesc_sw128(b_hi + kk * 32, 16, 1024);
+                        const uint64_t dbl = sdesc_sw128(b_lo + kk * 32, 16, 1024);
+                        umma_tf32_pair(dt, dah, dbl, idesc, (c > 0 || kk > 0) ? 1u : 0u);   // small terms first
+                        umma_tf32_pair(dt, dal, dbh, idesc, 1u);
+                        umma_tf32_pair(dt, dah, dbh, idesc, 1u);
+                    }
+                    umma_commit_pair_both(&empty[s]);      // the stage may be reloaded in both CTAs
+                }
+                umma_commit_pair_both(&tfull[acc]);        // tile complete (also on the error path)
+            }
+        }
+    } else if (warp >= P_EPI_WARP0) {
+        // ---------------- epilogue (both CTAs): thread et owns row et of this CTA's 128
+        const int quad = warp - P_EPI_WARP0;
+        const int et = threadIdx.x - 32 * P_EPI_WARP0;
+        const uint32_t te = mapa_shared(&tempty[0], 0);
+        volatile int* abort_flag = epi_abort;
+        int gs = 0;
+        for (int lt = 0; lt < my_tiles; ++lt) {
+            const int acc = lt & 1;
+            const uint32_t use = uint32_t(lt >> 1);
+            int tm, tn;
+            tile_coords(cl + lt * ncl, g, tm, tn);
+            if (!mbar_wait(&tfull[acc], use & 1u, g.st, 315)) *abort_flag = 1;
+            named_barrier_sync(EPI_BARRIER, 32 * EPI_WARPS);   // all four warps leave together on a timeout
+            if (*abort_flag) break;
+            tc_fence_after();
+            const int y = tm * PBM + int(rank) * P_ROWS;
+#pragma unroll 1
+            for (int j = 0; j < PBN / SLAB; ++j, ++gs) {
+                float v[32];
+                tmem_ld_32x32b_x32(tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * PBN + j * SLAB), v);
+                if (j == PBN / SLAB - 1) {   // accumulator drained in this CTA
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(te + uint32_t(acc) * 8u);
+                }
+                uint8_t* buf = cbuf + size_t(gs & 1) * SLAB_BYTES;
+                if (et == 0) bulk_wait_group_read<1>();   // the store that last used this buffer has read it
+                named_barrier_sync(EPI_BARRIER, 32 * EPI_WARPS);
+                uint8_t* row = buf + size_t(et) * (SLAB * 4);
+#pragma unroll
+                for (int q = 0; q < SLAB / 4; ++q)
+                    *reinterpret_cast<float4*>(row + ((q ^ (et & 7)) << 4)) =
+                        make_float4(g.alpha * v[4 * q], g.alpha * v[4 * q + 1], g.alpha * v[4 * q + 2],
+                                    g.alpha * v[4 * q + 3]);
+                fence_proxy_async_smem();
+                named_barrier_sync(EPI_BARRIER, 32 * EPI_WARPS);
+                if (et == 0) {
+                    const int x = tn * PBN + j * SLAB;
+                    if (x < g.N && y < g.M) {
+                        if (g.accumulate)
+                            tma_reduce_add_2d(&maps.c, buf, x, y);
+                        else
+                            tma_store_2d(&maps.c, buf, x, y);
+                    }
+                    bulk_commit_group();
+                }
+            }
+        }
+        if (et == 0) bulk_wait_group<0>();   // every store has reached global memory
+    }
+    tc_fence_before();
+    cluster_sync();          // no remote arrival or pair MMA is still pending
+    if (warp == 0) tmem_dealloc_pair(tmem_base, P_TMEM_COLS);
+}
+
 }  // namespace tg
 
 namespace {
@@ -334,6 +525,43 @@ int launch_variant(const tg::Maps& maps, const tg::Args& g, cudaStream_t stream)
     const int n_sms = dev < 64 ? sms[dev].load() : 0;
     const int grid = std::max(1, std::min(g.tiles, n_sms > 0 ? n_sms : 148));
     if (launch_pdl(tg::tgemm_kernel<PRESPLIT>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, maps, g) !=
+        cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    count_launch();
+    return GPTQ_OK;
+}
+// Pre-split products at least this deep (and wider than one 128-row tile in
+// both M and N) run on SM pairs.  A build-time tuning knob.
+#ifndef GPTQ_TGEMM_PAIR_MIN_K
+#define GPTQ_TGEMM_PAIR_MIN_K 256
+#endif
+
+int launch_pair(const tg::Maps& maps, tg::Args g, cudaStream_t stream) {
+    using namespace tg;
+    static std::atomic<bool> attr_set[64];
+    static std::atomic<int> sms[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (dev < 64 && !attr_set[dev]) {
+        int n = 0;
+        if (cudaFuncSetAttribute(tgemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(P_SMEM_BYTES)) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        sms[dev] = n;
+        attr_set[dev] = true;
+    }
+    g.tiles_m = (g.M + PBM - 1) / PBM;
+    g.tiles_n = (g.N + PBN - 1) / PBN;
+    if (g.lower_only) {
+        g.tiles = 0;
+        for (int tm = 0; tm < g.tiles_m; ++tm) g.tiles += std::min(g.tiles_n, tm + 1);
+    } else {
+        g.tiles = g.tiles_m * g.tiles_n;
+    }
+    const int n_sms = dev < 64 ? sms[dev].load() : 0;
+    const int clusters = std::max(1, std::min(g.tiles, (n_sms > 0 ? n_sms : 148) / 2));
+    if (launch_pdl(tgemm_pair_kernel, dim3(2 * clusters), dim3(P_THREADS), P_SMEM_BYTES, stream, maps, g) !=
         cudaSuccess)
         return GPTQ_ERR_CUDA;
     count_launch();
@@ -386,6 +614,7 @@ int launch_tgemm(int M, int N, int K, float alpha, const float* A, const float* 
         g.tiles = g.tiles_m * g.tiles_n;
     }
     g.st = st;
+    if (presplit && K >= GPTQ_TGEMM_PAIR_MIN_K && M > BM && N > BN) return launch_pair(maps, g, stream);
     return presplit ? launch_variant<true>(maps, g, stream) : launch_variant<false>(maps, g, stream);
 }
 

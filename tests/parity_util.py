@@ -20,8 +20,9 @@ Tolerances (stated once, used by every parity test):
            a row of d_in codes is up to rho * d_in / 2, and fp32 arithmetic
            against the fp64 oracle has rho of a few 1e-6.  So the identical
            fraction is held to min(99.9%, 1 - rho_max * d_in / 2), and where a
-           comparison has over 1e5 decisions, the flips themselves to at most
-           rho_max * decisions + 2 (rho_max = RHO_MAX * maxq / 15).
+           comparison on one common U has over 1e5 decisions, the flips
+           themselves to at most rho_max * decisions + 2 (rho_max = RHO_MAX *
+           maxq / 15).
   loss     ||W X^T - W^ X^T||^2 within 0.5% (relative) of the oracle's
   grid     per-row scales/zeros (from the original W) and RTN: bit-exact;
            group scales/zeros: bit-exact given the GPU's own group min/max.
@@ -110,8 +111,11 @@ def grid_flip_at_tie(ref, r, gi, s_gpu, z_gpu):
 
 
 def check_codes(got, ref, what="", match=CODE_MATCH, bits=None, groupsize=-1, gpu_scales=None,
-                gpu_zeros=None):
-    """`ref` is the oracle's output dict (with the trace when available)."""
+                gpu_zeros=None, rate_check=False):
+    """`ref` is the oracle's output dict (with the trace when available).
+    rate_check: also bound the flips per decision (for comparisons on one
+    common U, where the rate measures the sweep's arithmetic; end to end it
+    also depends on how H's fp32 error is amplified by its conditioning)."""
     got = np.asarray(got)
     rc = np.asarray(ref["codes"])
     d_in = rc.shape[1]
@@ -121,7 +125,7 @@ def check_codes(got, ref, what="", match=CODE_MATCH, bits=None, groupsize=-1, gp
     need = min(match, 1.0 - rho * d_in / 2)
     assert frac >= need, f"{what}: only {frac:.6f} of codes identical (need {need:.6f})"
     flips, decisions = decision_stats(got, rc)
-    if decisions > 100000:
+    if rate_check and decisions > 100000:
         assert flips <= rho * decisions + 2, f"{what}: {flips} flips in {decisions} decisions"
     if "W_at" not in ref:
         return frac

@@ -268,7 +268,7 @@ def test_sweep_given_oracle_u(bits, groupsize, d_out, d_in):
     s, z = fp16_values(scales), fp16_values(zeros)
     # finer grids meet more near-ties (fp32 vs fp64 state), hence more flips
     check_codes(got, ref, "sweep", match=CODE_MATCH if bits <= 4 else 0.99, groupsize=groupsize,
-                gpu_scales=s, gpu_zeros=z)
+                gpu_scales=s, gpu_zeros=z, rate_check=True)
     if groupsize < 0:
         assert np.array_equal(s, ref["scales"]) and np.array_equal(z, ref["zeros"])
     else:
@@ -430,7 +430,7 @@ def _full_size_check(p, n_rows_sample=48, seed=0, match=CODE_MATCH, sweep_rows=6
     got_s = unpack_gpu_codes(codes, p.bits, p.d_in)
     ss, zs = fp16_values(scales), fp16_values(zeros)
     frac_s = check_codes(got_s, ref_s, p.name + " (sweep alone)", match=sweep_match, groupsize=p.groupsize,
-                         gpu_scales=ss, gpu_zeros=zs)
+                         gpu_scales=ss, gpu_zeros=zs, rate_check=True)
     Qs = dequant_rows(got_s, ss, zs, p.groupsize)
     lg = oracle.layer_loss_hessian(p.W[srows], Qs, H)
     lo = oracle.layer_loss_hessian(p.W[srows], ref_s["Q"], H)
