@@ -82,6 +82,7 @@ struct Params {
     int tiles;      // T (T + 1) / 2 tiles (ta <= tb) of 256 x 256, T = ceil(d / 256)
     int T;
     int late_wait;  // the previous kernel in the stream is this kernel on another batch
+    int wave;       // SM pairs of the device: tiles t with (t / wave) odd walk the rows backwards
 };
 
 // Launch order of the tiles (ta, tb), ta <= tb.  Pairs that run at the same
@@ -172,13 +173,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- TMA producer (both CTAs)
+            // ---------------- TMA producer (both CTAs).  Tiles of odd waves walk
+            // the calibration rows backwards: they start on the rows the previous
+            // wave read last, which are still in L2 (X of a 16384-row batch is
+            // about the size of L2), instead of on the rows it evicted first.
+            // Measured at 4096 x 16384: DRAM traffic per launch 308 -> 266 MB
+            // (201 MB algorithmic), time unchanged (the kernel is not bound by
+            // DRAM).  An L2 prefetch of X three steps ahead of the ring was
+            // slower (3.62 against 3.41 ms per 16 batches).
+            const bool rev = ((int(blockIdx.x >> 1) / p.wave) & 1) != 0;
             for (int ks = 0; ks < ksteps; ++ks) {
                 const int s = ks % STAGES;
                 const uint32_t round = ks / STAGES;
                 if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, st, 111)) break;
-                const int pair = ks / kper;
-                const int r0 = (ks - pair * kper) * BK;
+                const int kk = rev ? ksteps - 1 - ks : ks;
+                const int pair = kk / kper;
+                const int r0 = (kk - pair * kper) * BK;
                 uint8_t* sa = smem + size_t(s) * STAGE_BYTES;
                 uint8_t* sb = sa + A_BYTES;
                 if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
@@ -334,6 +344,17 @@ int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, voi
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return GPTQ_ERR_CUDA;
     p.late_wait = (after_own_launch && dtype != GPTQ_F32) ? 1 : 0;
+    {
+        static std::atomic<int> sms[64];
+        int dv = 0;
+        if (cudaGetDevice(&dv) != cudaSuccess) return GPTQ_ERR_CUDA;
+        if (dv < 64 && sms[dv].load() == 0) {
+            int n = 0;
+            if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dv) != cudaSuccess) return GPTQ_ERR_CUDA;
+            sms[dv] = n;
+        }
+        p.wave = std::max(1, (dv < 64 ? sms[dv].load() : 148) / 2);
+    }
     p.T = int((d + BNP - 1) / BNP);
     p.tiles = p.T * (p.T + 1) / 2;
     static std::atomic<bool> attr_set[64];
