@@ -82,7 +82,7 @@ struct Params {
     int tiles;      // T (T + 1) / 2 tiles (ta <= tb) of 256 x 256, T = ceil(d / 256)
     int T;
     int late_wait;  // the previous kernel in the stream is this kernel on another batch
-    int wave;       // SM pairs of the device: tiles t with (t / wave) odd walk the rows backwards
+    int wave;       // SM pairs of the device: the launch's clusters (one per pair)
 };
 
 // Launch order of the tiles (ta, tb), ta <= tb.  Pairs that run at the same
@@ -133,10 +133,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
 
     const uint32_t rank = cluster_ctarank();
-    int ta = 0, tb = 0;
-    tile_of(int(blockIdx.x >> 1), p.T, ta, tb);
-    const int a0 = ta * BNP + int(rank) * BMH;   // this CTA's H rows
-    const int b0 = tb * BNP;                     // the pair's H columns
+    // Persistent: cluster cl takes tiles cl, cl + ncl, ... (round lt of its
+    // tiles is wave lt of the launch).  The stage ring and the two TMEM
+    // accumulators run on across tiles, so a tile's loads and MMAs start while
+    // the previous tile's last chunk is promoted and added into H.
+    const int cl = int(blockIdx.x >> 1), ncl = int(gridDim.x >> 1);
+    const int my_tiles = p.tiles > cl ? (p.tiles - cl + ncl - 1) / ncl : 0;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -162,8 +164,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
     // Wait for the previous kernel in the stream before any global access --
     // unless it is this kernel on another batch (late_wait): that one never
-    // writes X, so only the final update of H has to wait for it, and the whole
-    // main loop overlaps its last wave.
+    // writes X, so only the updates of H have to wait for it, and the main
+    // loop overlaps its last tiles.
     if (!p.late_wait) pdl_wait();
     pdl_trigger();
 
@@ -181,54 +183,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // (201 MB algorithmic), time unchanged (the kernel is not bound by
             // DRAM).  An L2 prefetch of X three steps ahead of the ring was
             // slower (3.62 against 3.41 ms per 16 batches).
-            const bool rev = ((int(blockIdx.x >> 1) / p.wave) & 1) != 0;
-            for (int ks = 0; ks < ksteps; ++ks) {
-                const int s = ks % STAGES;
-                const uint32_t round = ks / STAGES;
-                if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, st, 111)) break;
-                const int kk = rev ? ksteps - 1 - ks : ks;
-                const int pair = kk / kper;
-                const int r0 = (kk - pair * kper) * BK;
-                uint8_t* sa = smem + size_t(s) * STAGE_BYTES;
-                uint8_t* sb = sa + A_BYTES;
-                if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
-                const uint32_t fb = mapa_shared(&full[s], 0);
+            int gs = 0;   // stages issued so far, over all tiles
+            bool ok = true;
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                int ta = 0, tb = 0;
+                tile_of(cl + lt * ncl, p.T, ta, tb);
+                const int a0 = ta * BNP + int(rank) * BMH;   // this CTA's H rows
+                const int b0 = tb * BNP;                     // the pair's H columns
+                const bool rev = (lt & 1) != 0;
+                for (int ks = 0; ks < ksteps; ++ks, ++gs) {
+                    const int s = gs % STAGES;
+                    const uint32_t round = uint32_t(gs / STAGES);
+                    if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, st, 111)) { ok = false; break; }
+                    const int kk = rev ? ksteps - 1 - ks : ks;
+                    const int pair = kk / kper;
+                    const int r0 = (kk - pair * kper) * BK;
+                    uint8_t* sa = smem + size_t(s) * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
+                    const uint32_t fb = mapa_shared(&full[s], 0);
 #pragma unroll
-                for (int h = 0; h < BMH / 64; ++h)
-                    tma_load_3d_pair(sa + h * CHUNK_BYTES, &tmX, a0 + 64 * h, r0, p.pa[pair], fb);
+                    for (int h = 0; h < BMH / 64; ++h)
+                        tma_load_3d_pair(sa + h * CHUNK_BYTES, &tmX, a0 + 64 * h, r0, p.pa[pair], fb);
 #pragma unroll
-                for (int h = 0; h < BNP / 128; ++h)
-                    tma_load_3d_pair(sb + h * CHUNK_BYTES, &tmX, b0 + int(rank) * 128 + 64 * h, r0, p.pb[pair], fb);
+                    for (int h = 0; h < BNP / 128; ++h)
+                        tma_load_3d_pair(sb + h * CHUNK_BYTES, &tmX, b0 + int(rank) * 128 + 64 * h, r0, p.pb[pair],
+                                         fb);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             // ---------------- MMA issuer (CTA 0 only)
             constexpr uint32_t idesc = idesc_bf16_mn_mn(2 * BMH, BNP);
+            int gs = 0, gc = 0;   // stages and chunks consumed so far, over all tiles
             bool ok = true;
-            for (int c = 0; c < nchunks && ok; ++c) {
-                const int buf = c & 1;
-                const int use = c >> 1;
-                if (use > 0 && !mbar_wait_cluster(&tempty[buf], uint32_t(use - 1) & 1u, st, 115)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t dt = tmem_base + uint32_t(buf * BNP);
-                const int k_end = min(ksteps, (c + 1) * CHUNK);
-                for (int ks = c * CHUNK; ks < k_end; ++ks) {
-                    const int s = ks % STAGES;
-                    const uint32_t round = ks / STAGES;
-                    if (!mbar_wait(&full[s], round & 1u, st, 112)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + size_t(s) * STAGE_BYTES);
-                    const uint32_t sb = sa + A_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t da = sdesc_sw128(sa + kk * 2048, CHUNK_BYTES, 1024);
-                        const uint64_t db = sdesc_sw128(sb + kk * 2048, CHUNK_BYTES, 1024);
-                        umma_f16_pair(dt, da, db, idesc, (ks > c * CHUNK || kk > 0) ? 1u : 0u);
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                for (int c = 0; c < nchunks && ok; ++c, ++gc) {
+                    const int buf = gc & 1;
+                    const int use = gc >> 1;
+                    if (use > 0 && !mbar_wait_cluster(&tempty[buf], uint32_t(use - 1) & 1u, st, 115)) {
+                        ok = false;
+                        break;
                     }
-                    umma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
+                    tc_fence_after();
+                    const uint32_t dt = tmem_base + uint32_t(buf * BNP);
+                    const int k_end = min(ksteps, (c + 1) * CHUNK);
+                    for (int ks = c * CHUNK; ks < k_end; ++ks, ++gs) {
+                        const int s = gs % STAGES;
+                        const uint32_t round = uint32_t(gs / STAGES);
+                        if (!mbar_wait(&full[s], round & 1u, st, 112)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t sa = smem_u32(smem + size_t(s) * STAGE_BYTES);
+                        const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t da = sdesc_sw128(sa + kk * 2048, CHUNK_BYTES, 1024);
+                            const uint64_t db = sdesc_sw128(sb + kk * 2048, CHUNK_BYTES, 1024);
+                            umma_f16_pair(dt, da, db, idesc, (ks > c * CHUNK || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit_pair_both(&empty[s]);   // frees the stage in both CTAs
+                    }
+                    umma_commit_pair_both(&tfull[buf]);     // chunk complete (also on the error path)
                 }
-                umma_commit_pair_both(&tfull[buf]);     // chunk complete (also on the error path)
             }
         }
     } else {
@@ -238,48 +255,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int half = e >> 2;
         const uint32_t lane_addr = uint32_t(quad * 32) << 16;
         const uint32_t te = mapa_shared(&tempty[0], 0);   // CTA 0's tempty[0]; [1] is 8 bytes on
-        float acc[128];
-#pragma unroll
-        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+        int gc = 0;
         bool ok = true;
-        for (int c = 0; c < nchunks; ++c) {
-            const int buf = c & 1;
-            const int use = c >> 1;
-            if (!mbar_wait(&tfull[buf], uint32_t(use) & 1u, st, 113)) { ok = false; break; }
-            tc_fence_after();
+        for (int lt = 0; lt < my_tiles && ok; ++lt) {
+            int ta = 0, tb = 0;
+            tile_of(cl + lt * ncl, p.T, ta, tb);
+            const int a0 = ta * BNP + int(rank) * BMH;
+            const int b0 = tb * BNP;
+            float acc[128];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float v[32];
-                tmem_ld_32x32b_x32(tmem_base + lane_addr + uint32_t(buf * BNP + half * 128 + cc * 32), v);
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            for (int c = 0; c < nchunks; ++c, ++gc) {
+                const int buf = gc & 1;
+                const int use = gc >> 1;
+                if (!mbar_wait(&tfull[buf], uint32_t(use) & 1u, st, 113)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) acc[cc * 32 + i] += v[i];
+                for (int cc = 0; cc < 4; ++cc) {
+                    float v[32];
+                    tmem_ld_32x32b_x32(tmem_base + lane_addr + uint32_t(buf * BNP + half * 128 + cc * 32), v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[cc * 32 + i] += v[i];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(te + uint32_t(buf) * 8u);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(te + uint32_t(buf) * 8u);
-        }
-        const int a = a0 + quad * 32 + lane;   // TMEM lane == row of this CTA's half
-        if (p.late_wait) pdl_wait();           // the previous batch's H is complete
-        if (ok && nchunks > 0 && a < p.d) {
-            float* hrow = H + size_t(a) * p.d;
+            const int a = a0 + quad * 32 + lane;   // TMEM lane == row of this CTA's half
+            if (p.late_wait) pdl_wait();           // the previous batch's H is complete
+            if (ok && nchunks > 0 && a < p.d) {
+                float* hrow = H + size_t(a) * p.d;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const int b = b0 + half * 128 + cc * 32;
-                if (b + 32 <= p.d) {
-                    float4* dst = reinterpret_cast<float4*>(hrow + b);
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int b = b0 + half * 128 + cc * 32;
+                    if (b + 32 <= p.d) {
+                        float4* dst = reinterpret_cast<float4*>(hrow + b);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float4 h = dst[q];
-                        h.x = fmaf(p.alpha, acc[cc * 32 + 4 * q + 0], h.x);
-                        h.y = fmaf(p.alpha, acc[cc * 32 + 4 * q + 1], h.y);
-                        h.z = fmaf(p.alpha, acc[cc * 32 + 4 * q + 2], h.z);
-                        h.w = fmaf(p.alpha, acc[cc * 32 + 4 * q + 3], h.w);
-                        dst[q] = h;
+                        for (int q = 0; q < 8; ++q) {
+                            float4 h = dst[q];
+                            h.x = fmaf(p.alpha, acc[cc * 32 + 4 * q + 0], h.x);
+                            h.y = fmaf(p.alpha, acc[cc * 32 + 4 * q + 1], h.y);
+                            h.z = fmaf(p.alpha, acc[cc * 32 + 4 * q + 2], h.z);
+                            h.w = fmaf(p.alpha, acc[cc * 32 + 4 * q + 3], h.w);
+                            dst[q] = h;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            if (b + q < p.d) hrow[b + q] = fmaf(p.alpha, acc[cc * 32 + q], hrow[b + q]);
                     }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 32; ++q)
-                        if (b + q < p.d) hrow[b + q] = fmaf(p.alpha, acc[cc * 32 + q], hrow[b + q]);
                 }
             }
         }
@@ -366,7 +390,8 @@ int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, voi
             return GPTQ_ERR_CUDA;
         attr_set[dev] = true;
     }
-    if (launch_pdl(syrk_pair_kernel, dim3(2 * p.tiles), dim3(THREADS), SMEM_BYTES, stream, tm, p, H, st) !=
+    const int clusters = std::max(1, std::min(p.tiles, p.wave));
+    if (launch_pdl(syrk_pair_kernel, dim3(2 * clusters), dim3(THREADS), SMEM_BYTES, stream, tm, p, H, st) !=
         cudaSuccess)
         return GPTQ_ERR_CUDA;
     count_launch();
