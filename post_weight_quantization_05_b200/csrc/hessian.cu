@@ -65,9 +65,12 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 #endif
 constexpr int STAGES = GPTQ_HESS_STAGES;
 constexpr int TMEM_COLS = 2 * BNP;         // two accumulator buffers
-constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + size_t(STAGES) * STAGE_BYTES + 256 /*barriers*/;
+constexpr int FLUSH_COLS = 32;                       // columns of H per reduce-add
+constexpr int FLUSH_BYTES = BMH * FLUSH_COLS * 4;    // one staged slab: 128 rows x 32 fp32 (16 KB)
+constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + size_t(STAGES) * STAGE_BYTES +
+                              2 * size_t(FLUSH_BYTES) /*one staging slab per column half*/ + 256 /*barriers*/;
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
-static_assert((2 * STAGES + 4) * 8 + 4 <= 256, "barrier area");
+static_assert((2 * STAGES + 4) * 8 + 4 + 8 <= 256, "barrier area");
 
 // Pair protocol: CTA r (r = 0, 1) loads a-columns a0 + 128 r .. + 127 and
 // b-columns b0 + 128 r .. + 127 of each slab; both CTAs' TMA loads complete on
@@ -122,15 +125,17 @@ __device__ __forceinline__ void tile_of(int t, int T, int& ta, int& tb) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    syrk_pair_kernel(const __grid_constant__ CUtensorMap tmX, const Params p, float* __restrict__ H,
+    syrk_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmH, const Params p,
                      DevStatus* st) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(STAGES) * STAGE_BYTES);  // CTA 0: both halves landed
+    uint8_t* flush_buf = smem + size_t(STAGES) * STAGE_BYTES;                            // [2][FLUSH_BYTES]
+    uint64_t* full = reinterpret_cast<uint64_t*>(flush_buf + 2 * size_t(FLUSH_BYTES));    // CTA 0: both halves landed
     uint64_t* empty = full + STAGES;    // both CTAs: the pair's MMAs are done with the stage
     uint64_t* tfull = empty + STAGES;   // [2] both CTAs: chunk summed in buffer b
     uint64_t* tempty = tfull + 2;       // [2] CTA 0: buffer b drained by both CTAs
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    int* half_abort = reinterpret_cast<int*>(tmem_slot + 1);   // [2] an epilogue half gave up on a wait
 
     const uint32_t rank = cluster_ctarank();
     // Persistent: cluster cl takes tiles cl, cl + ncl, ... (round lt of its
@@ -151,6 +156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 2 * EPI_WARPS);
+            half_abort[b] = 0;
         }
         fence_mbar_init();
     }
@@ -257,7 +263,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const uint32_t te = mapa_shared(&tempty[0], 0);   // CTA 0's tempty[0]; [1] is 8 bytes on
         int gc = 0;
         bool ok = true;
-        for (int lt = 0; lt < my_tiles && ok; ++lt) {
+        volatile int* abort_flag = half_abort + half;
+        for (int lt = 0; lt < my_tiles; ++lt) {
             int ta = 0, tb = 0;
             tile_of(cl + lt * ncl, p.T, ta, tb);
             const int a0 = ta * BNP + int(rank) * BMH;
@@ -281,32 +288,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(te + uint32_t(buf) * 8u);
             }
-            const int a = a0 + quad * 32 + lane;   // TMEM lane == row of this CTA's half
+            // 2 * sum into H: the half's four warps stage 32 columns of their 128
+            // rows at a time in shared memory (128-byte swizzle) and one thread
+            // adds them into H with a TMA reduce-add, which the L2 applies as one
+            // rounded fp32 addition per element (the same result as h + 2 sum
+            // in the SM), without the SM waiting for H's old values.
+            // the half's four warps decide together (a named barrier has no time
+            // limit, so none may skip the ones below alone)
+            if (!ok) *abort_flag = 1;
+            named_barrier_sync(1 + half, 32 * EPI_WARPS / 2);
+            if (*abort_flag) break;
             if (p.late_wait) pdl_wait();           // the previous batch's H is complete
-            if (ok && nchunks > 0 && a < p.d) {
-                float* hrow = H + size_t(a) * p.d;
+            if (nchunks > 0) {
+                const int row = quad * 32 + lane;  // TMEM lane == row of this CTA's 128
+                uint8_t* buf = flush_buf + size_t(half) * FLUSH_BYTES;
+                const bool issuer = (quad == 0 && lane == 0);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
-                    const int b = b0 + half * 128 + cc * 32;
-                    if (b + 32 <= p.d) {
-                        float4* dst = reinterpret_cast<float4*>(hrow + b);
+                    if (issuer) bulk_wait_group_read<0>();   // the last reduce from this slab has read it
+                    named_barrier_sync(1 + half, 32 * EPI_WARPS / 2);
+                    uint8_t* rowp = buf + size_t(row) * (FLUSH_COLS * 4);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 h = dst[q];
-                            h.x = fmaf(p.alpha, acc[cc * 32 + 4 * q + 0], h.x);
-                            h.y = fmaf(p.alpha, acc[cc * 32 + 4 * q + 1], h.y);
-                            h.z = fmaf(p.alpha, acc[cc * 32 + 4 * q + 2], h.z);
-                            h.w = fmaf(p.alpha, acc[cc * 32 + 4 * q + 3], h.w);
-                            dst[q] = h;
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q)
-                            if (b + q < p.d) hrow[b + q] = fmaf(p.alpha, acc[cc * 32 + q], hrow[b + q]);
+                    for (int q = 0; q < FLUSH_COLS / 4; ++q)
+                        *reinterpret_cast<float4*>(rowp + ((q ^ (row & 7)) << 4)) =
+                            make_float4(p.alpha * acc[cc * 32 + 4 * q], p.alpha * acc[cc * 32 + 4 * q + 1],
+                                        p.alpha * acc[cc * 32 + 4 * q + 2], p.alpha * acc[cc * 32 + 4 * q + 3]);
+                    fence_proxy_async_smem();
+                    named_barrier_sync(1 + half, 32 * EPI_WARPS / 2);
+                    if (issuer) {
+                        tma_reduce_add_2d(&tmH, buf, b0 + half * 128 + cc * FLUSH_COLS, a0);
+                        bulk_commit_group();
                     }
                 }
             }
         }
+        if (quad == 0 && lane == 0) bulk_wait_group<0>();   // every reduce has reached H
     }
     tc_fence_before();
     cluster_sync();          // no remote arrival or pair MMA is still pending
@@ -391,7 +407,18 @@ int launch_hessian(const void* X, int dtype, int64_t n, int64_t d, float* H, voi
         attr_set[dev] = true;
     }
     const int clusters = std::max(1, std::min(p.tiles, p.wave));
-    if (launch_pdl(syrk_pair_kernel, dim3(2 * clusters), dim3(THREADS), SMEM_BYTES, stream, tm, p, H, st) !=
+    CUtensorMap tmH;   // H as fp32 [d, d], boxes of 32 columns x 128 rows, 128-byte swizzle
+    {
+        const cuuint64_t hd[2] = {cuuint64_t(d), cuuint64_t(d)};
+        const cuuint64_t hs[1] = {cuuint64_t(d) * 4};
+        const cuuint32_t hb[2] = {FLUSH_COLS, BMH};
+        const cuuint32_t he[2] = {1, 1};
+        if (encode(&tmH, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, H, hd, hs, hb, he, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GPTQ_ERR_CUDA;
+    }
+    if (launch_pdl(syrk_pair_kernel, dim3(2 * clusters), dim3(THREADS), SMEM_BYTES, stream, tm, tmH, p, st) !=
         cudaSuccess)
         return GPTQ_ERR_CUDA;
     count_launch();
