@@ -125,11 +125,15 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // One 128 x 128 diagonal block: L L^T = A_kk and L^-1, in one CTA of 12 warps.
 // The block is cut into 4 x 4 sub-blocks of 32.  Step kb (o = 32 kb):
-//   A: warp 0 factors the diagonal sub-block (kb, kb) in registers; the warps
-//      on the other three schedulers meanwhile finish step kb-1: its trailing
-//      update beyond block column kb and its step of the inverse's update;
-//   B: warp 0 inverts the diagonal sub-block; warps 1-3 solve the sub-blocks
-//      below against it (one row per thread);
+//   A: warp 0 (the leader) runs the Cholesky of the diagonal sub-block
+//      (kb, kb) in registers, lane = row, and publishes each column of L_kk
+//      and 1 / L[c][c] in shared memory, in groups of columns.  Followers
+//      trail it group by group: warp w in 1 .. 3-kb solves rows o + 32 w +
+//      lane of the panel below against L_kk^T, and warp YW builds column
+//      `lane` of L_kk^-1 (forward substitution on e_lane).  Meanwhile the
+//      other warps (not those sharing the leader's scheduler) finish step
+//      kb-1: its trailing update beyond block column kb and its step of the
+//      inverse's update.
 //   C: the trailing update of block column kb+1 (what step kb+1 needs first)
 //      and step kb of the inverse's block solve.
 // The inverse Y = L^-1 is built right-looking on the identity (Y = X after
@@ -140,97 +144,89 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 constexpr int SB = 32;
 constexpr int LDS = NB + 4;              // S and Yt row stride (floats)
-constexpr int LDI = SB + 4;              // Lr row stride
-constexpr int DIAG_THREADS = 384;           // 12 warps
-constexpr int LDD = NB + 1;              // stride of the transposed inverse before it is written out
-constexpr size_t DIAG_SMEM = (size_t(2) * NB * LDS + size_t(SB) * LDI + 2 * SB + NB) * sizeof(float);
+constexpr int LDI = SB + 4;              // Lr and Lp row stride
+constexpr int DIAG_THREADS = 384;        // 12 warps
+constexpr int YW = 5;                    // the follower that builds L_kk^-1 (not on the leader's scheduler)
+constexpr size_t DIAG_SMEM = (size_t(2) * NB * LDS + size_t(2) * SB * LDI + SB) * sizeof(float);
 
-// The 32 x 32 pieces are template recursions so that every register index is
-// a compile-time constant (a rolled loop would put the row in local memory).
+// The leader's columns are published in groups of GROUP steps; group g of
+// sub-block kb completes mbarrier 4 kb + g (each used once, so every wait is
+// for phase 0).  Followers sleep in the barrier's bounded wait instead of
+// polling shared memory beside the leader.
+constexpr int GROUP = 8;
+constexpr int NGROUPS = (NB / SB) * (SB / GROUP);
 
-// Right-looking Cholesky of a 32 x 32 block by one warp, lane = row: a[] holds
-// row `lane` (entries j > lane are don't-care).  Step C reads column C of the
-// current matrix from cb[C & 1] (each lane published its own entry), and every
-// lane applies  a[j] -= a[lane][C] a[j][C] / a[C][C]  with the unscaled column,
-// so the only serial work per step is one rsqrt; a[C] is then scaled to
-// L[lane][C] and entry C+1 is published for the next step.
+// Leader step C (template recursion keeps every register index a
+// compile-time constant).  a[] holds row `lane` of the sub-block (entries
+// right of the diagonal are don't-care); piv is entry (C, C) after the steps
+// before C.  Column C is scaled to L's (l = a[C] / sqrt(piv)), published as
+// row C of Lp (Lp[C][j] = L[j][C]) with rs[C] = 1 / L[C][C], and l * L[j][C]
+// is subtracted from every a[j], j > C.  The next pivot comes from lane C+1's
+// own l by a shuffle, beside the shared-memory round trip.  After every
+// GROUP steps lane 0 arrives on the group's barrier (release: the warp's
+// published columns become visible to the followers' waits).
 template <int C>
-struct RowChol32 {
-    __device__ __forceinline__ static void run(float (&a)[SB], int lane, float* __restrict__ cb,
-                                               float* __restrict__ invd, uint32_t& bad, uint32_t& nonfinite) {
-        const float* cin = cb + (C & 1) * SB;
-        const float piv = cin[C];
+struct LeadStep {
+    __device__ __forceinline__ static void run(float (&a)[SB], float piv, int lane, float* __restrict__ Lp,
+                                               float* __restrict__ rs_out, uint64_t* grp, uint32_t& bad,
+                                               uint32_t& nonfinite) {
         bad |= uint32_t(!(piv > 0.0f && isfinite(piv))) << C;   // bit C: pivot C failed
         nonfinite |= uint32_t(!isfinite(piv)) << C;
-        const float inv = rsqrtf(piv);
-        const float lm = a[C] * (inv * inv);
-#pragma unroll
-        for (int j4 = ((C + 1) / 4) * 4; j4 < SB; j4 += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(cin + j4);
-            if (j4 + 0 > C) a[j4 + 0] = fmaf(-lm, v.x, a[j4 + 0]);
-            if (j4 + 1 > C) a[j4 + 1] = fmaf(-lm, v.y, a[j4 + 1]);
-            if (j4 + 2 > C) a[j4 + 2] = fmaf(-lm, v.z, a[j4 + 2]);
-            if (j4 + 3 > C) a[j4 + 3] = fmaf(-lm, v.w, a[j4 + 3]);
-        }
-        a[C] *= inv;
-        invd[C] = inv;
+        const float rs = rsqrtf(piv);
+        const float l = a[C] * rs;
+        a[C] = l;
+        float* col = Lp + C * LDI;
+        col[lane] = l;
+        rs_out[C] = rs;   // every lane: the same value, one broadcast write, no branch
         if constexpr (C + 1 < SB) {
-            cb[((C + 1) & 1) * SB + lane] = a[C + 1];
+            const float next = __shfl_sync(0xffffffffu, fmaf(-l, l, a[C + 1]), C + 1);
             __syncwarp();
-            RowChol32<C + 1>::run(a, lane, cb, invd, bad, nonfinite);
+            if constexpr ((C + 1) % GROUP == 0) {
+                if (lane == 0) mbar_arrive(grp + (C + 1) / GROUP - 1);
+            }
+#pragma unroll
+            for (int j4 = ((C + 1) / 4) * 4; j4 < SB; j4 += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(col + j4);
+                const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (j4 + q > C) a[j4 + q] = fmaf(-l, v[q], a[j4 + q]);
+            }
+            LeadStep<C + 1>::run(a, next, lane, Lp, rs_out, grp, bad, nonfinite);
+        } else {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(grp + SB / GROUP - 1);
         }
     }
 };
 
-// Warp-level Cholesky of one 32 x 32 diagonal sub-block in place: `row` is
-// this lane's row (row stride LDS in shared memory).  Kept out of line so that
-// its registers are allocated on their own, away from the rest of the kernel.
-__device__ __noinline__ void chol_sub_block(float* __restrict__ row, int lane, float* __restrict__ cb,
-                                            float* __restrict__ invd, uint32_t* badmask, uint32_t* nonfinite) {
-    float a[SB];
-#pragma unroll
-    for (int j = 0; j < SB; j += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(row + j);
-        a[j] = v.x; a[j + 1] = v.y; a[j + 2] = v.z; a[j + 3] = v.w;
-    }
-    cb[lane] = a[0];
-    __syncwarp();
-    uint32_t bad = 0, nf = 0;
-    RowChol32<0>::run(a, lane, cb, invd, bad, nf);
-#pragma unroll
-    for (int j = 0; j < SB; j += 4)
-        *reinterpret_cast<float4*>(row + j) =
-            make_float4(j <= lane ? a[j] : 0.0f, j + 1 <= lane ? a[j + 1] : 0.0f, j + 2 <= lane ? a[j + 2] : 0.0f,
-                        j + 3 <= lane ? a[j + 3] : 0.0f);
-    *badmask = bad;
-    *nonfinite = nf;
-}
-
-// One row x[] (32 values) solved against L (32 x 32 lower, shared memory,
-// row stride LDS):  x <- x L^-T  (right-looking, invd[c] = 1/L[c][c]).
+// Follower step C: once the leader has published column C, x[C] is scaled by
+// 1 / L[C][C] and x[j] -= x[C] L[j][C] for j > C.  With x = a panel row that
+// is the solve x <- x L^-T; with x = e_lane it builds column `lane` of L^-1.
+// A follower waits once per group of columns.  After a wait that timed out
+// (ok == false) the remaining steps run without waiting; the kernel then
+// stops at its next barrier.
 template <int C>
-struct Trsm32 {
-    __device__ __forceinline__ static void run(float (&x)[SB], const float* __restrict__ L,
-                                               const float* __restrict__ invd) {
-        const float xc = x[C] * invd[C];
+struct FollowStep {
+    __device__ __forceinline__ static void run(float (&x)[SB], const float* __restrict__ Lp,
+                                               const float* __restrict__ rs, uint64_t* grp, bool& ok, DevStatus* st) {
+        if constexpr (C % GROUP == 0) {
+            if (ok) ok = mbar_wait(grp + C / GROUP, 0, st, 0x600 + C);
+        }
+        const float xc = x[C] * rs[C];
         x[C] = xc;
+        if constexpr (C + 1 < SB) {
+            const float* col = Lp + C * LDI;
 #pragma unroll
-        for (int j = C + 1; j < SB; ++j) x[j] = fmaf(-xc, L[j * LDS + C], x[j]);
-        if constexpr (C + 1 < SB) Trsm32<C + 1>::run(x, L, invd);
-    }
-};
-
-// Column `lane` of L^-1 for a 32 x 32 lower L (shared memory, row stride LDS)
-// by forward substitution on e_lane; reads of L are broadcasts.
-template <int I>
-struct ColInv32 {
-    __device__ __forceinline__ static void run(float (&y)[SB], const float* __restrict__ L,
-                                               const float* __restrict__ invd) {
-        const float yi = y[I] * invd[I];
-        y[I] = yi;
+            for (int j4 = ((C + 1) / 4) * 4; j4 < SB; j4 += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(col + j4);
+                const float v[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-        for (int r = I + 1; r < SB; ++r) y[r] = fmaf(-L[r * LDS + I], yi, y[r]);
-        if constexpr (I + 1 < SB) ColInv32<I + 1>::run(y, L, invd);
+                for (int q = 0; q < 4; ++q)
+                    if (j4 + q > C) x[j4 + q] = fmaf(-xc, v[q], x[j4 + q]);
+            }
+            FollowStep<C + 1>::run(x, Lp, rs, grp, ok, st);
+        }
     }
 };
 
@@ -270,6 +266,60 @@ __device__ __forceinline__ void sub_block_update(const float* __restrict__ P, co
         for (int b = 0; b < 4; ++b) Out[(r0 + g + 8 * a) * LDS + c0 + 16 * s + h + 4 * b] -= acc[a][b];
 }
 
+// Phase A of step kb for the leader: the Cholesky of the diagonal sub-block
+// (its factor is not written back: nothing reads L_kk afterwards).  Kept out
+// of line, like the followers, so that its registers are allocated on their
+// own, away from the rest of the kernel.
+__device__ __noinline__ void lead_warp(const float* __restrict__ S, float* __restrict__ Lp, float* __restrict__ rs,
+                                       uint64_t* grp, int o, int lane, uint32_t* badmask, uint32_t* nonfinite) {
+    float a[SB];
+    const float* arow = S + (o + lane) * LDS + o;
+#pragma unroll
+    for (int j = 0; j < SB; j += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(arow + j);
+        a[j] = v.x; a[j + 1] = v.y; a[j + 2] = v.z; a[j + 3] = v.w;
+    }
+    uint32_t bad = 0, nf = 0;
+    LeadStep<0>::run(a, __shfl_sync(0xffffffffu, a[0], 0), lane, Lp, rs, grp, bad, nf);
+    *badmask = bad;
+    *nonfinite = nf;
+}
+
+// Phase A of step kb for a follower: row_group = w >= 1 solves rows
+// o + 32 w + lane of the panel in place; row_group = 0 builds column `lane`
+// of L_kk^-1 and writes it as Yt row o + lane and into Lr (row-major).
+// Returns false if a wait for the leader timed out.
+__device__ __noinline__ bool follow_warp(float* __restrict__ S, float* __restrict__ Yt, float* __restrict__ Lr,
+                                         const float* __restrict__ Lp, const float* __restrict__ rs, uint64_t* grp,
+                                         int o, int row_group, int lane, DevStatus* st) {
+    float x[SB];
+    float* xrow = S + (o + SB * row_group + lane) * LDS + o;
+    if (row_group == 0) {
+#pragma unroll
+        for (int j = 0; j < SB; ++j) x[j] = (j == lane) ? 1.0f : 0.0f;
+    } else {
+#pragma unroll
+        for (int j = 0; j < SB; j += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(xrow + j);
+            x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
+        }
+    }
+    bool ok = true;
+    FollowStep<0>::run(x, Lp, rs, grp, ok, st);
+    if (row_group == 0) {
+#pragma unroll
+        for (int r = 0; r < SB; r += 4)
+            *reinterpret_cast<float4*>(Yt + (o + lane) * LDS + o + r) = make_float4(x[r], x[r + 1], x[r + 2], x[r + 3]);
+#pragma unroll
+        for (int r = 0; r < SB; ++r) Lr[r * LDI + lane] = x[r];
+    } else {
+#pragma unroll
+        for (int j = 0; j < SB; j += 4)
+            *reinterpret_cast<float4*>(xrow + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+    }
+    return ok;
+}
+
 // Factor the diagonal block A[k0:k0+NB, k0:k0+NB] = L L^T and write
 //   Dinv = L^-1 (NB x NB row-major, zeros above the diagonal) and
 //   Z[k0 + c][k0 + r] = L^-1[r][c]  (the diagonal block of Z = L'^-T).
@@ -282,9 +332,10 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
     float* S = sm;                     // [NB][LDS] the block, factored in place (lower)
     float* Yt = S + NB * LDS;          // [NB][LDS] X, then Y, transposed (upper)
     float* Lr = Yt + NB * LDS;         // [SB][LDI] L_kk^-1 of the current step, row-major
-    float* cb = Lr + SB * LDI;         // [2][SB] published column (Cholesky steps)
-    float* invd = cb + 2 * SB;         // [NB] 1 / L[c][c]
+    float* Lp = Lr + SB * LDI;         // [SB][LDI] the leader's published columns: Lp[c][j] = L_kk[j][c]
+    float* rs = Lp + SB * LDI;         // [SB] 1 / L_kk[c][c]
     __shared__ int failed;
+    __shared__ __align__(8) uint64_t grp_bar[NGROUPS];   // the leader's column groups, one barrier per group
     pdl_wait();
     pdl_trigger();
     if (*info != 0) return;
@@ -315,35 +366,43 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
             *reinterpret_cast<float4*>(Yt + r * LDS + c) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
     }
-    if (t == 0) failed = 0;
+    if (t == 0) {
+        failed = 0;
+        for (int g = 0; g < NGROUPS; ++g) mbar_init(&grp_bar[g], 1);
+    }
     __syncthreads();
 
     for (int kb = 0; kb < NB / SB; ++kb) {
         const int o = kb * SB;
-        // ---- A: factor the diagonal sub-block (warp 0) || inverse update of step kb-1
+        const int npanel = NB / SB - kb;   // 32-row groups of block column kb
+        // ---- A: Cholesky (leader) || panel solve and L_kk^-1 (followers) || rest of step kb-1
         if (warp == 0) {
             uint32_t badmask = 0, nonfinite = 0;   // the same in every lane
-            chol_sub_block(S + (o + lane) * LDS + o, lane, cb, invd + o, &badmask, &nonfinite);
+            lead_warp(S, Lp, rs, grp_bar + kb * (SB / GROUP), o, lane, &badmask, &nonfinite);
             if (badmask != 0 && lane == 0) {   // the first failing pivot of this sub-block
                 const int bad = __ffs(int(badmask)) - 1;
                 failed = 1;
                 if (atomicCAS(info, 0, k0 + o + bad + 1) == 0)
                     record_error(st, (nonfinite >> bad) & 1u ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_PD, k0 + o + bad + 1);
             }
-        } else if ((warp & 3) != 0 && kb > 0) {
-            // Work of step kb-1 that step kb's Cholesky does not wait for, on the
-            // warps that do not share warp 0's scheduler:
+        } else if (warp < npanel || warp == YW) {
+            if (!follow_warp(S, Yt, Lr, Lp, rs, grp_bar + kb * (SB / GROUP), o, warp == YW ? 0 : warp, lane, st))
+                failed = 1;
+        } else if (kb > 0 && (warp & 3) != 0) {
+            // Work of step kb-1 that step kb's panel does not wait for, on the
+            // warps other than YW that do not share the leader's scheduler:
             //  - the trailing update of step kb-1 beyond block column kb:
             //    pairs (bi, bj), kb < bj <= bi;
             //  - X_ij -= L_{i,kb-1} Y_{kb-1,j} for i >= kb, j < kb, transposed:
             //    Yt[j-block][i-block] -= Yt[j-block][(kb-1)-block] S[i-block][(kb-1)-block]^T.
-            const int w = warp - 1 - (warp >> 2);              // 0 .. 3 * DIAG_THREADS / 128 - 1
+            const int w = warp - npanel - (warp > 4) - (warp > YW) - (warp > 8);
+            const int nw = DIAG_THREADS / 32 - npanel - 3;
             const int nf = NB / SB - kb - 1;                   // sub-block columns after kb
             const int far_tasks = nf * (nf + 1);               // two per pair
             const int nj = kb, ni = NB / SB - kb;
             const int tasks = far_tasks + 2 * ni * nj;
             const int po = (kb - 1) * SB;
-            for (int task = w; task < tasks; task += 3 * DIAG_THREADS / 128) {
+            for (int task = w; task < tasks; task += nw) {
                 if (task < far_tasks) {
                     int p = task >> 1, bi = kb + 1;
                     while (p > bi - (kb + 1)) { p -= bi - kb; ++bi; }
@@ -359,38 +418,10 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
         __syncthreads();
         if (failed) return;
 
-        // ---- B: invert the diagonal sub-block (warp 0) || solve the rows below (warps 1-3)
-        const int below = NB - o - SB;
-        if (warp == 0) {
-            float y[SB];
-#pragma unroll
-            for (int r = 0; r < SB; ++r) y[r] = (r == lane) ? 1.0f : 0.0f;
-            ColInv32<0>::run(y, S + o * LDS + o, invd + o);
-            // Yt rows o + lane (= column lane of L_kk^-1) and Lr (row-major copy)
-#pragma unroll
-            for (int r = 0; r < SB; r += 4)
-                *reinterpret_cast<float4*>(Yt + (o + lane) * LDS + o + r) = make_float4(y[r], y[r + 1], y[r + 2], y[r + 3]);
-#pragma unroll
-            for (int r = 0; r < SB; ++r) Lr[r * LDI + lane] = y[r];
-        } else if (t - 32 < below) {
-            const int r = o + SB + (t - 32);
-            float x[SB];
-#pragma unroll
-            for (int k = 0; k < SB; k += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(S + r * LDS + o + k);
-                x[k] = v.x; x[k + 1] = v.y; x[k + 2] = v.z; x[k + 3] = v.w;
-            }
-            Trsm32<0>::run(x, S + o * LDS + o, invd + o);
-#pragma unroll
-            for (int k = 0; k < SB; k += 4)
-                *reinterpret_cast<float4*>(S + r * LDS + o + k) = make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
-        }
-        __syncthreads();
-
-        // ---- C: trailing update of the factorization || inverse solve of step kb
+        // ---- C: trailing update of block column kb+1 || inverse solve of step kb
         {
             // only block column kb+1 here (what step kb+1 needs first); the rest of
-            // this step's update runs beside step kb+1's Cholesky
+            // this step's update runs beside step kb+1's panel
             const int nrest = NB / SB - kb - 1;            // sub-block rows after kb
             const int pair_warps = 2 * nrest;              // two warps per pair (bi, kb+1)
             if (warp < pair_warps) {
@@ -432,20 +463,24 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
         __syncthreads();
     }
 
-    // Z's diagonal block = Yt (rows); Dinv = Yt^T, transposed into the factor's
-    // (now free) buffer with an odd row stride -- conflict-free on both sides --
-    // and written out row by row
-    float* D = S;   // [NB][LDD]
-    for (int idx = t; idx < NB * NB; idx += DIAG_THREADS) {
-        const int c = idx / NB, r = idx % NB;
-        const float v = Yt[c * LDS + r];
-        Z[size_t(k0 + c) * d + k0 + r] = v;
-        D[r * LDD + c] = v;
+    // Z's diagonal block = Yt, as float4 rows; Dinv = Yt^T, gathered four
+    // columns at a time into the factor's (now free) buffer -- column reads
+    // and float4 writes both free of bank conflicts -- and written out as
+    // float4 rows.
+    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
+        const int c = idx / (NB / 4), r4 = (idx % (NB / 4)) * 4;
+        *reinterpret_cast<float4*>(Z + size_t(k0 + c) * d + k0 + r4) = *reinterpret_cast<const float4*>(Yt + c * LDS + r4);
+    }
+    float* D = S;   // [NB][LDS]
+    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
+        const int r = idx % NB, c4 = (idx / NB) * 4;
+        *reinterpret_cast<float4*>(D + r * LDS + c4) =
+            make_float4(Yt[c4 * LDS + r], Yt[(c4 + 1) * LDS + r], Yt[(c4 + 2) * LDS + r], Yt[(c4 + 3) * LDS + r]);
     }
     __syncthreads();
-    for (int idx = t; idx < NB * NB; idx += DIAG_THREADS) {
-        const int r = idx / NB, c = idx % NB;
-        Dinv[idx] = D[r * LDD + c];
+    for (int idx = t; idx < NB * NB / 4; idx += DIAG_THREADS) {
+        const int r = idx / (NB / 4), c4 = (idx % (NB / 4)) * 4;
+        *reinterpret_cast<float4*>(Dinv + size_t(r) * NB + c4) = *reinterpret_cast<const float4*>(D + r * LDS + c4);
     }
 }
 

@@ -23,10 +23,12 @@
 //    issues TMA, one thread of CTA 0 issues the MMAs.
 //  - Promotion: the tensor core's fp32 accumulation loses about half an ulp
 //    per accumulation step (measured: relative error ~4e-5 over a chain of
-//    16384 rows).  So the K loop is cut into chunks of 512 rows, each summed
+//    16384 rows).  So the K loop is cut into chunks of 1024 rows, each summed
 //    into one of two TMEM buffers (2 x 256 columns) while eight epilogue warps
 //    per CTA drain the other buffer and add it into fp32 registers (round to
-//    nearest); at the end they add 2 * sum into H.
+//    nearest); at the end they add 2 * sum into H.  Measured relative error
+//    of H over 65536 bench rows: 6.5e-7 with 512-row chunks, 1.4e-6 with
+//    1024, 3.3e-6 with 2048; 1024 rows take 2.4% less time than 512.
 //  - fp32 inputs are split into three bf16 terms by `split3_kernel`; the
 //    contraction then runs over the six leading cross products
 //    (hh, hm, mh, mm, hl, lh), which the K loop walks one after another.
@@ -47,7 +49,7 @@ namespace hess {
 #define GPTQ_HESS_BK 128
 #endif
 #ifndef GPTQ_HESS_PROMOTE_ROWS
-#define GPTQ_HESS_PROMOTE_ROWS 512
+#define GPTQ_HESS_PROMOTE_ROWS 1024
 #endif
 constexpr int BK = GPTQ_HESS_BK;            // calibration rows per stage
 constexpr int CHUNK = GPTQ_HESS_PROMOTE_ROWS / BK;   // k-steps (of BK rows) summed in TMEM before promotion
