@@ -131,11 +131,13 @@ __global__ void __launch_bounds__(256)
 //      trail it group by group: warp w in 1 .. 3-kb solves rows o + 32 w +
 //      lane of the panel below against L_kk^T, and warp YW builds column
 //      `lane` of L_kk^-1 (forward substitution on e_lane).  Meanwhile the
-//      other warps (not those sharing the leader's scheduler) finish step
-//      kb-1: its trailing update beyond block column kb and its step of the
-//      inverse's update.
-//   C: the trailing update of block column kb+1 (what step kb+1 needs first)
-//      and step kb of the inverse's block solve.
+//      other warps (not those sharing the leader's scheduler) apply step
+//      kb-1's update to block column kb+1 and to the inverse's rows of
+//      block kb.
+//   C: step kb's update of block column kb+1 (what step kb+1 needs first),
+//      step kb of the inverse's block solve, and the rest of step kb-1's
+//      updates (the blocks that phase A of step kb+1 does not read).
+// Every block receives its updates in the same order on every run.
 // The inverse Y = L^-1 is built right-looking on the identity (Y = X after
 //   X_k <- L_kk^-1 X_k;  X_i -= L_ik X_k  (i > k)  for k = 0..3)
 // and kept transposed (Yt = Y^T = L^-T) so that every product reads both of
@@ -147,7 +149,8 @@ constexpr int LDS = NB + 4;              // S and Yt row stride (floats)
 constexpr int LDI = SB + 4;              // Lr and Lp row stride
 constexpr int DIAG_THREADS = 384;        // 12 warps
 constexpr int YW = 5;                    // the follower that builds L_kk^-1 (not on the leader's scheduler)
-constexpr size_t DIAG_SMEM = (size_t(2) * NB * LDS + size_t(2) * SB * LDI + SB) * sizeof(float);
+static_assert(NB / SB == 4, "the diagonal kernel's task lists are written for 4 x 4 sub-blocks");
+constexpr size_t DIAG_SMEM = (size_t(2) * NB * LDS + size_t(2) * SB * LDI + 2 * SB) * sizeof(float);
 
 // The leader's columns are published in groups of GROUP steps; group g of
 // sub-block kb completes mbarrier 4 kb + g (each used once, so every wait is
@@ -164,14 +167,15 @@ constexpr int NGROUPS = (NB / SB) * (SB / GROUP);
 // is subtracted from every a[j], j > C.  The next pivot comes from lane C+1's
 // own l by a shuffle, beside the shared-memory round trip.  After every
 // GROUP steps lane 0 arrives on the group's barrier (release: the warp's
-// published columns become visible to the followers' waits).
+// published columns become visible to the followers' waits).  The pivots go
+// to shared memory and are tested after the last step: tested inside the
+// chain, they cost a third of its time.
 template <int C>
 struct LeadStep {
     __device__ __forceinline__ static void run(float (&a)[SB], float piv, int lane, float* __restrict__ Lp,
-                                               float* __restrict__ rs_out, uint64_t* grp, uint32_t& bad,
-                                               uint32_t& nonfinite) {
-        bad |= uint32_t(!(piv > 0.0f && isfinite(piv))) << C;   // bit C: pivot C failed
-        nonfinite |= uint32_t(!isfinite(piv)) << C;
+                                               float* __restrict__ rs_out, float* __restrict__ piv_out,
+                                               uint64_t* grp) {
+        piv_out[C] = piv;   // checked once after the last step, off the chain
         const float rs = rsqrtf(piv);
         const float l = a[C] * rs;
         a[C] = l;
@@ -192,7 +196,7 @@ struct LeadStep {
                 for (int q = 0; q < 4; ++q)
                     if (j4 + q > C) a[j4 + q] = fmaf(-l, v[q], a[j4 + q]);
             }
-            LeadStep<C + 1>::run(a, next, lane, Lp, rs_out, grp, bad, nonfinite);
+            LeadStep<C + 1>::run(a, next, lane, Lp, rs_out, piv_out, grp);
         } else {
             __syncwarp();
             if (lane == 0) mbar_arrive(grp + SB / GROUP - 1);
@@ -271,7 +275,8 @@ __device__ __forceinline__ void sub_block_update(const float* __restrict__ P, co
 // of line, like the followers, so that its registers are allocated on their
 // own, away from the rest of the kernel.
 __device__ __noinline__ void lead_warp(const float* __restrict__ S, float* __restrict__ Lp, float* __restrict__ rs,
-                                       uint64_t* grp, int o, int lane, uint32_t* badmask, uint32_t* nonfinite) {
+                                       float* __restrict__ pv, uint64_t* grp, int o, int lane, uint32_t* badmask,
+                                       uint32_t* nonfinite) {
     float a[SB];
     const float* arow = S + (o + lane) * LDS + o;
 #pragma unroll
@@ -279,10 +284,11 @@ __device__ __noinline__ void lead_warp(const float* __restrict__ S, float* __res
         const float4 v = *reinterpret_cast<const float4*>(arow + j);
         a[j] = v.x; a[j + 1] = v.y; a[j + 2] = v.z; a[j + 3] = v.w;
     }
-    uint32_t bad = 0, nf = 0;
-    LeadStep<0>::run(a, __shfl_sync(0xffffffffu, a[0], 0), lane, Lp, rs, grp, bad, nf);
-    *badmask = bad;
-    *nonfinite = nf;
+    LeadStep<0>::run(a, __shfl_sync(0xffffffffu, a[0], 0), lane, Lp, rs, pv, grp);
+    __syncwarp();
+    const float piv = pv[lane];   // bit c: pivot c failed
+    *badmask = __ballot_sync(0xffffffffu, !(piv > 0.0f && isfinite(piv)));
+    *nonfinite = __ballot_sync(0xffffffffu, !isfinite(piv));
 }
 
 // Phase A of step kb for a follower: row_group = w >= 1 solves rows
@@ -334,6 +340,7 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
     float* Lr = Yt + NB * LDS;         // [SB][LDI] L_kk^-1 of the current step, row-major
     float* Lp = Lr + SB * LDI;         // [SB][LDI] the leader's published columns: Lp[c][j] = L_kk[j][c]
     float* rs = Lp + SB * LDI;         // [SB] 1 / L_kk[c][c]
+    float* pv = rs + SB;               // [SB] the pivots L_kk[c][c]^2, for the positivity test
     __shared__ int failed;
     __shared__ __align__(8) uint64_t grp_bar[NGROUPS];   // the leader's column groups, one barrier per group
     pdl_wait();
@@ -378,7 +385,7 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
         // ---- A: Cholesky (leader) || panel solve and L_kk^-1 (followers) || rest of step kb-1
         if (warp == 0) {
             uint32_t badmask = 0, nonfinite = 0;   // the same in every lane
-            lead_warp(S, Lp, rs, grp_bar + kb * (SB / GROUP), o, lane, &badmask, &nonfinite);
+            lead_warp(S, Lp, rs, pv, grp_bar + kb * (SB / GROUP), o, lane, &badmask, &nonfinite);
             if (badmask != 0 && lane == 0) {   // the first failing pivot of this sub-block
                 const int bad = __ffs(int(badmask)) - 1;
                 failed = 1;
@@ -389,48 +396,43 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
             if (!follow_warp(S, Yt, Lr, Lp, rs, grp_bar + kb * (SB / GROUP), o, warp == YW ? 0 : warp, lane, st))
                 failed = 1;
         } else if (kb > 0 && (warp & 3) != 0) {
-            // Work of step kb-1 that step kb's panel does not wait for, on the
-            // warps other than YW that do not share the leader's scheduler:
-            //  - the trailing update of step kb-1 beyond block column kb:
-            //    pairs (bi, bj), kb < bj <= bi;
-            //  - X_ij -= L_{i,kb-1} Y_{kb-1,j} for i >= kb, j < kb, transposed:
-            //    Yt[j-block][i-block] -= Yt[j-block][(kb-1)-block] S[i-block][(kb-1)-block]^T.
+            // What step kb's phase C needs of step kb-1, on the warps other than YW
+            // that do not share the leader's scheduler, in halves of 32 x 32
+            // sub-blocks (P = block column kb-1 of L):
+            //  - block column kb+1: S[bi][kb+1] -= L_{bi,kb-1} L_{kb+1,kb-1}^T, bi > kb;
+            //  - X_{kb,j} -= L_{kb,kb-1} Y_{kb-1,j} for j < kb, transposed:
+            //    Yt[j-block][kb-block] -= Yt[j-block][(kb-1)-block] S[kb-block][(kb-1)-block]^T.
             const int w = warp - npanel - (warp > 4) - (warp > YW) - (warp > 8);
             const int nw = DIAG_THREADS / 32 - npanel - 3;
-            const int nf = NB / SB - kb - 1;                   // sub-block columns after kb
-            const int far_tasks = nf * (nf + 1);               // two per pair
-            const int nj = kb, ni = NB / SB - kb;
-            const int tasks = far_tasks + 2 * ni * nj;
+            const int ncol = 2 * (NB / SB - kb - 1);
+            const int tasks = ncol + 2 * kb;
             const int po = (kb - 1) * SB;
             for (int task = w; task < tasks; task += nw) {
-                if (task < far_tasks) {
-                    int p = task >> 1, bi = kb + 1;
-                    while (p > bi - (kb + 1)) { p -= bi - kb; ++bi; }
-                    const int bj = kb + 1 + p;
-                    sub_block_update(S + po, S + po, S, bi * SB, bj * SB, task & 1, lane);
+                if (task < ncol) {
+                    const int bi = kb + 1 + (task >> 1);
+                    sub_block_update(S + po, S + po, S, bi * SB, (kb + 1) * SB, task & 1, lane);
                 } else {
-                    const int blk = (task - far_tasks) >> 1, sh = (task - far_tasks) & 1;
-                    const int j = blk % nj, i = kb + blk / nj;
-                    sub_block_update(Yt + po, S + po, Yt, j * SB, i * SB, sh, lane);
+                    const int j = (task - ncol) >> 1;
+                    sub_block_update(Yt + po, S + po, Yt, j * SB, kb * SB, (task - ncol) & 1, lane);
                 }
             }
         }
         __syncthreads();
         if (failed) return;
 
-        // ---- C: trailing update of block column kb+1 || inverse solve of step kb
+        // ---- C: step kb's update of block column kb+1 (what step kb+1 needs first)
+        //      || step kb of the inverse's block solve || the rest of step kb-1
         {
-            // only block column kb+1 here (what step kb+1 needs first); the rest of
-            // this step's update runs beside step kb+1's panel
-            const int nrest = NB / SB - kb - 1;            // sub-block rows after kb
-            const int pair_warps = 2 * nrest;              // two warps per pair (bi, kb+1)
-            if (warp < pair_warps) {
+            const int n3 = 2 * (NB / SB - kb - 1);     // lookahead: two warps per pair (bi, kb+1)
+            const int n5 = kb == 1 ? 2 : 0;            // step kb-1 beyond column kb+1: pair (3, 3), only for kb = 1
+            const int n6 = kb >= 1 ? 2 * kb * (NB / SB - kb - 1) : 0;   // X_{i,j}, i > kb, j < kb, of step kb-1
+            if (warp < n3) {
                 const int bi = kb + 1 + (warp >> 1);
                 sub_block_update(S + o, S + o, S, bi * SB, (kb + 1) * SB, warp & 1, lane);
-            } else if (warp < pair_warps + kb) {
+            } else if (warp < n3 + kb) {
                 // Y_{kb,j} = L_kk^-1 X_{kb,j} for j < kb: thread = column c of block j,
                 // reading X_{kb,j}[., c] as row (j*SB + c) of Yt
-                const int u = t - 32 * pair_warps;             // 0 .. 32 kb - 1
+                const int u = t - 32 * n3;                     // 0 .. 32 kb - 1
                 float* row = Yt + (size_t(u)) * LDS + o;       // j = u / SB, c = u % SB: row j*SB + c = u
                 float x[SB];
 #pragma unroll
@@ -457,6 +459,16 @@ __global__ void __launch_bounds__(DIAG_THREADS, 1)
                         y4[q] = acc;
                     }
                     *reinterpret_cast<float4*>(row + r) = make_float4(y4[0], y4[1], y4[2], y4[3]);
+                }
+            } else if (warp < n3 + kb + n5 + n6) {
+                const int task = warp - n3 - kb, po = (kb - 1) * SB;
+                if (task < n5) {
+                    // S[3][3] -= L_{3,0} L_{3,0}^T (step 0 beyond column 2)
+                    sub_block_update(S + po, S + po, S, 3 * SB, 3 * SB, task & 1, lane);
+                } else {
+                    // Yt[j-block][i-block] -= Yt[j-block][(kb-1)-block] S[i-block][(kb-1)-block]^T
+                    const int blk = (task - n5) >> 1, j = blk % kb, i = kb + 1 + blk / kb;
+                    sub_block_update(Yt + po, S + po, Yt, j * SB, i * SB, (task - n5) & 1, lane);
                 }
             }
         }
