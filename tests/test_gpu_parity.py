@@ -237,6 +237,26 @@ def test_prepare_hinv_not_positive_definite():
     assert torch.isnan(Ut).all()
 
 
+@pytest.mark.parametrize("c0", [197, 255, 300])
+def test_prepare_hinv_not_positive_definite_inside(c0):
+    """H = I except one diagonal entry of -1.  The factorization works on the
+    index-reversed matrix, so its pivot c0 (H's index d-1-c0) is the first to
+    fail: -1 + lambda < 0.  c0 = 197 and 255 fall inside the second diagonal
+    block (sub-blocks 2 and 3, the last row of a sub-block for 255), 300 in the
+    third.  info and the status detail are c0 + 1, and U is all NaN."""
+    d = 384
+    H = np.eye(d, dtype=np.float32)
+    H[d - 1 - c0, d - 1 - c0] = -1.0
+    Ut = torch.empty((d, d), dtype=torch.float32, device="cuda")
+    info = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    ws = api.workspace(api.prepare_hinv_workspace_size(d), "cuda")
+    api.prepare_hinv(torch.from_numpy(H).cuda(), Ut, ws, 0.01, info)
+    code, detail = api.get_status(raise_on_error=False)
+    assert code == 3 and detail == c0 + 1
+    assert int(info.item()) == c0 + 1
+    assert torch.isnan(Ut).all()
+
+
 def test_prepare_hinv_nonfinite():
     d = 128
     H = np.eye(d, dtype=np.float32)
